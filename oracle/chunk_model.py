@@ -1,0 +1,96 @@
+"""fp64 chunk-by-chunk (WY/UT) model of the KDA operator.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
+
+The wiki page "Kimi Linear 高效注意力架构", section "Kimi Delta Attention (KDA)",
+says the operator has a hardware-efficient chunkwise form (its "硬件高效分块算法"
+bullet) and gives its cost terms T d_k d_v + T C d_h + T C^2 (comparison table,
+row "时间复杂度"); it does not print the chunk equations.  The rewrite below is
+derived here from the state-update equation alone and is exact in real
+arithmetic; ``tests/test_oracle_pins.py`` pins it to the token recurrence.
+
+Within one chunk of L <= C tokens that starts from state S (rows r, i = tokens):
+
+  g_r     = sum_{j <= r} log alpha_j          (inclusive, per key channel)
+  u_r     = beta_r (v_r - S_{r-1}^T Diag(alpha_r) k_r)   so that
+  S_r     = Diag(alpha_r) S_{r-1} + k_r u_r^T            (state-update equation)
+  A_{ri}  = beta_r <k_r * exp(g_r - g_i), k_i>    for i < r, else 0
+  T       = (I + A)^{-1} Diag(beta)                       (unit lower triangular)
+  U       = T V - T (K * exp(g)) S                        (rows u_r)
+  P_{ri}  = <q_r * exp(g_r - g_i), k_i>          for i <= r, else 0
+  O       = (Q * exp(g)) S + P U                          (rows o_r = S_r^T q_r)
+  S_next  = Diag(exp(g_L)) S + (K * exp(g_L - g))^T U
+
+Every exponent is formed as a difference before exp, so nothing overflows; the
+chunk model is slow on purpose and only runs on small inputs.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def chunk_stages(q, k, v, log_alpha, beta):
+    """S-independent quantities of one chunk (fp64).
+
+    q, k, log_alpha: [L, d_k]; v: [L, d_v]; beta: [L].
+    Returns dict with g, A, T, P, Kg (= K*exp(g)), Qg (= Q*exp(g)),
+    Khat (= K*exp(g_L - g)), Gamma (= exp(g_L)), Ut (= T V), W (= T Kg).
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    la = np.asarray(log_alpha, np.float64)
+    b = np.asarray(beta, np.float64)
+    L = q.shape[0]
+    g = np.cumsum(la, axis=0)
+    # decay between token i and a later token r, per channel: exp(g_r - g_i)
+    diff = np.exp(g[:, None, :] - g[None, :, :])            # [L, L, d_k]
+    kk = np.einsum("rc,ic,ric->ri", k, k, diff)
+    qk = np.einsum("rc,ic,ric->ri", q, k, diff)
+    strict = np.tril(np.ones((L, L)), -1)
+    incl = np.tril(np.ones((L, L)), 0)
+    A = b[:, None] * kk * strict
+    T = np.linalg.solve(np.eye(L) + A, np.diag(b))
+    P = qk * incl
+    Kg = k * np.exp(g)
+    Qg = q * np.exp(g)
+    Khat = k * np.exp(g[-1][None, :] - g)
+    return dict(g=g, A=A, T=T, P=P, Kg=Kg, Qg=Qg, Khat=Khat, Gamma=np.exp(g[-1]),
+                Ut=T @ v, W=T @ Kg)
+
+
+def chunk_step(st, S):
+    """Apply one chunk to state S [d_k, d_v]; return (O [L, d_v], S_next, U)."""
+    U = st["Ut"] - st["W"] @ S
+    O = st["Qg"] @ S + st["P"] @ U
+    S_next = st["Gamma"][:, None] * S + st["Khat"].T @ U
+    return O, S_next, U
+
+
+def prefill(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk: int = 64):
+    """Chunked fp64 prefill over a packed batch; same shapes as ``oracle.prefill``.
+
+    Chunks start at each sequence's first token and never cross a boundary; the
+    last chunk of a sequence may be shorter than ``chunk``.
+    """
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    la = np.asarray(log_alpha, np.float64)
+    b = np.asarray(beta, np.float64)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    cu = np.asarray(cu_seqlens, np.int64)
+    N = cu.shape[0] - 1
+    o = np.zeros((T, H, dv))
+    S_out = np.zeros((N, H, dk, dv))
+    for n in range(N):
+        for h in range(H):
+            S = np.zeros((dk, dv)) if S0 is None else np.array(S0[n, h], np.float64)
+            for s in range(int(cu[n]), int(cu[n + 1]), chunk):
+                e = min(s + chunk, int(cu[n + 1]))
+                st = chunk_stages(q[s:e, h], k[s:e, h], v[s:e, h], la[s:e, h], b[s:e, h])
+                O, S, _ = chunk_step(st, S)
+                o[s:e, h] = O
+            S_out[n, h] = S
+    return o, S_out
