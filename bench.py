@@ -1,0 +1,396 @@
+"""Benchmark of the B200 KDA operator: prefill tokens/s (headline) and decode us/step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one ``kda_prefill`` call over the whole workload (every sequence and
+head), inputs resident in HBM.  The default workload is ``batched_prefill``
+(8 sequences x 8192 tokens, H = 32, d_k = d_v = 128, bf16 q/k/v, fp32 gates and
+state).  The decode workload (256 sequences x 32 heads, 64 consecutive steps) is
+timed in the same run and reported under ``decode``.
+
+With N > 1 (one process per GPU under torchrun) every rank runs its own copy of
+the workload (the operator's (sequence, head) units are independent, so there is
+no collective on the data path): weak scaling, value = all ranks' tokens / max
+rank time.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this operator
+has) on the host cores over a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from gated_delta_rule_126_b200 import inputs  # noqa: E402
+
+METRIC = "KDA prefill tokens/s & decode µs/step (H=32,d=128) on 1 B200; % of roofline"
+UNIT = "tokens/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# Algorithmic work per head-token of prefill at chunk C = 64, d = 128, and per
+# head-step of decode (derivation in the design notes):
+#   flops = 5*C*d + 6*d^2 (causal C x C products at half, three state products);
+#   bytes = q,k,v bf16 + log alpha f32 + beta f32 + o bf16.
+def prefill_flops_per_head_token(C, d):
+    return 5 * C * d + 6 * d * d
+
+
+def prefill_bytes_per_head_token(dk, dv, qkv_bytes):
+    return (2 * dk + dv) * qkv_bytes + 4 * dk + 4 + dv * qkv_bytes
+
+
+def decode_bytes_per_head_step(dk, dv, qkv_bytes):
+    return 2 * 4 * dk * dv + prefill_bytes_per_head_token(dk, dv, qkv_bytes)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *exc):
+        time.sleep(0.2)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[2:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def time_region(fn, steps, stream):
+    """Device time of ``steps`` calls of fn, CUDA events on the launching stream."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / 1e3
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+def oracle_sample(w, budget_head_tokens, seed_device="cpu"):
+    """Time the fp64 oracle on a bounded sample of workload w (host cores).
+
+    The sample is whole sequences of the workload's packing, in order, on all H
+    heads, until ``budget_head_tokens`` head-tokens are covered; a sequence longer
+    than a sixteenth of the budget is skipped, so the sample holds at least 16
+    (sequence, head) units to spread over the worker threads.  Inputs are drawn with the same recipe on the CPU.
+    Returns (tokens/s, cores, description, seconds); a token counts all H heads.
+    """
+    import oracle
+    H = w.H
+    chosen, tok = [], 0
+    for L in w.seqlens:
+        if L > max(budget_head_tokens // 16, 1):
+            continue
+        if tok + L * H > budget_head_tokens and chosen:
+            break
+        chosen.append(L)
+        tok += L * H
+    if not chosen:  # every sequence is long: take a prefix of the first one
+        chosen = [max(1, budget_head_tokens // H)]
+    inp = inputs.prefill_inputs(chosen, H, w.dk, w.dv, w.dtype, w.s0_std, w.seed,
+                                device=seed_device)
+    f64 = lambda t: t.to(torch.float64).numpy()
+    cores = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.prefill(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), f64(inp["log_alpha"]),
+                   f64(inp["beta"]), inp["cu_seqlens_host"],
+                   S0=None if inp["S0"] is None else f64(inp["S0"]), nthreads=cores)
+    dt = time.perf_counter() - t0
+    value = sum(chosen) / dt
+    sample = (f"{len(chosen)} sequence(s) ({min(chosen)}..{max(chosen)} tokens) x {H} heads "
+              f"= {sum(chosen) * H} head-tokens, fp64 oracle, {dt:.1f} s on {cores} threads")
+    return value, cores, sample, dt
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = inputs.WORKLOADS[args.workload]
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, cores, sample, _ = oracle_sample(w, args.ref_head_tokens)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "total_tokens": w.total_tokens, "H": w.H,
+                       "d_k": w.dk, "d_v": w.dv, "chunk": w.chunk},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    from gated_delta_rule_126_b200 import kda_decode_step, kda_prefill, prefill_workspace_size
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    peaks, peak_kind = load_peaks()
+    w = inputs.WORKLOADS[args.workload]
+    assert w.kind == "prefill"
+    inp = inputs.prefill_inputs(w.seqlens, w.H, w.dk, w.dv, w.dtype, w.s0_std,
+                                w.seed + 1000 * rank, device=dev)
+    T, N = w.total_tokens, len(w.seqlens)
+    o = torch.empty(T, w.H, w.dv, dtype=inp["q"].dtype, device=dev)
+    S_final = torch.empty(N, w.H, w.dk, w.dv, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(256, prefill_workspace_size(N, T, w.H, w.dk, w.dv, w.chunk,
+                                                     inp["q"].dtype)),
+                     dtype=torch.uint8, device=dev)
+    cu_host = inp["cu_seqlens_host"]
+
+    def step():
+        kda_prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                    inp["cu_seqlens"], cu_host, S0=inp["S0"], chunk=w.chunk, o=o,
+                    S_final=S_final, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    barrier(world)
+    with ClockSampler(local) as clk:
+        elapsed = time_region(step, args.steps, stream)
+    barrier(world)
+    elapsed = max_over_ranks(elapsed, world)
+    ms = elapsed / args.steps * 1e3
+    value = world * T * args.steps / elapsed
+
+    # roofline of the prefill kernel (one launch per step; events above bracket the
+    # call, which also holds a one-thread-block ordering kernel of a few microseconds)
+    qkv_bytes = inp["q"].element_size()
+    head_tokens = T * w.H
+    alg_bytes = head_tokens * prefill_bytes_per_head_token(w.dk, w.dv, qkv_bytes)
+    alg_bytes += N * w.H * w.dk * w.dv * 4 * (2 if inp["S0"] is not None else 1)
+    alg_flops = head_tokens * prefill_flops_per_head_token(w.chunk, w.dk)
+    t_launch = elapsed / args.steps
+    hbm_peak = peaks["hbm_gbs"]
+    tc_peak = peaks["bf16_tflops"]
+    achieved_gbs = alg_bytes / t_launch / 1e9
+    achieved_tf = alg_flops / t_launch / 1e12
+    t_roof = max(alg_bytes / (hbm_peak * 1e9), alg_flops / (tc_peak * 1e12))
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved_gbs / hbm_peak, "traffic": None,
+                "peak_source": f"{peak_kind} hbm_gbs (copy, burst)",
+                "alg_bytes_per_launch": alg_bytes, "alg_flops_per_launch": alg_flops,
+                "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
+                           "frac": achieved_tf / tc_peak,
+                           "peak_source": f"{peak_kind} bf16_tflops (burst)"},
+                "frac_of_max_bound": t_roof / t_launch}
+
+    # end to end through the public API: pinned host inputs -> device -> kda_prefill ->
+    # host outputs, every step
+    e2e = None
+    if not args.no_e2e:
+        names = ["q", "k", "v", "log_alpha", "beta"]
+        host = {n: inp[n].cpu().pin_memory() for n in names}
+        h_s0 = inp["S0"].cpu().pin_memory() if inp["S0"] is not None else None
+        h_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        h_S = torch.empty(S_final.shape, dtype=S_final.dtype, pin_memory=True)
+        dbuf = {n: torch.empty_like(inp[n]) for n in names}
+        d_s0 = torch.empty_like(inp["S0"]) if inp["S0"] is not None else None
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        h2d += 0 if h_s0 is None else h_s0.numel() * 4
+        h2d += len(cu_host) * 4
+        d2h = h_o.numel() * h_o.element_size() + h_S.numel() * 4
+        cu_pinned = torch.tensor(cu_host, dtype=torch.int32).pin_memory()
+        d_cu = torch.empty_like(inp["cu_seqlens"])
+
+        def e2e_step():
+            for n in names:
+                dbuf[n].copy_(host[n], non_blocking=True)
+            if d_s0 is not None:
+                d_s0.copy_(h_s0, non_blocking=True)
+            d_cu.copy_(cu_pinned, non_blocking=True)
+            kda_prefill(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["log_alpha"], dbuf["beta"],
+                        d_cu, cu_host, S0=d_s0, chunk=w.chunk, o=o, S_final=S_final,
+                        workspace=ws, stream=stream)
+            h_o.copy_(o, non_blocking=True)
+            h_S.copy_(S_final, non_blocking=True)
+
+        e2e_step()
+        barrier(world)
+        e_steps = max(1, min(args.steps, 5))
+        e_el = max_over_ranks(time_region(e2e_step, e_steps, stream), world)
+        e2e = {"value": world * T * e_steps / e_el, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": e_steps}
+        del host, dbuf, h_o, h_S
+
+    # decode: 256 sequences x 32 heads, 64 consecutive one-token steps
+    decode = None
+    if not args.no_decode:
+        dw = inputs.WORKLOADS["decode"]
+        dinp = inputs.workload_inputs(dw, device=dev)
+        S = dinp["S0"].clone()
+        od = torch.empty(dw.batch, dw.H, dw.dv, dtype=dinp["q"].dtype, device=dev)
+
+        def dstep_all():
+            for t in range(dw.steps):
+                kda_decode_step(dinp["q"][t], dinp["k"][t], dinp["v"][t], dinp["log_alpha"][t],
+                                dinp["beta"][t], S, o=od, stream=stream)
+
+        dstep_all()
+        barrier(world)
+        d_el = max_over_ranks(time_region(dstep_all, 3, stream), world)
+        us = d_el / (3 * dw.steps) * 1e6
+        dbytes = dw.batch * dw.H * decode_bytes_per_head_step(dw.dk, dw.dv, 2)
+        gbs = dbytes / (us * 1e-6) / 1e9
+        decode = {"workload": dw.name, "us_per_step": us, "batch": dw.batch, "H": dw.H,
+                  "steps_per_sequence": dw.steps,
+                  "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
+                               "frac": gbs / hbm_peak, "traffic": None,
+                               "alg_bytes_per_launch": dbytes,
+                               "peak_source": f"{peak_kind} hbm_gbs (copy, burst)"},
+                  "gpu_launches_per_step": 1}
+        del dinp, S
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, sample, _ = oracle_sample(inputs.WORKLOADS[args.workload], args.ref_head_tokens)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": w.name, "num_seqs": N, "seq_lens": "x".join(
+                    str(x) for x in sorted(set(w.seqlens))) if N < 10 else f"{N} varlen",
+                    "total_tokens_per_gpu": T, "H": w.H, "d_k": w.dk, "d_v": w.dv,
+                    "chunk": w.chunk, "state": "fp32", "gates": "fp32",
+                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                    "l2": "inputs larger than L2 (no flush)"},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": 2 * args.steps, "clocks": clk.summary(), "decode": decode}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="batched_prefill",
+                    choices=[k for k, v in inputs.WORKLOADS.items() if v.kind == "prefill"])
+    ap.add_argument("--ref-head-tokens", type=int, default=1 << 20,
+                    help="size of the oracle's timed sample in head-tokens")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,1 +1,19 @@
-"""B200-native Kimi Delta Attention (KDA) operator: package root (filled in below)."""
+"""B200-native Kimi Delta Attention (KDA) operator.
+
+The operator runs in hand-written sm_100a CUDA kernels behind the C ABI declared
+in ``include/kda.h`` (library ``lib/libkda_b200.so``, built by
+``python -m gated_delta_rule_126_b200.build``).  This package is the thin Python
+binding over that ABI, with the same names:
+
+* ``kda_prefill``     -- chunked prefill over packed variable-length sequences;
+* ``kda_decode_step`` -- one recurrent decode step for a batch of sequences;
+* ``prefill_workspace_size``, ``workspace_status``, ``KdaError``.
+
+``inputs`` holds the seeded synthetic input generators.  Importing the package
+does not load the CUDA library; the first call does, and raises if it is missing.
+"""
+from ._binding import (KdaError, kda_decode_step, kda_prefill, load, prefill_workspace_size,
+                       workspace_status)
+
+__all__ = ["KdaError", "kda_decode_step", "kda_prefill", "load", "prefill_workspace_size",
+           "workspace_status"]

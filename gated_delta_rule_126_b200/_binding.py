@@ -1,0 +1,184 @@
+"""ctypes binding of ``include/kda.h`` (argument marshalling only).
+
+Every step of the operator runs in the CUDA library ``lib/libkda_b200.so``; this
+module only turns torch tensors into pointers and sizes, allocates outputs with
+torch when the caller does not pass them, and raises on a non-OK status.  There is
+no CPU fallback: if the library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libkda_b200.so")
+
+KDA_OK = 0
+STATUS_NAMES = {0: "KDA_OK", 1: "KDA_ERR_INVALID_ARG", 2: "KDA_ERR_UNSUPPORTED",
+                3: "KDA_ERR_WORKSPACE", 4: "KDA_ERR_CUDA", 5: "KDA_ERR_DEVICE_FAULT"}
+DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class KdaError(RuntimeError):
+    """A KDA library call returned a status other than KDA_OK."""
+
+    def __init__(self, status: int, what: str):
+        self.status = int(status)
+        super().__init__(f"{what}: {STATUS_NAMES.get(self.status, self.status)}")
+
+
+def _declare(lib):
+    c = ctypes
+    vp, i32, i64, sz = c.c_void_p, c.c_int, c.c_int64, c.c_size_t
+    lib.kda_status_string.restype = c.c_char_p
+    lib.kda_status_string.argtypes = [i32]
+    lib.kda_version.restype = i32
+    lib.kda_version.argtypes = []
+    lib.kda_prefill_workspace_size.restype = sz
+    lib.kda_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
+    lib.kda_prefill.restype = i32
+    lib.kda_prefill.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                vp, vp, vp, sz, vp]
+    lib.kda_decode_step.restype = i32
+    lib.kda_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, vp]
+    lib.kda_workspace_status.restype = i32
+    lib.kda_workspace_status.argtypes = [vp, vp]
+    return lib
+
+
+def load(path: str = LIB_PATH):
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    f"KDA CUDA library not found at {path}; build it with "
+                    "`python -m gated_delta_rule_126_b200.build`")
+            _lib = _declare(ctypes.CDLL(path))
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != KDA_OK:
+        raise KdaError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def prefill_workspace_size(num_seqs, total_tokens, H, d_k, d_v, chunk=64, dtype=torch.bfloat16):
+    return int(load().kda_prefill_workspace_size(int(num_seqs), int(total_tokens), int(H),
+                                                 int(d_k), int(d_v), int(chunk),
+                                                 DTYPE_CODE[dtype]))
+
+
+def kda_prefill(q, k, v, log_alpha, beta, cu_seqlens, cu_seqlens_host=None, S0=None,
+                chunk=64, o=None, S_final=None, workspace=None, stream=None):
+    """Chunked KDA prefill over packed sequences (see ``kda_prefill`` in kda.h).
+
+    q, k [T,H,d_k], v [T,H,d_v] (float32 or bfloat16), log_alpha [T,H,d_k] f32,
+    beta [T,H] f32, cu_seqlens [N+1] int32 on the device, cu_seqlens_host the same
+    offsets as a list or CPU tensor (copied from the device when omitted, which
+    synchronises), S0 [N,H,d_k,d_v] f32 or None.  Returns ``(o, S_final)``.
+    """
+    lib = load()
+    dev = q.device
+    dt = q.dtype
+    if dt not in DTYPE_CODE:
+        raise ValueError("q/k/v dtype must be float32 or bfloat16")
+    _need(q, "q", dt)
+    T, H, dk = q.shape
+    _need(k, "k", dt, dev)
+    _need(v, "v", dt, dev)
+    dv = v.shape[2]
+    _need(log_alpha, "log_alpha", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu()
+    cu_h = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
+    N = cu_h.numel() - 1
+    if cu_seqlens.numel() != N + 1:
+        raise ValueError("cu_seqlens and cu_seqlens_host differ in length")
+    if o is None:
+        o = torch.empty(T, H, dv, dtype=dt, device=dev)
+    if S_final is None:
+        S_final = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    _need(o, "o", dt, dev)
+    _need(S_final, "S_final", torch.float32, dev)
+    ws_bytes = prefill_workspace_size(N, T, H, dk, dv, chunk, dt)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = lib.kda_prefill(_ptr(q), _ptr(k), _ptr(v), DTYPE_CODE[dt], _ptr(log_alpha),
+                             _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
+                             ctypes.c_void_p(cu_h.data_ptr()), N, H, dk, dv, int(chunk),
+                             _ptr(o), _ptr(S_final), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(),
+                             _stream_handle(stream))
+    _check(st, "kda_prefill")
+    return o, S_final
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, S, o=None, stream=None):
+    """One decode step for B sequences (see ``kda_decode_step`` in kda.h).
+
+    q, k [B,H,d_k], v [B,H,d_v], log_alpha [B,H,d_k] f32, beta [B,H] f32,
+    S [B,H,d_k,d_v] f32 (updated in place).  Returns o [B,H,d_v].
+    """
+    lib = load()
+    dev = q.device
+    dt = q.dtype
+    if dt not in DTYPE_CODE:
+        raise ValueError("q/k/v dtype must be float32 or bfloat16")
+    _need(q, "q", dt)
+    B, H, dk = q.shape
+    _need(k, "k", dt, dev)
+    _need(v, "v", dt, dev)
+    dv = v.shape[2]
+    _need(log_alpha, "log_alpha", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(S, "S", torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=dt, device=dev)
+    _need(o, "o", dt, dev)
+    with torch.cuda.device(dev):
+        st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), DTYPE_CODE[dt], _ptr(log_alpha),
+                                 _ptr(beta), _ptr(S), B, H, dk, dv, _ptr(o),
+                                 _stream_handle(stream))
+    _check(st, "kda_decode_step")
+    return o
+
+
+def workspace_status(workspace, stream=None):
+    """Status flagged by the kernels of the last prefill that used ``workspace``."""
+    return int(load().kda_workspace_status(_ptr(workspace), _stream_handle(stream)))

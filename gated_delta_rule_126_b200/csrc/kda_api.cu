@@ -1,0 +1,123 @@
+// C-ABI entry points of the KDA library: argument checks on the host, then
+// kernel launches on the caller's stream.  See include/kda.h for the contract.
+#include <cstring>
+
+#include "kda_internal.h"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+kda_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+bool dtype_ok(kda_dtype_t t) { return t == KDA_DTYPE_F32 || t == KDA_DTYPE_BF16; }
+
+// Shapes every prefill kernel here accepts.
+kda_status_t check_prefill_shape(int num_seqs, int H, int d_k, int d_v, int chunk, kda_dtype_t dt) {
+    if (num_seqs < 0 || H < 1 || d_k < 1 || d_v < 1 || !dtype_ok(dt)) return KDA_ERR_INVALID_ARG;
+    if (chunk != 16 && chunk != 32 && chunk != 64) return KDA_ERR_UNSUPPORTED;
+    if (d_k > 128 || d_v > 128) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_status_string(kda_status_t s) {
+    switch (s) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+        case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+        case KDA_ERR_DEVICE_FAULT: return "KDA_ERR_DEVICE_FAULT";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+int kda_version(void) { return kVersion; }
+
+size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H, int d_k, int d_v,
+                                  int chunk, kda_dtype_t qkv_dtype) {
+    if (total_tokens < 0 || total_tokens > INT32_MAX) return 0;
+    if (check_prefill_shape(num_seqs, H, d_k, d_v, chunk, qkv_dtype) != KDA_OK) return 0;
+    return kda::workspace_layout(num_seqs).total;
+}
+
+kda_status_t kda_prefill(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                         const float *log_alpha, const float *beta, const float *S0,
+                         const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                         int num_seqs, int H, int d_k, int d_v, int chunk, void *o,
+                         float *S_final, void *workspace, size_t workspace_bytes,
+                         kda_stream_t stream) {
+    const kda_status_t shape = check_prefill_shape(num_seqs, H, d_k, d_v, chunk, qkv_dtype);
+    if (shape != KDA_OK) return shape;
+    if (!cu_seqlens_host || !cu_seqlens_dev || !S_final) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens_host[0] != 0) return KDA_ERR_INVALID_ARG;
+    int max_len = 0;
+    for (int n = 0; n < num_seqs; ++n) {
+        const int64_t len = int64_t(cu_seqlens_host[n + 1]) - cu_seqlens_host[n];
+        if (len < 0) return KDA_ERR_INVALID_ARG;
+        if (len > max_len) max_len = int(len);
+    }
+    const int64_t T = cu_seqlens_host[num_seqs];
+    if (T > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(S_final) || (S0 && !aligned16(S0))) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+                  !aligned16(log_alpha)))
+        return KDA_ERR_INVALID_ARG;
+    const kda::WorkspaceLayout wl = kda::workspace_layout(num_seqs);
+    if (!workspace || workspace_bytes < wl.total) return KDA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_WORKSPACE;
+
+    kda::PrefillArgs a;
+    a.q = q; a.k = k; a.v = v; a.dtype = qkv_dtype;
+    a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0;
+    a.cu_seqlens = cu_seqlens_dev;
+    a.num_seqs = num_seqs; a.H = H; a.dk = d_k; a.dv = d_v; a.chunk = chunk;
+    a.total_tokens = T; a.max_seqlen = max_len;
+    a.o = o; a.S_final = S_final;
+    a.status = static_cast<kda::DeviceStatus *>(workspace);
+    a.order = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + wl.order_offset);
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (num_seqs == 0) return KDA_OK;
+    cudaError_t err = cudaMemsetAsync(a.status, 0, sizeof(kda::DeviceStatus), st);
+    if (err != cudaSuccess) return KDA_ERR_CUDA;
+    err = kda::launch_order_by_length(a, st);
+    if (err != cudaSuccess) return KDA_ERR_CUDA;
+    if (kda::prefill_tc_supported(a)) return from_cuda(kda::launch_prefill_tc(a, st));
+    return from_cuda(kda::launch_prefill_simt(a, st));
+}
+
+kda_status_t kda_decode_step(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                             const float *log_alpha, const float *beta, float *S, int B, int H,
+                             int d_k, int d_v, void *o, kda_stream_t stream) {
+    if (B < 0 || H < 1 || d_k < 1 || d_v < 1 || !dtype_ok(qkv_dtype)) return KDA_ERR_INVALID_ARG;
+    if (d_k > 128 || d_v > 128 || (d_v % 4) != 0) return KDA_ERR_UNSUPPORTED;
+    if (B == 0) return KDA_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(S)) return KDA_ERR_INVALID_ARG;
+    kda::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.dtype = qkv_dtype;
+    a.log_alpha = log_alpha; a.beta = beta; a.S = S;
+    a.B = B; a.H = H; a.dk = d_k; a.dv = d_v; a.o = o;
+    return from_cuda(kda::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kda_status_t kda_workspace_status(const void *workspace, kda_stream_t stream) {
+    if (!workspace) return KDA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return KDA_ERR_CUDA;
+    kda::DeviceStatus h{};
+    if (cudaMemcpy(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (h.flag == 0) return KDA_OK;
+    if (cudaMemset(const_cast<void *>(workspace), 0, sizeof(h)) != cudaSuccess) return KDA_ERR_CUDA;
+    return KDA_ERR_DEVICE_FAULT;
+}
+
+}  // extern "C"

@@ -1,0 +1,150 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention (KDA) operator.
+ *
+ * The operator (wiki page "Kimi Linear 高效注意力架构", section "Kimi Delta
+ * Attention (KDA)", state-update equation): per head a d_k x d_v state
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *
+ * with one decay alpha_t,i in (0, 1] per key channel (same section, channel-wise
+ * decay bullet; passed here as log alpha) and a scalar beta_t; the read-out is
+ * the delta-rule read-out of the post-update state, o_t = S_t^T q_t.  The pages
+ * fix the state at d_k x d_v = 128 x 128 per head (same section, linear
+ * complexity bullet).  q and k are used as given: the L2 normalisation and any
+ * scaling of q belong to the caller (the KDA layer normalises q and k before the
+ * operator, section "模型架构").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor pointers are DEVICE pointers to caller-owned memory, except the
+ *   ones named *_host.  The library never allocates or frees device memory.
+ * - Layouts are dense row-major, tokens packed over sequences:
+ *       q, k       [T_total, H, d_k]   dtype qkv_dtype
+ *       v, o       [T_total, H, d_v]   dtype qkv_dtype
+ *       log_alpha  [T_total, H, d_k]   float32, every value <= 0
+ *       beta       [T_total, H]        float32
+ *       S0/S_final [N, H, d_k, d_v]    float32, d_v contiguous
+ *   q, k, v, o, log_alpha, S0, S_final must be 16-byte aligned.
+ * - Work is queued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *   and runs asynchronously; the call returns once it is queued.
+ * - Argument errors are found on the host before anything is queued; they
+ *   leave all outputs untouched and return KDA_ERR_INVALID_ARG or
+ *   KDA_ERR_UNSUPPORTED.  A failed launch returns KDA_ERR_CUDA.  No call aborts,
+ *   throws, or prints.
+ */
+#ifndef KDA_B200_KDA_H
+#define KDA_B200_KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbols of this header are the library's only exported ones. */
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *kda_stream_t;
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad cu_seqlens, misalignment */
+    KDA_ERR_UNSUPPORTED = 2,   /* legal arguments no kernel here implements */
+    KDA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required */
+    KDA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    KDA_ERR_DEVICE_FAULT = 5   /* a kernel flagged an internal error (see kda_workspace_status) */
+} kda_status_t;
+
+typedef enum {
+    KDA_DTYPE_F32 = 0,   /* float32 q/k/v/o */
+    KDA_DTYPE_BF16 = 1   /* bfloat16 q/k/v/o (state and gates stay float32) */
+} kda_dtype_t;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+KDA_API const char *kda_status_string(kda_status_t status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+KDA_API int kda_version(void);
+
+/*
+ * Bytes of device workspace kda_prefill needs for these sizes.  Depends only on
+ * its arguments; returns 0 for arguments kda_prefill would reject.
+ */
+KDA_API size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H, int d_k,
+                                  int d_v, int chunk, kda_dtype_t qkv_dtype);
+
+/*
+ * kda_prefill -- chunked prefill over packed variable-length sequences.
+ *
+ * Runs the state-update equation over every token of every sequence and head,
+ * starting from S0 (NULL = zero state), writes o_t = S_t^T q_t for every token
+ * and the state after each sequence's last token to S_final.  The work is
+ * organised in chunks of `chunk` tokens (the chunkwise form named in the KDA
+ * section's "硬件高效分块算法" bullet); chunks start at each sequence's first token
+ * and never cross a sequence boundary.  The result does not depend on `chunk`
+ * except through rounding.
+ *
+ *   q, k, v, qkv_dtype   inputs, layouts above
+ *   log_alpha, beta      float32 gates, layouts above
+ *   S0                   float32 initial states or NULL; may alias S_final
+ *   cu_seqlens_dev       int32 [num_seqs + 1] device copy of the offsets
+ *   cu_seqlens_host      int32 [num_seqs + 1] host copy of the same offsets
+ *                        (read during the call only; must equal the device copy)
+ *                        cu_seqlens[0] = 0, non-decreasing; zero-length
+ *                        sequences are allowed and give S_final = S0 (or 0)
+ *   num_seqs, H, d_k, d_v  sizes: num_seqs >= 0, H >= 1, 1 <= d_k, d_v <= 128
+ *   chunk                16, 32 or 64
+ *   o                    [T_total, H, d_v] output, dtype qkv_dtype
+ *   S_final              [num_seqs, H, d_k, d_v] float32 output
+ *   workspace            device scratch of at least
+ *                        kda_prefill_workspace_size(...) bytes, 256-byte aligned;
+ *                        contents on entry are ignored; not to be shared by two
+ *                        calls that may run at the same time
+ *
+ * Supported: any 1 <= d_k, d_v <= 128 (float32 CUDA-core path); the tensor-core
+ * path is taken for bf16 with d_k = d_v = 128 and chunk = 64.  Anything else
+ * returns KDA_ERR_UNSUPPORTED.
+ */
+KDA_API kda_status_t kda_prefill(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                         const float *log_alpha, const float *beta, const float *S0,
+                         const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                         int num_seqs, int H, int d_k, int d_v, int chunk,
+                         void *o, float *S_final, void *workspace, size_t workspace_bytes,
+                         kda_stream_t stream);
+
+/*
+ * kda_decode_step -- one recurrent decode step for B independent sequences.
+ *
+ * For every (b, h): S <- (I - beta k k^T) Diag(alpha) S + beta k v^T in place,
+ * then o = S^T q (the same equation applied to a single token; the fixed-size
+ * state is what makes decode cost independent of context length, section
+ * "效率" of the same page).
+ *
+ *   q, k       [B, H, d_k] qkv_dtype      v, o  [B, H, d_v] qkv_dtype
+ *   log_alpha  [B, H, d_k] float32        beta  [B, H] float32
+ *   S          [B, H, d_k, d_v] float32, read and overwritten in place
+ * Supported: 1 <= d_k <= 128, d_v in {4, 8, ..., 128}.  B = 0 is a no-op.
+ */
+KDA_API kda_status_t kda_decode_step(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                             const float *log_alpha, const float *beta, float *S,
+                             int B, int H, int d_k, int d_v, void *o, kda_stream_t stream);
+
+/*
+ * kda_workspace_status -- waits for `stream`, then reports whether a kernel of
+ * the last kda_prefill call that used `workspace` flagged an internal error
+ * (KDA_ERR_DEVICE_FAULT, e.g. a bounded wait that ran out) and clears the flag.
+ * Returns KDA_OK when none did, KDA_ERR_CUDA when the wait itself failed.
+ */
+KDA_API kda_status_t kda_workspace_status(const void *workspace, kda_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_B200_KDA_H */

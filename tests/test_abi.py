@@ -1,0 +1,116 @@
+"""The C-ABI library loads, exports every symbol kda.h declares, and rejects bad
+arguments on the host (no GPU needed: every check here returns before any CUDA
+call is made)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from gated_delta_rule_126_b200 import _binding, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+INVALID, UNSUPPORTED, WORKSPACE = 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _binding.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"KDA_API\s+[\w\s\*]+?\b(kda_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_abi():
+    assert declared_symbols() == sorted([
+        "kda_decode_step", "kda_prefill", "kda_prefill_workspace_size", "kda_status_string",
+        "kda_version", "kda_workspace_status"])
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    # nothing else is exported from the library's own code
+    out = os.popen(f"nm -D --defined-only {_binding.LIB_PATH}").read()
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln and "kda" in ln}
+    assert exported == set(declared_symbols())
+
+
+def test_status_strings_and_version(lib):
+    for code, name in _binding.STATUS_NAMES.items():
+        assert lib.kda_status_string(code).decode() == name
+    assert lib.kda_status_string(99).decode() == "KDA_ERR_UNKNOWN"
+    assert lib.kda_version() >= 100
+
+
+def test_workspace_size(lib):
+    ws = lib.kda_prefill_workspace_size
+    assert ws(8, 65536, 32, 128, 128, 64, 1) >= 256
+    assert ws(8, 65536, 32, 128, 128, 48, 1) == 0        # unsupported chunk
+    assert ws(8, 65536, 32, 129, 128, 64, 1) == 0        # d_k too large
+    assert ws(-1, 0, 32, 128, 128, 64, 1) == 0
+    assert ws(1, -5, 32, 128, 128, 64, 1) == 0
+    assert ws(1, 1 << 40, 32, 128, 128, 64, 1) == 0      # more tokens than int32 offsets
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: every case fails on the host
+
+
+def _prefill(lib, cu_host, N, H=2, dk=16, dv=16, chunk=16, dtype=0, ptr=FAKE, ws=FAKE,
+             ws_bytes=1 << 20, s0=None, out=FAKE):
+    arr = (ctypes.c_int32 * len(cu_host))(*cu_host) if cu_host is not None else None
+    return lib.kda_prefill(ptr, ptr, ptr, dtype, ptr, ptr, s0, FAKE, arr, N, H, dk, dv, chunk,
+                           out, out, ws, ws_bytes, None)
+
+
+def test_prefill_rejects_bad_arguments(lib):
+    assert _prefill(lib, [0, 4], 1, H=0) == INVALID
+    assert _prefill(lib, [0, 4], 1, dk=0) == INVALID
+    assert _prefill(lib, [0, 4], 1, dtype=7) == INVALID
+    assert _prefill(lib, [0, 4], -1) == INVALID
+    assert _prefill(lib, [0, 4], 1, chunk=48) == UNSUPPORTED
+    assert _prefill(lib, [0, 4], 1, dk=256) == UNSUPPORTED
+    assert _prefill(lib, None, 1) == INVALID                     # no host offsets
+    assert _prefill(lib, [1, 4], 1) == INVALID                   # must start at 0
+    assert _prefill(lib, [0, 4, 3], 2) == INVALID                # decreasing
+    assert _prefill(lib, [0, 4], 1, ptr=None) == INVALID         # null inputs
+    assert _prefill(lib, [0, 4], 1, ptr=ctypes.c_void_p((1 << 20) + 4)) == INVALID  # misaligned
+    assert _prefill(lib, [0, 4], 1, out=None) == INVALID         # null outputs
+    assert _prefill(lib, [0, 4], 1, s0=ctypes.c_void_p((1 << 20) + 8)) == INVALID
+    assert _prefill(lib, [0, 4], 1, ws=None) == WORKSPACE
+    assert _prefill(lib, [0, 4], 1, ws_bytes=16) == WORKSPACE
+    assert _prefill(lib, [0, 4], 1, ws=ctypes.c_void_p((1 << 20) + 64)) == WORKSPACE
+
+
+def test_decode_rejects_bad_arguments(lib):
+    f = lib.kda_decode_step
+    assert f(FAKE, FAKE, FAKE, 1, FAKE, FAKE, FAKE, -1, 2, 128, 128, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, 1, FAKE, FAKE, FAKE, 4, 0, 128, 128, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, 1, FAKE, FAKE, FAKE, 4, 2, 128, 130, FAKE, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 1, FAKE, FAKE, FAKE, 4, 2, 128, 126, FAKE, None) == UNSUPPORTED
+    assert f(FAKE, FAKE, FAKE, 1, FAKE, FAKE, None, 4, 2, 128, 128, FAKE, None) == INVALID
+    assert f(FAKE, FAKE, FAKE, 1, FAKE, FAKE, ctypes.c_void_p((1 << 20) + 4), 4, 2, 128, 128,
+             FAKE, None) == INVALID
+    assert f(None, None, None, 1, None, None, None, 0, 2, 128, 128, None, None) == 0  # B = 0
+
+
+def test_binding_raises_without_library(tmp_path):
+    saved = _binding._lib
+    try:
+        _binding._lib = None
+        with pytest.raises(RuntimeError, match="not found"):
+            _binding.load(str(tmp_path / "missing.so"))
+    finally:
+        _binding._lib = saved
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU failure mode")
+def test_valid_call_without_gpu_reports_cuda_error(lib):
+    # arguments pass the host checks, then the first CUDA call fails: KDA_ERR_CUDA, no crash
+    assert _prefill(lib, [0, 4], 1) == 4
