@@ -1,10 +1,631 @@
-// Tensor-core (tcgen05) chunked prefill for bf16 q/k/v, d_k = d_v = 128, chunk 64.
+// Tensor-core (tcgen05) chunked KDA prefill: bf16 q/k/v, d_k = d_v = 128, chunk 64.
+//
+// Operator: state-update equation of the KDA section of the wiki page "Kimi Linear
+// 高效注意力架构" ("Kimi Delta Attention (KDA)"), read-out o_t = S_t^T q_t, evaluated
+// chunk by chunk in the WY/UT form (the chunkwise algorithm of the same section's
+// "硬件高效分块算法" bullet; its cost terms T d_k d_v + T C d + T C^2 are the
+// comparison table's).  Within a chunk of L <= 64 tokens starting from state S,
+// with g the inclusive running sum of log alpha per key channel:
+//   A_ri = beta_r <k_r e^{g_r - g_i}, k_i> (i < r),   T = (I + A)^{-1} Diag(beta)
+//   P_ri = <q_r e^{g_r - g_i}, k_i> (i <= r)
+//   U = T (V - (K e^{g}) S),   O = (Q e^{g}) S + P U,   S <- Diag(e^{g_L}) S + (K e^{g_L - g})^T U
+//
+// Design (one CTA of 256 threads per (sequence, head), walking its chunks):
+// * The fp32 state is kept TRANSPOSED in tensor memory, S^T[j][c] (TMEM lane = value
+//   column j, 128 lanes), for the whole sequence.  Written this way every product of
+//   the chunk step is a 128-row UMMA with d_v on the M side:
+//     M1  [A; P]^raw   = [K e^{g-g_m}; Q e^{g-g_m}] (K e^{g_m-g})^T   M=128 N=64  K=128
+//     M2  Z            = S^T [K e^{g}; Q e^{g}]^T                    M=128 N=128 K=128
+//     M3  U^T          = Y^T T^T,  Y^T = V^T - Z[:, :64]             M=128 N=64  K=64
+//     M4  S^T         += U^T (K e^{g_L-g})     (after S^T *= e^{g_L}) M=128 N=128 K=64
+//     M5  Z[:, 64:]   += U^T P^T  ( = O^T )                           M=128 N=64  K=64
+//   g_m is the chunk's middle token: the per-pair decay e^{g_r - g_i} is split
+//   into two factors bounded by e^{|g_L|/2}.
+// * Operands are fp16 (fp32 accumulation): the S-dependent chain keeps the
+//   relative error near fp16's 2^-11, which the parity bounds need (bf16 operands
+//   do not meet them).  S^T as an operand lives in TMEM (fp16 pairs per column).
+// * q, k, v and log alpha tiles arrive by TMA in the 128-byte swizzled layout that
+//   the UMMA descriptors use, so the decayed operand rows are built in place.
+// * T is formed in fp32 by a blocked (16x16) forward substitution in shared memory.
+// * All waits are bounded: a wait that runs out sets the workspace error flag and
+//   the CTA stops after its next barrier.
+#include <cuda.h>
+
 #include "kda_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace kda {
+namespace {
 
-bool prefill_tc_supported(const PrefillArgs &) { return false; }
+constexpr int C = 64;    // chunk
+constexpr int D = 128;   // d_k = d_v
+constexpr int NT = 256;  // threads
 
-cudaError_t launch_prefill_tc(const PrefillArgs &, cudaStream_t) { return cudaErrorNotSupported; }
+// Shared memory map (bytes from a 1024-aligned base).
+constexpr uint32_t OFF_QK = 0;        // raw k|q boxes -> [K e^{g-g_m}; Q e^{g-g_m}]  (128 x 128 fp16)
+constexpr uint32_t OFF_LA = 32768;    // raw log alpha boxes -> g (fp32, 64 x 128)
+constexpr uint32_t OFF_V = 65536;     // raw v boxes (bf16, 64 x 128)
+constexpr uint32_t OFF_KB = 81920;    // K e^{g_m - g}   (64 x 128 fp16)
+constexpr uint32_t OFF_KQG = 98304;   // [K e^{g}; Q e^{g}] (128 x 128 fp16)
+constexpr uint32_t OFF_KH = 131072;   // (K e^{g_L - g})^T (128 x 64 fp16)
+constexpr uint32_t OFF_P = 147456;    // P (64 x 64 fp16)
+constexpr uint32_t OFF_T = 155648;    // T (64 x 64 fp16)
+constexpr uint32_t OFF_Y = 163840;    // Y^T (128 x 64 fp16)
+constexpr uint32_t OFF_U = 180224;    // U^T (128 x 64 fp16)
+constexpr uint32_t OFF_VEC = 196608;  // vectors, barriers
+// fp32 scratch of the triangular solve, inside the Kb/KQg region once M1/M2 are done
+constexpr int LDF = 68;
+constexpr uint32_t OFF_AF = OFF_KB;
+constexpr uint32_t OFF_XF = OFF_KB + 64 * LDF * 4;
+constexpr uint32_t OFF_WS = OFF_XF + 64 * LDF * 4;
+static_assert(OFF_WS + 64 * 16 * 4 <= OFF_KH, "solve scratch overflows the Kb/KQg region");
+constexpr uint32_t OFF_GM = OFF_VEC;          // g at the middle token (128 f32)
+constexpr uint32_t OFF_EGM = OFF_VEC + 512;   // e^{g_m}
+constexpr uint32_t OFF_GC = OFF_VEC + 1024;   // g_L
+constexpr uint32_t OFF_GAM = OFF_VEC + 1536;  // e^{g_L}
+constexpr uint32_t OFF_BETA = OFF_VEC + 2048; // beta (64 f32)
+constexpr uint32_t OFF_BAR = OFF_VEC + 2304;  // 4 mbarriers
+constexpr uint32_t OFF_MISC = OFF_VEC + 2336; // tmem base, abort flag
+constexpr uint32_t SMEM_USED = OFF_VEC + 2368;
+constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // + alignment slack
+
+// Tensor memory columns.
+constexpr uint32_t TS = 0;      // S^T fp32         128 cols
+constexpr uint32_t TZ = 128;    // Z fp32           128 cols
+constexpr uint32_t TU = 256;    // U^T fp32          64 cols
+constexpr uint32_t TAP = 320;   // [A; P] raw fp32   64 cols
+constexpr uint32_t TSOP = 384;  // S^T fp16 operand  64 cols
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr uint32_t IDESC_N64 = ptx::idesc_f16_f32(128, 64);
+constexpr uint32_t IDESC_N128 = ptx::idesc_f16_f32(128, 128);
+constexpr long long kWaitCycles = 4000000000LL;  // about two seconds
+
+// byte offset of 16-byte chunk `ch` of row `r` in a 128-byte-row swizzled tile
+__device__ __forceinline__ uint32_t sw(int r, int ch) { return uint32_t(r) * 128u + (uint32_t((ch ^ (r & 7))) << 4); }
+
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+struct TcMaps {
+    CUtensorMap q, k, v, la;
+};
+
+__global__ void __launch_bounds__(NT, 1)
+    prefill_tc_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_s = ptx::smem_u32(smem_raw);
+    const uint32_t pad = ((raw_s + 1023u) & ~1023u) - raw_s;
+    uint8_t *sm = smem_raw + pad;
+    const uint32_t sb = raw_s + pad;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = a.H;
+    const int h = blockIdx.x % H;
+    const int seq = a.order[blockIdx.x / H];
+    const int bos = a.cu_seqlens[seq], eos = a.cu_seqlens[seq + 1];
+    const int nchunks = (eos - bos + C - 1) / C;
+
+    float *s_gm = reinterpret_cast<float *>(sm + OFF_GM);
+    float *s_egm = reinterpret_cast<float *>(sm + OFF_EGM);
+    float *s_gc = reinterpret_cast<float *>(sm + OFF_GC);
+    float *s_gam = reinterpret_cast<float *>(sm + OFF_GAM);
+    float *s_beta = reinterpret_cast<float *>(sm + OFF_BETA);
+    uint64_t *bar_qk = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    uint64_t *bar_la = bar_qk + 1;
+    uint64_t *bar_v = bar_qk + 2;
+    uint64_t *bar_mma = bar_qk + 3;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
+    int *s_abort = reinterpret_cast<int *>(sm + OFF_MISC + 4);
+
+    if (warp == 0) {
+        ptx::tmem_alloc(s_tmem, TMEM_COLS);
+        ptx::tmem_relinquish();
+    }
+    if (tid == 32) {
+        ptx::mbar_init(bar_qk, 1);
+        ptx::mbar_init(bar_la, 1);
+        ptx::mbar_init(bar_v, 1);
+        ptx::mbar_init(bar_mma, 1);
+        ptx::fence_mbar_init();
+        *s_abort = 0;
+        ptx::prefetch_tmap(&maps.q);
+        ptx::prefetch_tmap(&maps.k);
+        ptx::prefetch_tmap(&maps.v);
+        ptx::prefetch_tmap(&maps.la);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tbase = *s_tmem;
+
+    auto load_qk = [&](int s) {
+        ptx::mbar_arrive_expect_tx(bar_qk, 4 * 8192);
+        ptx::tma_load_3d(sm + OFF_QK, &maps.k, bar_qk, 0, h, s);
+        ptx::tma_load_3d(sm + OFF_QK + 8192, &maps.q, bar_qk, 0, h, s);
+        ptx::tma_load_3d(sm + OFF_QK + 16384, &maps.k, bar_qk, 64, h, s);
+        ptx::tma_load_3d(sm + OFF_QK + 24576, &maps.q, bar_qk, 64, h, s);
+    };
+    auto load_la = [&](int s) {
+        ptx::mbar_arrive_expect_tx(bar_la, 4 * 8192);
+        for (int b = 0; b < 4; ++b) ptx::tma_load_3d(sm + OFF_LA + b * 8192, &maps.la, bar_la, 32 * b, h, s);
+    };
+    auto load_v = [&](int s) {
+        ptx::mbar_arrive_expect_tx(bar_v, 2 * 8192);
+        ptx::tma_load_3d(sm + OFF_V, &maps.v, bar_v, 0, h, s);
+        ptx::tma_load_3d(sm + OFF_V + 8192, &maps.v, bar_v, 64, h, s);
+    };
+    auto fail = [&]() {
+        atomicExch(&a.status->flag, 1u);
+        *s_abort = 1;
+    };
+    // Wait for the next phase of `bar`; `waited` counts completed phases and only
+    // advances on success, so an abort can drain the phase that timed out.
+    auto wait_on = [&](uint64_t *bar, int &waited) {
+        if (ptx::mbar_wait_bounded(bar, uint32_t(waited) & 1u, kWaitCycles))
+            ++waited;
+        else
+            fail();
+    };
+
+    // Loads and MMA groups issued (thread 0) and waited for (every thread); on an
+    // abort the CTA waits, bounded, for whatever it still has in flight.
+    int n_qk = 0, n_la = 0, n_v = 0, n_mma = 0;
+    int w_qk = 0, w_la = 0, w_v = 0, w_mma = 0;
+    if (tid == 0 && nchunks > 0) {
+        load_qk(bos);
+        load_la(bos);
+        load_v(bos);
+        n_qk = n_la = n_v = 1;
+    }
+
+    // Thread <-> TMEM mapping for the epilogues: warp w reads lanes 32*(w%4)...,
+    // its column half is w/4.  `row` is the TMEM lane = value column j.
+    const int qd = warp & 3, half = warp >> 2;
+    const int row = qd * 32 + lane;
+    const uint32_t tl = tbase + (uint32_t(qd * 32) << 16);
+    const size_t unit = size_t(seq) * H + h;
+
+    // Initial state: S^T[j][c] = S0[c][j] (fp32) and its fp16 operand copy.
+    {
+        uint32_t v[32], pk[32];
+        for (int p = 0; p < 2; ++p) {
+            for (int e = 0; e < 32; ++e) {
+                const int c = 64 * half + 32 * p + e;
+                const float x = a.S0 ? a.S0[(unit * D + c) * D + row] : 0.f;
+                v[e] = __float_as_uint(x);
+            }
+            ptx::tmem_st32(tl + TS + 64 * half + 32 * p, v);
+            for (int e = 0; e < 16; ++e)
+                pk[16 * p + e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+        }
+        ptx::tmem_st32(tl + TSOP + 32 * half, pk);
+        ptx::tmem_wait_st();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+
+    for (int ci = 0; ci < nchunks; ++ci) {
+        const int s = bos + ci * C;
+        const int L = min(C, eos - s);
+        const bool has_next = ci + 1 < nchunks;
+        const int s_next = s + C;
+
+        // ---- P1: g = running sum of log alpha per channel (in place), beta.
+        wait_on(bar_la, w_la);
+        if (tid < D) {
+            const int c = tid, box = c >> 5, lc = c & 31, lch = lc >> 2;
+            uint8_t *col = sm + OFF_LA + box * 8192 + (lc & 3) * 4;
+            const int rm = (L - 1) >> 1;
+            float g = 0.f, gmid = 0.f;
+            for (int r = 0; r < C; ++r) {
+                float *p = reinterpret_cast<float *>(col + sw(r, lch));
+                g += (r < L) ? *p : 0.f;
+                *p = g;
+                if (r == rm) gmid = g;
+            }
+            s_gm[c] = gmid;
+            s_egm[c] = expf(gmid);
+            s_gc[c] = g;
+            s_gam[c] = expf(g);
+        } else if (tid < D + C) {
+            const int r = tid - D;
+            s_beta[r] = (r < L) ? a.beta[size_t(s + r) * H + h] : 0.f;
+        }
+        wait_on(bar_qk, w_qk);
+        __syncthreads();
+        if (*s_abort) break;
+
+        // ---- P3: (K e^{g_L - g})^T, one channel row per thread pair, 32 tokens each.
+        {
+            const int c = tid & 127, ih = tid >> 7;
+            const int kb = c >> 6, kc = c & 63, kch = kc >> 3;
+            const uint8_t *kcol = sm + OFF_QK + kb * 16384 + (kc & 7) * 2;
+            const int box = c >> 5, lc = c & 31, lch = lc >> 2;
+            const uint8_t *gcol = sm + OFF_LA + box * 8192 + (lc & 3) * 4;
+            const float gl = s_gc[c];
+            for (int q8 = 0; q8 < 4; ++q8) {
+                uint32_t pk[4];
+                for (int e = 0; e < 8; e += 2) {
+                    float val[2];
+                    for (int u = 0; u < 2; ++u) {
+                        const int i = 32 * ih + 8 * q8 + e + u;
+                        const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kcol + sw(i, kch)));
+                        const float gi = *reinterpret_cast<const float *>(gcol + sw(i, lch));
+                        val[u] = (i < L) ? kv * __expf(gl - gi) : 0.f;
+                    }
+                    pk[e >> 1] = pack_h2(val[0], val[1]);
+                }
+                *reinterpret_cast<uint4 *>(sm + OFF_KH + sw(c, 4 * ih + q8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+        }
+        __syncthreads();
+
+        // ---- P2: decayed operand rows, built in place over the raw k|q rows.
+        {
+            const int r = tid & 63, part = tid >> 6, kb = part >> 1;
+            const bool valid = r < L;
+            for (int qq = 0; qq < 4; ++qq) {
+                const int ch = (part & 1) * 4 + qq;
+                const uint32_t ph16 = sw(r, ch);
+                const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + OFF_QK + kb * 16384 + ph16);
+                const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + OFF_QK + kb * 16384 + 8192 + ph16);
+                const int c0 = 64 * kb + 8 * ch;
+                const int box = c0 >> 5, lch = (c0 & 31) >> 2;
+                const float4 ga = *reinterpret_cast<const float4 *>(sm + OFF_LA + box * 8192 + sw(r, lch));
+                const float4 gb = *reinterpret_cast<const float4 *>(sm + OFF_LA + box * 8192 + sw(r, lch + 1));
+                const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
+                const uint32_t qw[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
+                uint32_t o_kt[4], o_qt[4], o_kb[4], o_kg[4], o_qg[4];
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    float kt[2], qt[2], kbv[2], kg[2], qg[2];
+                    for (int u = 0; u < 2; ++u) {
+                        const int e = 2 * e2 + u, c = c0 + e;
+                        const float kv = u ? bf16_hi(kw[e2]) : bf16_lo(kw[e2]);
+                        const float qv = u ? bf16_hi(qw[e2]) : bf16_lo(qw[e2]);
+                        const float up = __expf(gv[e] - s_gm[c]);
+                        const float dn = __expf(s_gm[c] - gv[e]);
+                        const float eg = up * s_egm[c];
+                        kt[u] = valid ? kv * up : 0.f;
+                        qt[u] = valid ? qv * up : 0.f;
+                        kbv[u] = valid ? kv * dn : 0.f;
+                        kg[u] = valid ? kv * eg : 0.f;
+                        qg[u] = valid ? qv * eg : 0.f;
+                    }
+                    o_kt[e2] = pack_h2(kt[0], kt[1]);
+                    o_qt[e2] = pack_h2(qt[0], qt[1]);
+                    o_kb[e2] = pack_h2(kbv[0], kbv[1]);
+                    o_kg[e2] = pack_h2(kg[0], kg[1]);
+                    o_qg[e2] = pack_h2(qg[0], qg[1]);
+                }
+                *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + ph16) = make_uint4(o_kt[0], o_kt[1], o_kt[2], o_kt[3]);
+                *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + 8192 + ph16) = make_uint4(o_qt[0], o_qt[1], o_qt[2], o_qt[3]);
+                *reinterpret_cast<uint4 *>(sm + OFF_KB + kb * 8192 + ph16) = make_uint4(o_kb[0], o_kb[1], o_kb[2], o_kb[3]);
+                *reinterpret_cast<uint4 *>(sm + OFF_KQG + kb * 16384 + ph16) = make_uint4(o_kg[0], o_kg[1], o_kg[2], o_kg[3]);
+                *reinterpret_cast<uint4 *>(sm + OFF_KQG + kb * 16384 + 8192 + ph16) = make_uint4(o_qg[0], o_qg[1], o_qg[2], o_qg[3]);
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---- M1 and M2, then the next chunk's log alpha (g is no longer read).
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t ka = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
+                const uint32_t kbo = uint32_t(ks >> 2) * 8192u + uint32_t(ks & 3) * 32u;
+                ptx::mma_ss(tbase + TAP, ptx::sdesc_sw128(sb + OFF_QK + ka), ptx::sdesc_sw128(sb + OFF_KB + kbo),
+                            IDESC_N64, ks > 0);
+            }
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint32_t kq = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
+                ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_KQG + kq), IDESC_N128,
+                            ks > 0);
+            }
+            ptx::mma_commit(bar_mma);
+            ++n_mma;
+            if (has_next) {
+                load_la(s_next);
+                ++n_la;
+            }
+        }
+        wait_on(bar_mma, w_mma);
+        ptx::tc_fence_after();
+        if (tid == 0 && has_next) {  // M1 has read the k|q tile
+            load_qk(s_next);
+            ++n_qk;
+        }
+        wait_on(bar_v, w_v);
+
+        // ---- E1: A rows -> fp32 scratch, P rows -> fp16 operand.  E2: Y^T, S^T *= e^{g_L}.
+        {
+            uint32_t v[32];
+            ptx::tmem_ld32(tl + TAP + 32 * half, v);
+            ptx::tmem_wait_ld();
+            if (qd < 2) {
+                const int r = row;
+                const float br = s_beta[r];
+                float *af = reinterpret_cast<float *>(sm + OFF_AF) + r * LDF + 32 * half;
+                for (int e = 0; e < 32; e += 4) {
+                    float4 x;
+                    const int i = 32 * half + e;
+                    x.x = (i + 0 < r) ? br * __uint_as_float(v[e + 0]) : 0.f;
+                    x.y = (i + 1 < r) ? br * __uint_as_float(v[e + 1]) : 0.f;
+                    x.z = (i + 2 < r) ? br * __uint_as_float(v[e + 2]) : 0.f;
+                    x.w = (i + 3 < r) ? br * __uint_as_float(v[e + 3]) : 0.f;
+                    *reinterpret_cast<float4 *>(af + e) = x;
+                }
+            } else {
+                const int r = row - 64;
+                for (int qq = 0; qq < 4; ++qq) {
+                    uint32_t pk[4];
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const int e = 8 * qq + 2 * e2, i = 32 * half + e;
+                        pk[e2] = pack_h2(i <= r ? __uint_as_float(v[e]) : 0.f,
+                                         i + 1 <= r ? __uint_as_float(v[e + 1]) : 0.f);
+                    }
+                    *reinterpret_cast<uint4 *>(sm + OFF_P + sw(r, 4 * half + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+            ptx::tmem_ld32(tl + TZ + 32 * half, v);
+            ptx::tmem_wait_ld();
+            {
+                const int j = row, vbox = j >> 6, jj = j & 63, vch = jj >> 3;
+                const uint8_t *vcol = sm + OFF_V + vbox * 8192 + (jj & 7) * 2;
+                for (int qq = 0; qq < 4; ++qq) {
+                    uint32_t pk[4];
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        float y[2];
+                        for (int u = 0; u < 2; ++u) {
+                            const int e = 8 * qq + 2 * e2 + u, i = 32 * half + e;
+                            const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vcol + sw(i, vch)));
+                            y[u] = (i < L) ? vv - __uint_as_float(v[e]) : 0.f;
+                        }
+                        pk[e2] = pack_h2(y[0], y[1]);
+                    }
+                    *reinterpret_cast<uint4 *>(sm + OFF_Y + sw(j, 4 * half + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+            for (int p = 0; p < 2; ++p) {
+                const uint32_t col = TS + 64 * half + 32 * p;
+                ptx::tmem_ld32(tl + col, v);
+                ptx::tmem_wait_ld();
+                for (int e = 0; e < 32; ++e)
+                    v[e] = __float_as_uint(__uint_as_float(v[e]) * s_gam[64 * half + 32 * p + e]);
+                ptx::tmem_st32(tl + col, v);
+            }
+            ptx::tmem_wait_st();
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+        if (*s_abort) break;
+        if (tid == 0 && has_next) {  // V has been read
+            load_v(s_next);
+            ++n_v;
+        }
+
+        // ---- T = (I + A)^{-1} Diag(beta): 16x16 diagonal blocks, then the blocks
+        // below them by distance from the diagonal.  Thread (row r, 4-column group jq).
+        {
+            float *Af = reinterpret_cast<float *>(sm + OFF_AF);
+            float *X = reinterpret_cast<float *>(sm + OFF_XF);
+            float *W = reinterpret_cast<float *>(sm + OFF_WS);
+            const int b = tid >> 6, rr = (tid >> 2) & 15, jq = tid & 3;
+            const int r = 16 * b + rr;
+            {
+                const int j = 16 * b + 4 * jq;
+                float acc[4];
+                for (int e = 0; e < 4; ++e) acc[e] = (rr == 4 * jq + e) ? 1.f : 0.f;
+                for (int st = 0; st < 16; ++st) {
+                    if (rr == st) *reinterpret_cast<float4 *>(X + r * LDF + j) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                    ptx::named_barrier(1 + b, 64);
+                    if (rr > st) {
+                        const float av = Af[r * LDF + 16 * b + st];
+                        const float4 xs = *reinterpret_cast<const float4 *>(X + (16 * b + st) * LDF + j);
+                        acc[0] -= av * xs.x;
+                        acc[1] -= av * xs.y;
+                        acc[2] -= av * xs.z;
+                        acc[3] -= av * xs.w;
+                    }
+                }
+            }
+            __syncthreads();
+            for (int d = 1; d <= 3; ++d) {
+                const int bj = b - d;
+                if (bj >= 0) {
+                    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int kk = 16 * bj; kk < 16 * b; ++kk) {
+                        const float av = Af[r * LDF + kk];
+                        const float4 xv = *reinterpret_cast<const float4 *>(X + kk * LDF + 16 * bj + 4 * jq);
+                        w.x += av * xv.x;
+                        w.y += av * xv.y;
+                        w.z += av * xv.z;
+                        w.w += av * xv.w;
+                    }
+                    *reinterpret_cast<float4 *>(W + r * 16 + 4 * jq) = w;
+                }
+                __syncthreads();
+                if (bj >= 0) {
+                    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int ss = 0; ss <= rr; ++ss) {
+                        const float xv = X[r * LDF + 16 * b + ss];
+                        const float4 wv = *reinterpret_cast<const float4 *>(W + (16 * b + ss) * 16 + 4 * jq);
+                        o.x -= xv * wv.x;
+                        o.y -= xv * wv.y;
+                        o.z -= xv * wv.z;
+                        o.w -= xv * wv.w;
+                    }
+                    *reinterpret_cast<float4 *>(X + r * LDF + 16 * bj + 4 * jq) = o;
+                }
+                __syncthreads();
+            }
+            // T[r][i] = X[r][i] beta_i for i <= r, as an fp16 operand (rows r, K = i).
+            {
+                const int rt = tid & 63, part = tid >> 6;
+                for (int qq = 0; qq < 2; ++qq) {
+                    const int ch = 2 * part + qq;
+                    uint32_t pk[4];
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const int i = 8 * ch + 2 * e2;
+                        const float x0 = (i <= rt) ? X[rt * LDF + i] * s_beta[i] : 0.f;
+                        const float x1 = (i + 1 <= rt) ? X[rt * LDF + i + 1] * s_beta[i + 1] : 0.f;
+                        pk[e2] = pack_h2(x0, x1);
+                    }
+                    *reinterpret_cast<uint4 *>(sm + OFF_T + sw(rt, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---- M3: U^T = Y^T T^T.
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            for (int ks = 0; ks < 4; ++ks)
+                ptx::mma_ss(tbase + TU, ptx::sdesc_sw128(sb + OFF_Y + 32 * ks), ptx::sdesc_sw128(sb + OFF_T + 32 * ks),
+                            IDESC_N64, ks > 0);
+            ptx::mma_commit(bar_mma);
+            ++n_mma;
+        }
+        wait_on(bar_mma, w_mma);
+        ptx::tc_fence_after();
+        {  // E3: U^T -> fp16 operand
+            uint32_t v[32];
+            ptx::tmem_ld32(tl + TU + 32 * half, v);
+            ptx::tmem_wait_ld();
+            for (int qq = 0; qq < 4; ++qq) {
+                uint32_t pk[4];
+                for (int e2 = 0; e2 < 4; ++e2) {
+                    const int e = 8 * qq + 2 * e2;
+                    pk[e2] = pack_h2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                }
+                *reinterpret_cast<uint4 *>(sm + OFF_U + sw(row, 4 * half + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_before();
+        __syncthreads();
+        if (*s_abort) break;
+
+        // ---- M4: S^T += U^T (K e^{g_L-g});  M5: O^T = Z[:, 64:] + U^T P^T.
+        if (tid == 0) {
+            ptx::tc_fence_after();
+            for (int ks = 0; ks < 4; ++ks)
+                ptx::mma_ss(tbase + TS, ptx::sdesc_sw128(sb + OFF_U + 32 * ks), ptx::sdesc_sw128(sb + OFF_KH + 32 * ks),
+                            IDESC_N128, 1u);
+            for (int ks = 0; ks < 4; ++ks)
+                ptx::mma_ss(tbase + TZ + 64, ptx::sdesc_sw128(sb + OFF_U + 32 * ks), ptx::sdesc_sw128(sb + OFF_P + 32 * ks),
+                            IDESC_N64, 1u);
+            ptx::mma_commit(bar_mma);
+            ++n_mma;
+        }
+        wait_on(bar_mma, w_mma);
+        ptx::tc_fence_after();
+        {  // E4: next S^T operand, outputs of this chunk.
+            uint32_t v[32], pk[32];
+            for (int p = 0; p < 2; ++p) {
+                ptx::tmem_ld32(tl + TS + 64 * half + 32 * p, v);
+                ptx::tmem_wait_ld();
+                for (int e = 0; e < 16; ++e)
+                    pk[16 * p + e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+            }
+            ptx::tmem_st32(tl + TSOP + 32 * half, pk);
+            ptx::tmem_ld32(tl + TZ + 64 + 32 * half, v);
+            ptx::tmem_wait_ld();
+            __nv_bfloat16 *op = static_cast<__nv_bfloat16 *>(a.o);
+            for (int e = 0; e < 32; ++e) {
+                const int r = 32 * half + e;
+                if (r < L) op[(size_t(s + r) * H + h) * D + row] = __float2bfloat16_rn(__uint_as_float(v[e]));
+            }
+            ptx::tmem_wait_st();
+        }
+        ptx::tc_fence_before();
+        __syncthreads();
+        if (*s_abort) break;
+    }
+
+    if (*s_abort && tid == 0) {  // drain what is still in flight (each wait bounded)
+        while (w_qk < n_qk) ptx::mbar_wait_bounded(bar_qk, uint32_t(w_qk++) & 1u, kWaitCycles);
+        while (w_la < n_la) ptx::mbar_wait_bounded(bar_la, uint32_t(w_la++) & 1u, kWaitCycles);
+        while (w_v < n_v) ptx::mbar_wait_bounded(bar_v, uint32_t(w_v++) & 1u, kWaitCycles);
+        while (w_mma < n_mma) ptx::mbar_wait_bounded(bar_mma, uint32_t(w_mma++) & 1u, kWaitCycles);
+    }
+    // Final state S_final[c][j] = S^T[j][c].
+    if (!*s_abort) {
+        ptx::tc_fence_after();
+        uint32_t v[32];
+        for (int p = 0; p < 2; ++p) {
+            ptx::tmem_ld32(tl + TS + 64 * half + 32 * p, v);
+            ptx::tmem_wait_ld();
+            for (int e = 0; e < 32; ++e) {
+                const int c = 64 * half + 32 * p + e;
+                a.S_final[(unit * D + c) * D + row] = __uint_as_float(v[e]);
+            }
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tbase, TMEM_COLS);
+    }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// [T, H, 128] row-major tensor, boxes of 128 bytes x 64 tokens, 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes, int H, int64_t T) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(H), cuuint64_t(T)};
+    const cuuint64_t strides[2] = {cuuint64_t(D) * elem_bytes, cuuint64_t(H) * D * elem_bytes};
+    const cuuint32_t box[3] = {cuuint32_t(128 / elem_bytes), 1u, cuuint32_t(C)};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool prefill_tc_supported(const PrefillArgs &a) {
+    return a.dtype == KDA_DTYPE_BF16 && a.dk == D && a.dv == D && a.chunk == C && a.total_tokens > 0 &&
+           a.num_seqs > 0;
+}
+
+cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
+    TcMaps maps;
+    if (!make_map(&maps.q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens) ||
+        !make_map(&maps.k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens) ||
+        !make_map(&maps.v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens) ||
+        !make_map(&maps.la, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.H, a.total_tokens))
+        return cudaErrorInvalidValue;
+    cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           int(SMEM_ALLOC));
+    if (err != cudaSuccess) return err;
+    const unsigned grid = unsigned(a.num_seqs) * unsigned(a.H);
+    prefill_tc_kernel<<<grid, NT, SMEM_ALLOC, stream>>>(maps, a);
+    return cudaGetLastError();
+}
 
 }  // namespace kda
