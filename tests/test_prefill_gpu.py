@@ -85,8 +85,11 @@ def test_split_invariance_and_aliasing():
     ob, Sb = kda_prefill(b["q"], b["k"], b["v"], b["log_alpha"], b["beta"], cu2, [0, T2],
                          S0=Sa, S_final=Sa)
     assert Sb.data_ptr() == Sa.data_ptr()
-    assert rel_l2(host64(torch.cat([oa, ob])), host64(o)) < 2e-3
-    assert rel_l2(host64(Sb), host64(S)) < 1e-4
+    # both runs carry the path's own rounding (fp16 tensor-core operands), so they
+    # agree to twice the parity bound rather than bit for bit
+    assert rel_l2(host64(torch.cat([oa, ob])), host64(o)) < 2 * TOL["bf16"]["o"]
+    assert rel_l2(host64(Sb), host64(S)) < 2 * TOL["bf16"]["S"]
+    compare_full(inp, o, S, "bf16")
 
 
 def test_prefill_then_decode_equals_longer_prefill():
@@ -101,8 +104,8 @@ def test_prefill_then_decode_equals_longer_prefill():
     for t in range(T, T + n):
         outs.append(kda_decode_step(inp["q"][t:t + 1], inp["k"][t:t + 1], inp["v"][t:t + 1],
                                     inp["log_alpha"][t:t + 1], inp["beta"][t:t + 1], S))
-    assert rel_l2(host64(torch.cat(outs)), host64(o_all[T:])) < 2e-3
-    assert rel_l2(host64(S[0]), host64(S_all[0])) < 1e-4
+    assert rel_l2(host64(torch.cat(outs)), host64(o_all[T:])) < 2 * TOL["bf16"]["o"]
+    assert rel_l2(host64(S[0]), host64(S_all[0])) < 2 * TOL["bf16"]["S"]
 
 
 def test_empty_sequences_keep_initial_state():
