@@ -11,22 +11,28 @@
 //   U = T (V - (K e^{g}) S),   O = (Q e^{g}) S + P U,   S <- Diag(e^{g_L}) S + (K e^{g_L - g})^T U
 //
 // Design (one CTA of 256 threads per (sequence, head), walking its chunks):
-// * The fp32 state is kept TRANSPOSED in tensor memory, S^T[j][c] (TMEM lane = value
-//   column j, 128 lanes), for the whole sequence.  Written this way every product of
-//   the chunk step is a 128-row UMMA with d_v on the M side:
-//     M1  [A; P]^raw   = [K e^{g-g_m}; Q e^{g-g_m}] (K e^{g_m-g})^T   M=128 N=64  K=128
-//     M2  Z            = S^T [K e^{g}; Q e^{g}]^T                    M=128 N=128 K=128
-//     M3  U^T          = Y^T T^T,  Y^T = V^T - Z[:, :64]             M=128 N=64  K=64
-//     M4  S^T         += U^T (K e^{g_L-g})     (after S^T *= e^{g_L}) M=128 N=128 K=64
-//     M5  Z[:, 64:]   += U^T P^T  ( = O^T )                           M=128 N=64  K=64
-//   g_m is the chunk's middle token: the per-pair decay e^{g_r - g_i} is split
-//   into two factors bounded by e^{|g_L|/2}.
+// * The fp32 state is kept TRANSPOSED in tensor memory (TMEM lane = value column
+//   j, 128 lanes) for the whole sequence, so every product of the chunk step is a
+//   128-row UMMA with d_v on the M side.  With Kt = K e^{g-g_m}, Qt = Q e^{g-g_m},
+//   Kb = K e^{g_m-g} (g_m: the chunk's middle token, so both factors stay within
+//   e^{+-|g_L|/2}) and the fp16 state operand Sop = S^T Diag(e^{g_m}):
+//     M1  [A; P]^raw = [Kt; Qt] Kb^T                 M=128 N=64  K=128
+//     M2  Z          = Sop [Kt; Qt]^T                M=128 N=128 K=128
+//           Z[:, :64] = (K e^{g} S)^T,  Z[:, 64:] = (Q e^{g} S)^T
+//     M3  U^T        = Y^T T^T,  Y^T = V^T - Z[:, :64]   M=128 N=64  K=64
+//     M4  R         += U^T Kb      (Kb read as an MN-major operand)  N=128 K=64
+//     M5  Z[:, 64:] += U^T P^T  ( = O^T )                   N=64  K=64
+//   TMEM holds R = S^T Diag(e^{g_m - g_L}) of the previous chunk rather than S^T:
+//   the per-channel factors e^{g_L - g_m} and e^{g_m} then fold into one rescale
+//   of R per chunk and into the fp16 pack of the next Sop, so no K e^{g},
+//   Q e^{g} or (K e^{g_L - g})^T tile is built.
 // * Operands are fp16 (fp32 accumulation): the S-dependent chain keeps the
 //   relative error near fp16's 2^-11, which the parity bounds need (bf16 operands
-//   do not meet them).  S^T as an operand lives in TMEM (fp16 pairs per column).
+//   do not meet them).  Sop lives in TMEM (fp16 pairs per column).
 // * q, k, v and log alpha tiles arrive by TMA in the 128-byte swizzled layout that
 //   the UMMA descriptors use, so the decayed operand rows are built in place.
 // * T is formed in fp32 by a blocked (16x16) forward substitution in shared memory.
+// * The running sums of the next chunk are formed while M4/M5 run.
 // * All waits are bounded: a wait that runs out sets the workspace error flag and
 //   the CTA stops after its next barrier.
 #include <cuda.h>
@@ -42,43 +48,44 @@ constexpr int D = 128;   // d_k = d_v
 constexpr int NT = 256;  // threads
 
 // Shared memory map (bytes from a 1024-aligned base).
-constexpr uint32_t OFF_QK = 0;        // raw k|q boxes -> [K e^{g-g_m}; Q e^{g-g_m}]  (128 x 128 fp16)
+constexpr uint32_t OFF_QK = 0;        // raw k|q boxes -> [Kt; Qt]  (128 x 128 fp16, K-major)
 constexpr uint32_t OFF_LA = 32768;    // raw log alpha boxes -> g (fp32, 64 x 128)
 constexpr uint32_t OFF_V = 65536;     // raw v boxes (bf16, 64 x 128)
-constexpr uint32_t OFF_KB = 81920;    // K e^{g_m - g}   (64 x 128 fp16)
-constexpr uint32_t OFF_KQG = 98304;   // [K e^{g}; Q e^{g}] (128 x 128 fp16)
-constexpr uint32_t OFF_KH = 131072;   // (K e^{g_L - g})^T (128 x 64 fp16)
-constexpr uint32_t OFF_P = 147456;    // P (64 x 64 fp16)
-constexpr uint32_t OFF_T = 155648;    // T (64 x 64 fp16)
-constexpr uint32_t OFF_Y = 163840;    // Y^T (128 x 64 fp16)
-constexpr uint32_t OFF_U = 180224;    // U^T (128 x 64 fp16)
-constexpr uint32_t OFF_VEC = 196608;  // vectors, barriers
-// fp32 scratch of the triangular solve, inside the Kb/KQg region once M1/M2 are done
+constexpr uint32_t OFF_KB = 81920;    // Kb (64 x 128 fp16): B of M1 (K-major) and of M4 (MN-major)
+constexpr uint32_t OFF_SCR = 98304;   // fp32 scratch of the triangular solve
 constexpr int LDF = 68;
-constexpr uint32_t OFF_AF = OFF_KB;
-constexpr uint32_t OFF_XF = OFF_KB + 64 * LDF * 4;
-constexpr uint32_t OFF_WS = OFF_XF + 64 * LDF * 4;
-static_assert(OFF_WS + 64 * 16 * 4 <= OFF_KH, "solve scratch overflows the Kb/KQg region");
-constexpr uint32_t OFF_GM = OFF_VEC;          // g at the middle token (128 f32)
-constexpr uint32_t OFF_EGM = OFF_VEC + 512;   // e^{g_m}
-constexpr uint32_t OFF_GC = OFF_VEC + 1024;   // g_L
-constexpr uint32_t OFF_GAM = OFF_VEC + 1536;  // e^{g_L}
-constexpr uint32_t OFF_BETA = OFF_VEC + 2048; // beta (64 f32)
-constexpr uint32_t OFF_BAR = OFF_VEC + 2304;  // 4 mbarriers
-constexpr uint32_t OFF_MISC = OFF_VEC + 2336; // tmem base, abort flag
-constexpr uint32_t SMEM_USED = OFF_VEC + 2368;
+constexpr int LDE = 20;
+constexpr uint32_t OFF_AF = OFF_SCR;
+constexpr uint32_t OFF_XF = OFF_AF + 64 * LDF * 4;
+constexpr uint32_t OFF_EB = OFF_XF + 64 * LDF * 4;  // six 16x16 blocks X_bb A_bk
+constexpr uint32_t OFF_P = 141312;    // P (64 x 64 fp16)
+static_assert(OFF_EB + 6 * 16 * LDE * 4 <= OFF_P, "solve scratch overflows");
+constexpr uint32_t OFF_T = OFF_P + 8192;     // T (64 x 64 fp16)
+constexpr uint32_t OFF_Y = OFF_T + 8192;     // Y^T (128 x 64 fp16); later the bf16 output tile
+constexpr uint32_t OFF_U = OFF_Y + 16384;    // U^T (128 x 64 fp16)
+constexpr uint32_t OFF_VEC = OFF_U + 16384;  // per-chunk vectors, two buffers (chunk parity)
+constexpr uint32_t VEC_GM = 0;        // g_m                  128 f32
+constexpr uint32_t VEC_EGM = 512;     // e^{g_m}
+constexpr uint32_t VEC_ECM = 1024;    // e^{g_L - g_m}
+constexpr uint32_t VEC_BETA = 1536;   // beta                 64 f32
+constexpr uint32_t VEC_BYTES = 1792;
+constexpr uint32_t OFF_HALF = OFF_VEC + 2 * VEC_BYTES;  // running sum over the first 32 tokens
+constexpr uint32_t OFF_BAR = OFF_HALF + 512;            // 4 mbarriers
+constexpr uint32_t OFF_MISC = OFF_BAR + 32;             // tmem base, abort flag
+constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // + alignment slack
 
 // Tensor memory columns.
-constexpr uint32_t TS = 0;      // S^T fp32         128 cols
-constexpr uint32_t TZ = 128;    // Z fp32           128 cols
-constexpr uint32_t TU = 256;    // U^T fp32          64 cols
-constexpr uint32_t TAP = 320;   // [A; P] raw fp32   64 cols
-constexpr uint32_t TSOP = 384;  // S^T fp16 operand  64 cols
+constexpr uint32_t TS = 0;      // R (fp32)          128 cols
+constexpr uint32_t TZ = 128;    // Z fp32            128 cols
+constexpr uint32_t TU = 256;    // U^T fp32           64 cols
+constexpr uint32_t TAP = 320;   // [A; P] raw fp32    64 cols
+constexpr uint32_t TSOP = 384;  // Sop fp16           64 cols
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t IDESC_N64 = ptx::idesc_f16_f32(128, 64);
 constexpr uint32_t IDESC_N128 = ptx::idesc_f16_f32(128, 128);
+constexpr uint32_t IDESC_N128_BMN = ptx::idesc_f16_f32(128, 128) | (1u << 16);  // B MN-major
 constexpr long long kWaitCycles = 4000000000LL;  // about two seconds
 
 // byte offset of 16-byte chunk `ch` of row `r` in a 128-byte-row swizzled tile
@@ -110,11 +117,7 @@ __global__ void __launch_bounds__(NT, 1)
     const int bos = a.cu_seqlens[seq], eos = a.cu_seqlens[seq + 1];
     const int nchunks = (eos - bos + C - 1) / C;
 
-    float *s_gm = reinterpret_cast<float *>(sm + OFF_GM);
-    float *s_egm = reinterpret_cast<float *>(sm + OFF_EGM);
-    float *s_gc = reinterpret_cast<float *>(sm + OFF_GC);
-    float *s_gam = reinterpret_cast<float *>(sm + OFF_GAM);
-    float *s_beta = reinterpret_cast<float *>(sm + OFF_BETA);
+    auto vec = [&](int par, uint32_t field) { return reinterpret_cast<float *>(sm + OFF_VEC + par * VEC_BYTES + field); };
     uint64_t *bar_qk = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint64_t *bar_la = bar_qk + 1;
     uint64_t *bar_v = bar_qk + 2;
@@ -183,6 +186,48 @@ __global__ void __launch_bounds__(NT, 1)
         n_qk = n_la = n_v = 1;
     }
 
+    // P1 of chunk `ci`: g = running sum of log alpha per channel, in place over the
+    // log alpha tile, and the chunk's vectors (buffer ci & 1).  Thread (channel c,
+    // half hf) scans tokens [32 hf, 32 hf + 32); the second half then adds the
+    // first half's total.  The middle token (L - 1) / 2 is always in the first half.
+    // `bval` is this thread's beta of the chunk (threads < 64), loaded ahead of time.
+    auto scan = [&](int ci, float bval) {
+        const int s = bos + ci * C, L = min(C, eos - s);
+        float *gm = vec(ci & 1, VEC_GM), *egm = vec(ci & 1, VEC_EGM), *ecm = vec(ci & 1, VEC_ECM);
+        float *beta = vec(ci & 1, VEC_BETA);
+        wait_on(bar_la, w_la);
+        const int c = tid & 127, hf = tid >> 7, box = c >> 5, lc = c & 31, lch = lc >> 2;
+        uint8_t *col = sm + OFF_LA + box * 8192 + (lc & 3) * 4;
+        float *s_half = reinterpret_cast<float *>(sm + OFF_HALF);
+        const int rm = (L - 1) >> 1;
+        float x[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int r = 32 * hf + i;
+            x[i] = (r < L) ? *reinterpret_cast<const float *>(col + sw(r, lch)) : 0.f;
+        }
+#pragma unroll
+        for (int i = 1; i < 32; ++i) x[i] += x[i - 1];
+        if (hf == 0) {
+            float gmid = 0.f;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) gmid = (i == rm) ? x[i] : gmid;
+            s_half[c] = x[31];
+            gm[c] = gmid;
+            egm[c] = expf(gmid);
+        }
+        if (tid < C) beta[tid] = bval;
+        __syncthreads();
+        if (hf == 1) {
+            const float off = s_half[c];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] += off;
+            ecm[c] = expf(x[31] - gm[c]);
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) *reinterpret_cast<float *>(col + sw(32 * hf + i, lch)) = x[i];
+    };
+
     // Thread <-> TMEM mapping for the epilogues: warp w reads lanes 32*(w%4)...,
     // its column half is w/4.  `row` is the TMEM lane = value column j.
     const int qd = warp & 3, half = warp >> 2;
@@ -190,8 +235,17 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t tl = tbase + (uint32_t(qd * 32) << 16);
     const size_t unit = size_t(seq) * H + h;
 
-    // Initial state: S^T[j][c] = S0[c][j] (fp32) and its fp16 operand copy.
+    // beta of a chunk is read from global memory one chunk ahead (a register)
+    auto load_beta = [&](int ci) {
+        const int s = bos + ci * C;
+        return (tid < C && ci < nchunks && s + tid < eos) ? a.beta[size_t(s + tid) * H + h] : 0.f;
+    };
+    if (nchunks > 0) scan(0, load_beta(0));
+    __syncthreads();
+
+    // Initial state: R = S0^T (fp32) and Sop = S0^T Diag(e^{g_m}) of chunk 0 (fp16).
     {
+        const float *egm0 = vec(0, VEC_EGM);
         uint32_t v[32], pk[32];
         for (int p = 0; p < 2; ++p) {
             for (int e = 0; e < 32; ++e) {
@@ -200,10 +254,12 @@ __global__ void __launch_bounds__(NT, 1)
                 v[e] = __float_as_uint(x);
             }
             ptx::tmem_st32(tl + TS + 64 * half + 32 * p, v);
-            for (int e = 0; e < 16; ++e)
-                pk[16 * p + e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+            for (int e = 0; e < 16; ++e) {
+                const int c = 64 * half + 32 * p + 2 * e;
+                pk[16 * p + e] = pack_h2(__uint_as_float(v[2 * e]) * egm0[c], __uint_as_float(v[2 * e + 1]) * egm0[c + 1]);
+            }
         }
-        ptx::tmem_st32(tl + TSOP + 32 * half, pk);
+        if (nchunks > 0) ptx::tmem_st32(tl + TSOP + 32 * half, pk);
         ptx::tmem_wait_st();
     }
     ptx::tc_fence_before();
@@ -214,61 +270,18 @@ __global__ void __launch_bounds__(NT, 1)
         const int L = min(C, eos - s);
         const bool has_next = ci + 1 < nchunks;
         const int s_next = s + C;
+        const int par = ci & 1;
+        const float *gm = vec(par, VEC_GM);
+        const float *beta = vec(par, VEC_BETA);
+        const float beta_next = load_beta(ci + 1);
 
-        // ---- P1: g = running sum of log alpha per channel (in place), beta.
-        wait_on(bar_la, w_la);
-        if (tid < D) {
-            const int c = tid, box = c >> 5, lc = c & 31, lch = lc >> 2;
-            uint8_t *col = sm + OFF_LA + box * 8192 + (lc & 3) * 4;
-            const int rm = (L - 1) >> 1;
-            float g = 0.f, gmid = 0.f;
-            for (int r = 0; r < C; ++r) {
-                float *p = reinterpret_cast<float *>(col + sw(r, lch));
-                g += (r < L) ? *p : 0.f;
-                *p = g;
-                if (r == rm) gmid = g;
-            }
-            s_gm[c] = gmid;
-            s_egm[c] = expf(gmid);
-            s_gc[c] = g;
-            s_gam[c] = expf(g);
-        } else if (tid < D + C) {
-            const int r = tid - D;
-            s_beta[r] = (r < L) ? a.beta[size_t(s + r) * H + h] : 0.f;
-        }
+        // ---- P2: Kt, Qt (in place over the raw k|q rows) and Kb; one (token row,
+        // 32-channel quarter) per thread.
         wait_on(bar_qk, w_qk);
-        __syncthreads();
-        if (*s_abort) break;
-
-        // ---- P3: (K e^{g_L - g})^T, one channel row per thread pair, 32 tokens each.
-        {
-            const int c = tid & 127, ih = tid >> 7;
-            const int kb = c >> 6, kc = c & 63, kch = kc >> 3;
-            const uint8_t *kcol = sm + OFF_QK + kb * 16384 + (kc & 7) * 2;
-            const int box = c >> 5, lc = c & 31, lch = lc >> 2;
-            const uint8_t *gcol = sm + OFF_LA + box * 8192 + (lc & 3) * 4;
-            const float gl = s_gc[c];
-            for (int q8 = 0; q8 < 4; ++q8) {
-                uint32_t pk[4];
-                for (int e = 0; e < 8; e += 2) {
-                    float val[2];
-                    for (int u = 0; u < 2; ++u) {
-                        const int i = 32 * ih + 8 * q8 + e + u;
-                        const float kv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(kcol + sw(i, kch)));
-                        const float gi = *reinterpret_cast<const float *>(gcol + sw(i, lch));
-                        val[u] = (i < L) ? kv * __expf(gl - gi) : 0.f;
-                    }
-                    pk[e >> 1] = pack_h2(val[0], val[1]);
-                }
-                *reinterpret_cast<uint4 *>(sm + OFF_KH + sw(c, 4 * ih + q8)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
-        }
-        __syncthreads();
-
-        // ---- P2: decayed operand rows, built in place over the raw k|q rows.
         {
             const int r = tid & 63, part = tid >> 6, kb = part >> 1;
             const bool valid = r < L;
+#pragma unroll
             for (int qq = 0; qq < 4; ++qq) {
                 const int ch = (part & 1) * 4 + qq;
                 const uint32_t ph16 = sw(r, ch);
@@ -278,42 +291,41 @@ __global__ void __launch_bounds__(NT, 1)
                 const int box = c0 >> 5, lch = (c0 & 31) >> 2;
                 const float4 ga = *reinterpret_cast<const float4 *>(sm + OFF_LA + box * 8192 + sw(r, lch));
                 const float4 gb = *reinterpret_cast<const float4 *>(sm + OFF_LA + box * 8192 + sw(r, lch + 1));
-                const float gv[8] = {ga.x, ga.y, ga.z, ga.w, gb.x, gb.y, gb.z, gb.w};
+                const float4 m0 = *reinterpret_cast<const float4 *>(gm + c0);
+                const float4 m1 = *reinterpret_cast<const float4 *>(gm + c0 + 4);
+                const float dg[8] = {ga.x - m0.x, ga.y - m0.y, ga.z - m0.z, ga.w - m0.w,
+                                     gb.x - m1.x, gb.y - m1.y, gb.z - m1.z, gb.w - m1.w};
                 const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
                 const uint32_t qw[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
-                uint32_t o_kt[4], o_qt[4], o_kb[4], o_kg[4], o_qg[4];
+                uint32_t o_kt[4], o_qt[4], o_kb[4];
+#pragma unroll
                 for (int e2 = 0; e2 < 4; ++e2) {
-                    float kt[2], qt[2], kbv[2], kg[2], qg[2];
+                    float kt[2], qt[2], kbv[2];
+#pragma unroll
                     for (int u = 0; u < 2; ++u) {
-                        const int e = 2 * e2 + u, c = c0 + e;
+                        const int e = 2 * e2 + u;
                         const float kv = u ? bf16_hi(kw[e2]) : bf16_lo(kw[e2]);
                         const float qv = u ? bf16_hi(qw[e2]) : bf16_lo(qw[e2]);
-                        const float up = __expf(gv[e] - s_gm[c]);
-                        const float dn = __expf(s_gm[c] - gv[e]);
-                        const float eg = up * s_egm[c];
+                        const float up = __expf(dg[e]);
+                        const float dn = __expf(-dg[e]);
                         kt[u] = valid ? kv * up : 0.f;
                         qt[u] = valid ? qv * up : 0.f;
                         kbv[u] = valid ? kv * dn : 0.f;
-                        kg[u] = valid ? kv * eg : 0.f;
-                        qg[u] = valid ? qv * eg : 0.f;
                     }
                     o_kt[e2] = pack_h2(kt[0], kt[1]);
                     o_qt[e2] = pack_h2(qt[0], qt[1]);
                     o_kb[e2] = pack_h2(kbv[0], kbv[1]);
-                    o_kg[e2] = pack_h2(kg[0], kg[1]);
-                    o_qg[e2] = pack_h2(qg[0], qg[1]);
                 }
                 *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + ph16) = make_uint4(o_kt[0], o_kt[1], o_kt[2], o_kt[3]);
                 *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + 8192 + ph16) = make_uint4(o_qt[0], o_qt[1], o_qt[2], o_qt[3]);
                 *reinterpret_cast<uint4 *>(sm + OFF_KB + kb * 8192 + ph16) = make_uint4(o_kb[0], o_kb[1], o_kb[2], o_kb[3]);
-                *reinterpret_cast<uint4 *>(sm + OFF_KQG + kb * 16384 + ph16) = make_uint4(o_kg[0], o_kg[1], o_kg[2], o_kg[3]);
-                *reinterpret_cast<uint4 *>(sm + OFF_KQG + kb * 16384 + 8192 + ph16) = make_uint4(o_qg[0], o_qg[1], o_qg[2], o_qg[3]);
             }
         }
         ptx::fence_proxy_async_smem();
         __syncthreads();
+        if (*s_abort) break;
 
-        // ---- M1 and M2, then the next chunk's log alpha (g is no longer read).
+        // ---- M1 and M2; then the next chunk's log alpha (g of this chunk is done).
         if (tid == 0) {
             ptx::tc_fence_after();
             for (int ks = 0; ks < 8; ++ks) {
@@ -324,7 +336,7 @@ __global__ void __launch_bounds__(NT, 1)
             }
             for (int ks = 0; ks < 8; ++ks) {
                 const uint32_t kq = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
-                ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_KQG + kq), IDESC_N128,
+                ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_QK + kq), IDESC_N128,
                             ks > 0);
             }
             ptx::mma_commit(bar_mma);
@@ -336,20 +348,21 @@ __global__ void __launch_bounds__(NT, 1)
         }
         wait_on(bar_mma, w_mma);
         ptx::tc_fence_after();
-        if (tid == 0 && has_next) {  // M1 has read the k|q tile
+        if (tid == 0 && has_next) {  // M1 and M2 have read the [Kt; Qt] tile
             load_qk(s_next);
             ++n_qk;
         }
         wait_on(bar_v, w_v);
 
-        // ---- E1: A rows -> fp32 scratch, P rows -> fp16 operand.  E2: Y^T, S^T *= e^{g_L}.
+        // ---- E1: A rows -> fp32 scratch, P rows -> fp16 operand.
+        // ---- E2: Y^T = V^T - Z[:, :64] -> fp16 operand; R *= e^{g_L - g_m}(prev) e^{g_m}.
         {
             uint32_t v[32];
             ptx::tmem_ld32(tl + TAP + 32 * half, v);
             ptx::tmem_wait_ld();
             if (qd < 2) {
                 const int r = row;
-                const float br = s_beta[r];
+                const float br = beta[r];
                 float *af = reinterpret_cast<float *>(sm + OFF_AF) + r * LDF + 32 * half;
                 for (int e = 0; e < 32; e += 4) {
                     float4 x;
@@ -391,12 +404,17 @@ __global__ void __launch_bounds__(NT, 1)
                     *reinterpret_cast<uint4 *>(sm + OFF_Y + sw(j, 4 * half + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
+            const float *egm = vec(par, VEC_EGM);
+            const float *ecm_prev = vec(par ^ 1, VEC_ECM);
             for (int p = 0; p < 2; ++p) {
                 const uint32_t col = TS + 64 * half + 32 * p;
                 ptx::tmem_ld32(tl + col, v);
                 ptx::tmem_wait_ld();
-                for (int e = 0; e < 32; ++e)
-                    v[e] = __float_as_uint(__uint_as_float(v[e]) * s_gam[64 * half + 32 * p + e]);
+                for (int e = 0; e < 32; ++e) {
+                    const int c = 64 * half + 32 * p + e;
+                    const float f = ci > 0 ? ecm_prev[c] * egm[c] : egm[c];
+                    v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+                }
                 ptx::tmem_st32(tl + col, v);
             }
             ptx::tmem_wait_st();
@@ -409,59 +427,82 @@ __global__ void __launch_bounds__(NT, 1)
             load_v(s_next);
             ++n_v;
         }
-
-        // ---- T = (I + A)^{-1} Diag(beta): 16x16 diagonal blocks, then the blocks
-        // below them by distance from the diagonal.  Thread (row r, 4-column group jq).
+        // ---- T = (I + A)^{-1} Diag(beta).  X = (I + A)^{-1} in 16x16 blocks: the four
+        // diagonal blocks by column substitution in registers (one warp each), then
+        // E_bk = X_bb A_bk for k < b, then the blocks below the diagonal by distance d,
+        // X_{b,b-d} = -sum_{k=b-d}^{b-1} E_bk X_{k,b-d}.
         {
-            float *Af = reinterpret_cast<float *>(sm + OFF_AF);
+            const float *Af = reinterpret_cast<const float *>(sm + OFF_AF);
             float *X = reinterpret_cast<float *>(sm + OFF_XF);
-            float *W = reinterpret_cast<float *>(sm + OFF_WS);
-            const int b = tid >> 6, rr = (tid >> 2) & 15, jq = tid & 3;
-            const int r = 16 * b + rr;
-            {
-                const int j = 16 * b + 4 * jq;
-                float acc[4];
-                for (int e = 0; e < 4; ++e) acc[e] = (rr == 4 * jq + e) ? 1.f : 0.f;
-                for (int st = 0; st < 16; ++st) {
-                    if (rr == st) *reinterpret_cast<float4 *>(X + r * LDF + j) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-                    ptx::named_barrier(1 + b, 64);
-                    if (rr > st) {
-                        const float av = Af[r * LDF + 16 * b + st];
-                        const float4 xs = *reinterpret_cast<const float4 *>(X + (16 * b + st) * LDF + j);
-                        acc[0] -= av * xs.x;
-                        acc[1] -= av * xs.y;
-                        acc[2] -= av * xs.z;
-                        acc[3] -= av * xs.w;
-                    }
+            float *E = reinterpret_cast<float *>(sm + OFF_EB);
+            if (warp < 4) {
+                const int b = warp, jj = lane & 15;
+                const float *ab = Af + (16 * b) * LDF + 16 * b;
+                float x[16];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jj) ? 1.f : 0.f;
+#pragma unroll
+                for (int ss = 0; ss < 16; ++ss) {  // x[ss] is final: eliminate it below
+#pragma unroll
+                    for (int rr = ss + 1; rr < 16; ++rr) x[rr] = fmaf(-ab[rr * LDF + ss], x[ss], x[rr]);
+                }
+                if (lane < 16) {
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) X[(16 * b + rr) * LDF + 16 * b + jj] = x[rr];
                 }
             }
             __syncthreads();
-            for (int d = 1; d <= 3; ++d) {
-                const int bj = b - d;
-                if (bj >= 0) {
-                    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int kk = 16 * bj; kk < 16 * b; ++kk) {
-                        const float av = Af[r * LDF + kk];
-                        const float4 xv = *reinterpret_cast<const float4 *>(X + kk * LDF + 16 * bj + 4 * jq);
-                        w.x += av * xv.x;
-                        w.y += av * xv.y;
-                        w.z += av * xv.z;
-                        w.w += av * xv.w;
-                    }
-                    *reinterpret_cast<float4 *>(W + r * 16 + 4 * jq) = w;
+            // E block e = b(b-1)/2 + k holds X_bb A_bk: 0:(1,0) 1:(2,0) 2:(2,1) 3:(3,0) 4:(3,1) 5:(3,2)
+            // one task = one row of a 16x16 block, 8 columns (two per block row)
+            if (tid < 6 * 32) {
+                const int e = tid >> 5, row = (tid & 31) >> 1, c8 = 8 * (tid & 1);
+                const int b = e == 0 ? 1 : (e < 3 ? 2 : 3);
+                const int k = e - b * (b - 1) / 2;
+                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {  // X_bb is zero above its diagonal
+                    const float xv = X[(16 * b + row) * LDF + 16 * b + m];
+                    const float4 a0 = *reinterpret_cast<const float4 *>(Af + (16 * b + m) * LDF + 16 * k + c8);
+                    const float4 a1 = *reinterpret_cast<const float4 *>(Af + (16 * b + m) * LDF + 16 * k + c8 + 4);
+                    acc[0] = fmaf(xv, a0.x, acc[0]);
+                    acc[1] = fmaf(xv, a0.y, acc[1]);
+                    acc[2] = fmaf(xv, a0.z, acc[2]);
+                    acc[3] = fmaf(xv, a0.w, acc[3]);
+                    acc[4] = fmaf(xv, a1.x, acc[4]);
+                    acc[5] = fmaf(xv, a1.y, acc[5]);
+                    acc[6] = fmaf(xv, a1.z, acc[6]);
+                    acc[7] = fmaf(xv, a1.w, acc[7]);
                 }
-                __syncthreads();
-                if (bj >= 0) {
-                    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int ss = 0; ss <= rr; ++ss) {
-                        const float xv = X[r * LDF + 16 * b + ss];
-                        const float4 wv = *reinterpret_cast<const float4 *>(W + (16 * b + ss) * 16 + 4 * jq);
-                        o.x -= xv * wv.x;
-                        o.y -= xv * wv.y;
-                        o.z -= xv * wv.z;
-                        o.w -= xv * wv.w;
+                float *eo = E + (e * 16 + row) * LDE + c8;
+                *reinterpret_cast<float4 *>(eo) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                *reinterpret_cast<float4 *>(eo + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            }
+            __syncthreads();
+            for (int d = 1; d <= 3; ++d) {
+                if (tid < (4 - d) * 32) {
+                    const int bj = tid >> 5, b = bj + d, row = (tid & 31) >> 1, c8 = 8 * (tid & 1);
+                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    for (int k = bj; k < b; ++k) {
+                        const float *eb = E + ((b * (b - 1) / 2 + k) * 16 + row) * LDE;
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) {
+                            const float ev = eb[m];
+                            const float *xr = X + (16 * k + m) * LDF + 16 * bj + c8;
+                            const float4 x0 = *reinterpret_cast<const float4 *>(xr);
+                            const float4 x1 = *reinterpret_cast<const float4 *>(xr + 4);
+                            acc[0] = fmaf(ev, x0.x, acc[0]);
+                            acc[1] = fmaf(ev, x0.y, acc[1]);
+                            acc[2] = fmaf(ev, x0.z, acc[2]);
+                            acc[3] = fmaf(ev, x0.w, acc[3]);
+                            acc[4] = fmaf(ev, x1.x, acc[4]);
+                            acc[5] = fmaf(ev, x1.y, acc[5]);
+                            acc[6] = fmaf(ev, x1.z, acc[6]);
+                            acc[7] = fmaf(ev, x1.w, acc[7]);
+                        }
                     }
-                    *reinterpret_cast<float4 *>(X + r * LDF + 16 * bj + 4 * jq) = o;
+                    float *xo = X + (16 * b + row) * LDF + 16 * bj + c8;
+                    *reinterpret_cast<float4 *>(xo) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+                    *reinterpret_cast<float4 *>(xo + 4) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
                 }
                 __syncthreads();
             }
@@ -473,8 +514,8 @@ __global__ void __launch_bounds__(NT, 1)
                     uint32_t pk[4];
                     for (int e2 = 0; e2 < 4; ++e2) {
                         const int i = 8 * ch + 2 * e2;
-                        const float x0 = (i <= rt) ? X[rt * LDF + i] * s_beta[i] : 0.f;
-                        const float x1 = (i + 1 <= rt) ? X[rt * LDF + i + 1] * s_beta[i + 1] : 0.f;
+                        const float x0 = (i <= rt) ? X[rt * LDF + i] * beta[i] : 0.f;
+                        const float x1 = (i + 1 <= rt) ? X[rt * LDF + i + 1] * beta[i + 1] : 0.f;
                         pk[e2] = pack_h2(x0, x1);
                     }
                     *reinterpret_cast<uint4 *>(sm + OFF_T + sw(rt, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -513,41 +554,58 @@ __global__ void __launch_bounds__(NT, 1)
         __syncthreads();
         if (*s_abort) break;
 
-        // ---- M4: S^T += U^T (K e^{g_L-g});  M5: O^T = Z[:, 64:] + U^T P^T.
+        // ---- M4: R += U^T Kb;  M5: O^T = Z[:, 64:] + U^T P^T.  The next chunk's
+        // running sums are formed meanwhile.
         if (tid == 0) {
             ptx::tc_fence_after();
             for (int ks = 0; ks < 4; ++ks)
-                ptx::mma_ss(tbase + TS, ptx::sdesc_sw128(sb + OFF_U + 32 * ks), ptx::sdesc_sw128(sb + OFF_KH + 32 * ks),
-                            IDESC_N128, 1u);
+                ptx::mma_ss(tbase + TS, ptx::sdesc_sw128(sb + OFF_U + 32 * ks),
+                            ptx::sdesc_sw128_mn(sb + OFF_KB + 2048 * ks, 8192, 1024), IDESC_N128_BMN, 1u);
             for (int ks = 0; ks < 4; ++ks)
                 ptx::mma_ss(tbase + TZ + 64, ptx::sdesc_sw128(sb + OFF_U + 32 * ks), ptx::sdesc_sw128(sb + OFF_P + 32 * ks),
                             IDESC_N64, 1u);
             ptx::mma_commit(bar_mma);
             ++n_mma;
         }
+        if (has_next) scan(ci + 1, beta_next);
         wait_on(bar_mma, w_mma);
         ptx::tc_fence_after();
-        {  // E4: next S^T operand, outputs of this chunk.
-            uint32_t v[32], pk[32];
-            for (int p = 0; p < 2; ++p) {
-                ptx::tmem_ld32(tl + TS + 64 * half + 32 * p, v);
-                ptx::tmem_wait_ld();
-                for (int e = 0; e < 16; ++e)
-                    pk[16 * p + e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+        {  // E4: next Sop = R Diag(e^{g_L - g_m} e^{g_m'}), outputs of this chunk.
+            uint32_t v[32], w[32], pk[32];
+            if (has_next) {
+                const float *ecm = vec(par, VEC_ECM);
+                const float *egm_next = vec(par ^ 1, VEC_EGM);
+                for (int p = 0; p < 2; ++p) {
+                    ptx::tmem_ld32(tl + TS + 64 * half + 32 * p, w);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int c = 64 * half + 32 * p + 2 * e;
+                        pk[16 * p + e] = pack_h2(__uint_as_float(w[2 * e]) * (ecm[c] * egm_next[c]),
+                                                 __uint_as_float(w[2 * e + 1]) * (ecm[c + 1] * egm_next[c + 1]));
+                    }
+                }
+                ptx::tmem_st32(tl + TSOP + 32 * half, pk);
             }
-            ptx::tmem_st32(tl + TSOP + 32 * half, pk);
             ptx::tmem_ld32(tl + TZ + 64 + 32 * half, v);
             ptx::tmem_wait_ld();
-            __nv_bfloat16 *op = static_cast<__nv_bfloat16 *>(a.o);
-            for (int e = 0; e < 32; ++e) {
-                const int r = 32 * half + e;
-                if (r < L) op[(size_t(s + r) * H + h) * D + row] = __float2bfloat16_rn(__uint_as_float(v[e]));
-            }
+            // stage O[r][j] (bf16, row-major) in the Y^T tile, which M3 has consumed
+            __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_Y);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) stage[(32 * half + e) * D + row] = __float2bfloat16_rn(__uint_as_float(v[e]));
             ptx::tmem_wait_st();
         }
         ptx::tc_fence_before();
         __syncthreads();
         if (*s_abort) break;
+        {  // rows r < L of the staged outputs, 16 bytes per thread
+            const uint4 *src = reinterpret_cast<const uint4 *>(sm + OFF_Y);
+            char *dst = static_cast<char *>(a.o) + (size_t(s) * H + h) * D * 2;
+            for (int t = tid; t < L * 16; t += NT) {
+                const int r = t >> 4, q = t & 15;
+                *reinterpret_cast<uint4 *>(dst + size_t(r) * H * D * 2 + q * 16) = src[r * 16 + q];
+            }
+        }
     }
 
     if (*s_abort && tid == 0) {  // drain what is still in flight (each wait bounded)
@@ -556,16 +614,18 @@ __global__ void __launch_bounds__(NT, 1)
         while (w_v < n_v) ptx::mbar_wait_bounded(bar_v, uint32_t(w_v++) & 1u, kWaitCycles);
         while (w_mma < n_mma) ptx::mbar_wait_bounded(bar_mma, uint32_t(w_mma++) & 1u, kWaitCycles);
     }
-    // Final state S_final[c][j] = S^T[j][c].
+    // Final state S_final[c][j] = R[j][c] e^{g_L - g_m}[c] of the last chunk.
     if (!*s_abort) {
         ptx::tc_fence_after();
+        const float *ecm_last = vec((nchunks - 1) & 1, VEC_ECM);
         uint32_t v[32];
         for (int p = 0; p < 2; ++p) {
             ptx::tmem_ld32(tl + TS + 64 * half + 32 * p, v);
             ptx::tmem_wait_ld();
             for (int e = 0; e < 32; ++e) {
                 const int c = 64 * half + 32 * p + e;
-                a.S_final[(unit * D + c) * D + row] = __uint_as_float(v[e]);
+                const float f = nchunks > 0 ? ecm_last[c] : 1.f;
+                a.S_final[(unit * D + c) * D + row] = __uint_as_float(v[e]) * f;
             }
         }
     }

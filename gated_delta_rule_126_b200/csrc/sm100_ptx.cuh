@@ -128,7 +128,21 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory matrix descriptor, MN-major operand in the 128-byte swizzle
+// layout: 64 MN elements (128 bytes) per row, one row per K index, 8-row K groups
+// `sbo` bytes apart and 64-element MN blocks `lbo` bytes apart.
+__device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= uint64_t((saddr >> 4) & 0x3FFFu);
+    d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+    d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+    d |= uint64_t(1u) << 46;
+    d |= uint64_t(2u) << 61;
+    return d;
+}
+
 // Instruction descriptor of kind::f16: fp16 A and B (both K-major), fp32 D.
+// Bit 16 set marks B as MN-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
     return (1u << 4)                       // D format: F32
          | (0u << 7) | (0u << 10)          // A, B format: F16
