@@ -136,6 +136,37 @@ KDA_API kda_status_t kda_decode_step(const void *q, const void *k, const void *v
                              int B, int H, int d_k, int d_v, void *o, kda_stream_t stream);
 
 /*
+ * kda_prefill_noalloc -- kda_prefill for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart: this is a deployment variant of kda_prefill.
+ * Some callers cannot call cudaMalloc where they run the operator (a host
+ * framework that owns every allocation, a plug-in handed only its inputs and
+ * outputs, a path where allocating would synchronise or fail under memory
+ * pressure).  This call takes the same arguments as kda_prefill minus the
+ * workspace and allocates nothing, with no library routine that allocates: its
+ * scratch (status word and sequence order) is one file-scope device array of
+ * 256 + 4 * KDA_NOALLOC_MAX_SEQS bytes that every GPU loading the library holds
+ * until the process exits.
+ *
+ * - num_seqs > KDA_NOALLOC_MAX_SEQS returns KDA_ERR_WORKSPACE before anything is
+ *   queued; every other check and result is kda_prefill's.
+ * - The first call on a device looks up the array's device address for that
+ *   device (once per device, with that device current); make that first call
+ *   before any stream capture.
+ * - All calls share the array and it keeps the last call's contents (the status
+ *   word is cleared at the start of each call): calls that may overlap on the GPU,
+ *   on any streams, race on it and must be ordered by the caller.
+ * - A kernel-side error flag set during this call is not reported back; use
+ *   kda_prefill with a workspace and kda_workspace_status to observe it.
+ */
+#define KDA_NOALLOC_MAX_SEQS 65536
+KDA_API kda_status_t kda_prefill_noalloc(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                                 const float *log_alpha, const float *beta, const float *S0,
+                                 const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                                 int num_seqs, int H, int d_k, int d_v, int chunk,
+                                 void *o, float *S_final, kda_stream_t stream);
+
+/*
  * kda_workspace_status -- waits for `stream`, then reports whether a kernel of
  * the last kda_prefill call that used `workspace` flagged an internal error
  * (KDA_ERR_DEVICE_FAULT, e.g. a bounded wait that ran out) and clears the flag.

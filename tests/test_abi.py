@@ -29,8 +29,8 @@ def declared_symbols():
 
 def test_header_declares_the_abi():
     assert declared_symbols() == sorted([
-        "kda_decode_step", "kda_prefill", "kda_prefill_workspace_size", "kda_status_string",
-        "kda_version", "kda_workspace_status"])
+        "kda_decode_step", "kda_prefill", "kda_prefill_noalloc", "kda_prefill_workspace_size",
+        "kda_status_string", "kda_version", "kda_workspace_status"])
 
 
 def test_library_exports_every_declared_symbol(lib):
