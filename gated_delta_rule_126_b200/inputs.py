@@ -79,6 +79,11 @@ WORKLOADS = {
     "batched_prefill": Workload("batched_prefill", "prefill", H=32, dk=128, dv=128,
                                 dtype="bf16", s0_std=0.0, seed=SEED_BASE + 2, chunk=64,
                                 seqlens=(8192,) * 8),
+    # a quarter of the batched workload (above L2, about 0.8 GB of inputs): the
+    # small case the profiler captures
+    "batched_prefill_2x8192": Workload("batched_prefill_2x8192", "prefill", H=32, dk=128, dv=128,
+                                       dtype="bf16", s0_std=0.0, seed=SEED_BASE + 2, chunk=64,
+                                       seqlens=(8192,) * 2),
     "decode": Workload("decode", "decode", H=32, dk=128, dv=128, dtype="bf16",
                        s0_std=S0_STD, seed=SEED_BASE + 3, batch=256, steps=64),
     "longctx_varlen_prefill": Workload("longctx_varlen_prefill", "prefill", H=32, dk=128,
