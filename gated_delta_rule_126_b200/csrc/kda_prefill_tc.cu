@@ -23,9 +23,9 @@
 //     M4  R         += U^T Kb      (Kb read as an MN-major operand)  N=128 K=64
 //     M5  Z[:, 64:] += U^T P^T  ( = O^T )                   N=64  K=64
 //   TMEM holds R = S^T Diag(e^{g_m - g_L}) of the previous chunk rather than S^T:
-//   the per-channel factors e^{g_L - g_m} and e^{g_m} then fold into one rescale
-//   of R per chunk and into the fp16 pack of the next Sop, so no K e^{g},
-//   Q e^{g} or (K e^{g_L - g})^T tile is built.
+//   the per-channel factors e^{g_L - g_m} and e^{g_m} then fold into one pass over
+//   R at the start of each chunk, which also packs Sop, so no K e^{g}, Q e^{g} or
+//   (K e^{g_L - g})^T tile is built.
 // * Operands are fp16 (fp32 accumulation): the S-dependent chain keeps the
 //   relative error near fp16's 2^-11, which the parity bounds need (bf16 operands
 //   do not meet them).  Sop lives in TMEM (fp16 pairs per column).
@@ -243,10 +243,9 @@ __global__ void __launch_bounds__(NT, 1)
     if (nchunks > 0) scan(0, load_beta(0));
     __syncthreads();
 
-    // Initial state: R = S0^T (fp32) and Sop = S0^T Diag(e^{g_m}) of chunk 0 (fp16).
+    // Initial state: R = S0^T (fp32).
     {
-        const float *egm0 = vec(0, VEC_EGM);
-        uint32_t v[32], pk[32];
+        uint32_t v[32];
         for (int p = 0; p < 2; ++p) {
             for (int e = 0; e < 32; ++e) {
                 const int c = 64 * half + 32 * p + e;
@@ -254,12 +253,7 @@ __global__ void __launch_bounds__(NT, 1)
                 v[e] = __float_as_uint(x);
             }
             ptx::tmem_st32(tl + TS + 64 * half + 32 * p, v);
-            for (int e = 0; e < 16; ++e) {
-                const int c = 64 * half + 32 * p + 2 * e;
-                pk[16 * p + e] = pack_h2(__uint_as_float(v[2 * e]) * egm0[c], __uint_as_float(v[2 * e + 1]) * egm0[c + 1]);
-            }
         }
-        if (nchunks > 0) ptx::tmem_st32(tl + TSOP + 32 * half, pk);
         ptx::tmem_wait_st();
     }
     ptx::tc_fence_before();
@@ -274,6 +268,32 @@ __global__ void __launch_bounds__(NT, 1)
         const float *gm = vec(par, VEC_GM);
         const float *beta = vec(par, VEC_BETA);
         const float beta_next = load_beta(ci + 1);
+
+        // ---- E0: R *= e^{g_L - g_m}(previous chunk) e^{g_m}, giving S^T Diag(e^{g_m}),
+        // and its fp16 copy Sop, the A operand of M2 (one pass over R).
+        {
+            const float *egm = vec(par, VEC_EGM);
+            const float *ecm_prev = vec(par ^ 1, VEC_ECM);
+            uint32_t v[32], pk[32];
+            for (int p = 0; p < 2; ++p) {
+                const uint32_t col = TS + 64 * half + 32 * p;
+                ptx::tmem_ld32(tl + col, v);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int c = 64 * half + 32 * p + e;
+                    const float f = ci > 0 ? ecm_prev[c] * egm[c] : egm[c];
+                    v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+                }
+                ptx::tmem_st32(tl + col, v);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[16 * p + e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+            }
+            ptx::tmem_st32(tl + TSOP + 32 * half, pk);
+            ptx::tmem_wait_st();
+        }
+        ptx::tc_fence_before();
 
         // ---- P2: Kt, Qt (in place over the raw k|q rows) and Kb; one (token row,
         // 32-channel quarter) per thread.
@@ -355,7 +375,7 @@ __global__ void __launch_bounds__(NT, 1)
         wait_on(bar_v, w_v);
 
         // ---- E1: A rows -> fp32 scratch, P rows -> fp16 operand.
-        // ---- E2: Y^T = V^T - Z[:, :64] -> fp16 operand; R *= e^{g_L - g_m}(prev) e^{g_m}.
+        // ---- E2: Y^T = V^T - Z[:, :64] -> fp16 operand.
         {
             uint32_t v[32];
             ptx::tmem_ld32(tl + TAP + 32 * half, v);
@@ -404,20 +424,6 @@ __global__ void __launch_bounds__(NT, 1)
                     *reinterpret_cast<uint4 *>(sm + OFF_Y + sw(j, 4 * half + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
-            const float *egm = vec(par, VEC_EGM);
-            const float *ecm_prev = vec(par ^ 1, VEC_ECM);
-            for (int p = 0; p < 2; ++p) {
-                const uint32_t col = TS + 64 * half + 32 * p;
-                ptx::tmem_ld32(tl + col, v);
-                ptx::tmem_wait_ld();
-                for (int e = 0; e < 32; ++e) {
-                    const int c = 64 * half + 32 * p + e;
-                    const float f = ci > 0 ? ecm_prev[c] * egm[c] : egm[c];
-                    v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-                }
-                ptx::tmem_st32(tl + col, v);
-            }
-            ptx::tmem_wait_st();
         }
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_before();
@@ -570,30 +576,14 @@ __global__ void __launch_bounds__(NT, 1)
         if (has_next) scan(ci + 1, beta_next);
         wait_on(bar_mma, w_mma);
         ptx::tc_fence_after();
-        {  // E4: next Sop = R Diag(e^{g_L - g_m} e^{g_m'}), outputs of this chunk.
-            uint32_t v[32], w[32], pk[32];
-            if (has_next) {
-                const float *ecm = vec(par, VEC_ECM);
-                const float *egm_next = vec(par ^ 1, VEC_EGM);
-                for (int p = 0; p < 2; ++p) {
-                    ptx::tmem_ld32(tl + TS + 64 * half + 32 * p, w);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int c = 64 * half + 32 * p + 2 * e;
-                        pk[16 * p + e] = pack_h2(__uint_as_float(w[2 * e]) * (ecm[c] * egm_next[c]),
-                                                 __uint_as_float(w[2 * e + 1]) * (ecm[c + 1] * egm_next[c + 1]));
-                    }
-                }
-                ptx::tmem_st32(tl + TSOP + 32 * half, pk);
-            }
+        {  // E4: outputs of this chunk.
+            uint32_t v[32];
             ptx::tmem_ld32(tl + TZ + 64 + 32 * half, v);
             ptx::tmem_wait_ld();
             // stage O[r][j] (bf16, row-major) in the Y^T tile, which M3 has consumed
             __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_Y);
 #pragma unroll
             for (int e = 0; e < 32; ++e) stage[(32 * half + e) * D + row] = __float2bfloat16_rn(__uint_as_float(v[e]));
-            ptx::tmem_wait_st();
         }
         ptx::tc_fence_before();
         __syncthreads();
