@@ -10,7 +10,7 @@
 //   P_ri = <q_r e^{g_r - g_i}, k_i> (i <= r)
 //   U = T (V - (K e^{g}) S),   O = (Q e^{g}) S + P U,   S <- Diag(e^{g_L}) S + (K e^{g_L - g})^T U
 //
-// Design (one CTA of 256 threads per (sequence, head), walking its chunks):
+// Design (one CTA of 384 threads per (sequence, head), walking its chunks):
 // * The fp32 state is kept TRANSPOSED in tensor memory (TMEM lane = value column
 //   j, 128 lanes) for the whole sequence, so every product of the chunk step is a
 //   128-row UMMA with d_v on the M side.  With Kt = K e^{g-g_m}, Qt = Q e^{g-g_m},
@@ -26,15 +26,21 @@
 //   the per-channel factors e^{g_L - g_m} and e^{g_m} then fold into one pass over
 //   R at the start of each chunk, which also packs Sop, so no K e^{g}, Q e^{g} or
 //   (K e^{g_L - g})^T tile is built.
+// * Two warp groups work on different chunks at once.  The prep group (warps
+//   4-11) builds chunk c + 1 -- running sums, decayed rows, M1, A and P, the
+//   triangular solve for T -- while the state group (warps 0-3) runs chunk c --
+//   the pass over R, M2, Y, M3, U, M4/M5 and the outputs.  They hand buffers over
+//   through release/acquire progress counters in shared memory; the decayed-row
+//   (Kb) and P tiles are double-buffered by chunk parity.
 // * Operands are fp16 (fp32 accumulation): the S-dependent chain keeps the
 //   relative error near fp16's 2^-11, which the parity bounds need (bf16 operands
 //   do not meet them).  Sop lives in TMEM (fp16 pairs per column).
 // * q, k, v and log alpha tiles arrive by TMA in the 128-byte swizzled layout that
 //   the UMMA descriptors use, so the decayed operand rows are built in place.
 // * T is formed in fp32 by a blocked (16x16) forward substitution in shared memory.
-// * The running sums of the next chunk are formed while M4/M5 run.
-// * All waits are bounded: a wait that runs out sets the workspace error flag and
-//   the CTA stops after its next barrier.
+// * Every wait is bounded: one that runs out sets the workspace error flag and
+//   both groups stop at their next group barrier (decided uniformly by a
+//   barrier-or), drain what they have in flight and free TMEM.
 #include <cuda.h>
 
 #include "kda_internal.h"
@@ -45,22 +51,25 @@ namespace {
 
 constexpr int C = 64;    // chunk
 constexpr int D = 128;   // d_k = d_v
-constexpr int NT = 256;  // threads
+constexpr int NS = 128;  // state group: warps 0-3
+constexpr int NP = 256;  // prep group: warps 4-11
+constexpr int NT = NS + NP;
+constexpr uint32_t BAR_S = 1, BAR_P = 2;  // named barriers of the two groups
 
 // Shared memory map (bytes from a 1024-aligned base).
 constexpr uint32_t OFF_QK = 0;        // raw k|q boxes -> [Kt; Qt]  (128 x 128 fp16, K-major)
 constexpr uint32_t OFF_LA = 32768;    // raw log alpha boxes -> g (fp32, 64 x 128)
 constexpr uint32_t OFF_V = 65536;     // raw v boxes (bf16, 64 x 128)
-constexpr uint32_t OFF_KB = 81920;    // Kb (64 x 128 fp16): B of M1 (K-major) and of M4 (MN-major)
-constexpr uint32_t OFF_SCR = 98304;   // fp32 scratch of the triangular solve
+constexpr uint32_t OFF_KB = 81920;    // Kb (64 x 128 fp16), two buffers
+constexpr uint32_t OFF_SCR = 114688;  // fp32 scratch of the triangular solve
 constexpr int LDF = 68;
 constexpr int LDE = 20;
 constexpr uint32_t OFF_AF = OFF_SCR;
 constexpr uint32_t OFF_XF = OFF_AF + 64 * LDF * 4;
 constexpr uint32_t OFF_EB = OFF_XF + 64 * LDF * 4;  // six 16x16 blocks X_bb A_bk
-constexpr uint32_t OFF_P = 141312;    // P (64 x 64 fp16)
+constexpr uint32_t OFF_P = 157696;    // P (64 x 64 fp16), two buffers
 static_assert(OFF_EB + 6 * 16 * LDE * 4 <= OFF_P, "solve scratch overflows");
-constexpr uint32_t OFF_T = OFF_P + 8192;     // T (64 x 64 fp16)
+constexpr uint32_t OFF_T = OFF_P + 16384;    // T (64 x 64 fp16)
 constexpr uint32_t OFF_Y = OFF_T + 8192;     // Y^T (128 x 64 fp16); later the bf16 output tile
 constexpr uint32_t OFF_U = OFF_Y + 16384;    // U^T (128 x 64 fp16)
 constexpr uint32_t OFF_VEC = OFF_U + 16384;  // per-chunk vectors, two buffers (chunk parity)
@@ -70,17 +79,23 @@ constexpr uint32_t VEC_ECM = 1024;    // e^{g_L - g_m}
 constexpr uint32_t VEC_BETA = 1536;   // beta                 64 f32
 constexpr uint32_t VEC_BYTES = 1792;
 constexpr uint32_t OFF_HALF = OFF_VEC + 2 * VEC_BYTES;  // running sum over the first 32 tokens
-constexpr uint32_t OFF_BAR = OFF_HALF + 512;            // 4 mbarriers
-constexpr uint32_t OFF_MISC = OFF_BAR + 32;             // tmem base, abort flag
+constexpr uint32_t OFF_BAR = OFF_HALF + 512;            // mbarriers
+constexpr int NBAR = 7;
+constexpr int B_QK = 0, B_LA = 1, B_V = 2, B_M1 = 3, B_M2 = 4, B_M3 = 5, B_M45 = 6;
+constexpr uint32_t OFF_CNT = OFF_BAR + 8 * NBAR;        // progress counters
+constexpr int CNT_ROWS = 0, CNT_TP = 1, CNT_E0 = 2, CNT_M2 = 3, CNT_M3 = 4, CNT_M45 = 5;
+constexpr uint32_t OFF_ISS = OFF_CNT + 32;              // phases issued / waited per mbarrier
+constexpr uint32_t OFF_WT = OFF_ISS + 4 * NBAR;
+constexpr uint32_t OFF_MISC = OFF_WT + 4 * NBAR;        // tmem base, abort flag
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // + alignment slack
 
 // Tensor memory columns.
-constexpr uint32_t TS = 0;      // R (fp32)          128 cols
-constexpr uint32_t TZ = 128;    // Z fp32            128 cols
-constexpr uint32_t TU = 256;    // U^T fp32           64 cols
-constexpr uint32_t TAP = 320;   // [A; P] raw fp32    64 cols
-constexpr uint32_t TSOP = 384;  // Sop fp16           64 cols
+constexpr uint32_t TS = 0;      // R (fp32)          128 cols   state group
+constexpr uint32_t TZ = 128;    // Z fp32            128 cols   state group
+constexpr uint32_t TU = 256;    // U^T fp32           64 cols   state group
+constexpr uint32_t TAP = 320;   // [A; P] raw fp32    64 cols   prep group
+constexpr uint32_t TSOP = 384;  // Sop fp16           64 cols   state group
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t IDESC_N64 = ptx::idesc_f16_f32(128, 64);
@@ -116,12 +131,13 @@ __global__ void __launch_bounds__(NT, 1)
     const int seq = a.order[blockIdx.x / H];
     const int bos = a.cu_seqlens[seq], eos = a.cu_seqlens[seq + 1];
     const int nchunks = (eos - bos + C - 1) / C;
+    const size_t unit = size_t(seq) * H + h;
 
     auto vec = [&](int par, uint32_t field) { return reinterpret_cast<float *>(sm + OFF_VEC + par * VEC_BYTES + field); };
-    uint64_t *bar_qk = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-    uint64_t *bar_la = bar_qk + 1;
-    uint64_t *bar_v = bar_qk + 2;
-    uint64_t *bar_mma = bar_qk + 3;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+    uint32_t *cnt = reinterpret_cast<uint32_t *>(sm + OFF_CNT);
+    uint32_t *iss = reinterpret_cast<uint32_t *>(sm + OFF_ISS);
+    uint32_t *wt = reinterpret_cast<uint32_t *>(sm + OFF_WT);
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     int *s_abort = reinterpret_cast<int *>(sm + OFF_MISC + 4);
 
@@ -130,10 +146,12 @@ __global__ void __launch_bounds__(NT, 1)
         ptx::tmem_relinquish();
     }
     if (tid == 32) {
-        ptx::mbar_init(bar_qk, 1);
-        ptx::mbar_init(bar_la, 1);
-        ptx::mbar_init(bar_v, 1);
-        ptx::mbar_init(bar_mma, 1);
+        for (int b = 0; b < NBAR; ++b) {
+            ptx::mbar_init(bars + b, 1);
+            iss[b] = 0;
+            wt[b] = 0;
+        }
+        for (int i = 0; i < 8; ++i) cnt[i] = 0;
         ptx::fence_mbar_init();
         *s_abort = 0;
         ptx::prefetch_tmap(&maps.q);
@@ -147,477 +165,530 @@ __global__ void __launch_bounds__(NT, 1)
     const uint32_t tbase = *s_tmem;
 
     auto load_qk = [&](int s) {
-        ptx::mbar_arrive_expect_tx(bar_qk, 4 * 8192);
-        ptx::tma_load_3d(sm + OFF_QK, &maps.k, bar_qk, 0, h, s);
-        ptx::tma_load_3d(sm + OFF_QK + 8192, &maps.q, bar_qk, 0, h, s);
-        ptx::tma_load_3d(sm + OFF_QK + 16384, &maps.k, bar_qk, 64, h, s);
-        ptx::tma_load_3d(sm + OFF_QK + 24576, &maps.q, bar_qk, 64, h, s);
+        ptx::mbar_arrive_expect_tx(bars + B_QK, 4 * 8192);
+        ptx::tma_load_3d(sm + OFF_QK, &maps.k, bars + B_QK, 0, h, s);
+        ptx::tma_load_3d(sm + OFF_QK + 8192, &maps.q, bars + B_QK, 0, h, s);
+        ptx::tma_load_3d(sm + OFF_QK + 16384, &maps.k, bars + B_QK, 64, h, s);
+        ptx::tma_load_3d(sm + OFF_QK + 24576, &maps.q, bars + B_QK, 64, h, s);
+        ++iss[B_QK];
     };
     auto load_la = [&](int s) {
-        ptx::mbar_arrive_expect_tx(bar_la, 4 * 8192);
-        for (int b = 0; b < 4; ++b) ptx::tma_load_3d(sm + OFF_LA + b * 8192, &maps.la, bar_la, 32 * b, h, s);
+        ptx::mbar_arrive_expect_tx(bars + B_LA, 4 * 8192);
+        for (int b = 0; b < 4; ++b) ptx::tma_load_3d(sm + OFF_LA + b * 8192, &maps.la, bars + B_LA, 32 * b, h, s);
+        ++iss[B_LA];
     };
     auto load_v = [&](int s) {
-        ptx::mbar_arrive_expect_tx(bar_v, 2 * 8192);
-        ptx::tma_load_3d(sm + OFF_V, &maps.v, bar_v, 0, h, s);
-        ptx::tma_load_3d(sm + OFF_V + 8192, &maps.v, bar_v, 64, h, s);
+        ptx::mbar_arrive_expect_tx(bars + B_V, 2 * 8192);
+        ptx::tma_load_3d(sm + OFF_V, &maps.v, bars + B_V, 0, h, s);
+        ptx::tma_load_3d(sm + OFF_V + 8192, &maps.v, bars + B_V, 64, h, s);
+        ++iss[B_V];
+    };
+    auto commit = [&](int b) {
+        ptx::mma_commit(bars + b);
+        ++iss[b];
     };
     auto fail = [&]() {
         atomicExch(&a.status->flag, 1u);
         *s_abort = 1;
     };
-    // Wait for the next phase of `bar`; `waited` counts completed phases and only
-    // advances on success, so an abort can drain the phase that timed out.
-    auto wait_on = [&](uint64_t *bar, int &waited) {
-        if (ptx::mbar_wait_bounded(bar, uint32_t(waited) & 1u, kWaitCycles))
-            ++waited;
-        else
-            fail();
-    };
-
-    // Loads and MMA groups issued (thread 0) and waited for (every thread); on an
-    // abort the CTA waits, bounded, for whatever it still has in flight.
-    int n_qk = 0, n_la = 0, n_v = 0, n_mma = 0;
-    int w_qk = 0, w_la = 0, w_v = 0, w_mma = 0;
-    if (tid == 0 && nchunks > 0) {
-        load_qk(bos);
-        load_la(bos);
-        load_v(bos);
-        n_qk = n_la = n_v = 1;
-    }
-
-    // P1 of chunk `ci`: g = running sum of log alpha per channel, in place over the
-    // log alpha tile, and the chunk's vectors (buffer ci & 1).  Thread (channel c,
-    // half hf) scans tokens [32 hf, 32 hf + 32); the second half then adds the
-    // first half's total.  The middle token (L - 1) / 2 is always in the first half.
-    // `bval` is this thread's beta of the chunk (threads < 64), loaded ahead of time.
-    auto scan = [&](int ci, float bval) {
-        const int s = bos + ci * C, L = min(C, eos - s);
-        float *gm = vec(ci & 1, VEC_GM), *egm = vec(ci & 1, VEC_EGM), *ecm = vec(ci & 1, VEC_ECM);
-        float *beta = vec(ci & 1, VEC_BETA);
-        wait_on(bar_la, w_la);
-        const int c = tid & 127, hf = tid >> 7, box = c >> 5, lc = c & 31, lch = lc >> 2;
-        uint8_t *col = sm + OFF_LA + box * 8192 + (lc & 3) * 4;
-        float *s_half = reinterpret_cast<float *>(sm + OFF_HALF);
-        const int rm = (L - 1) >> 1;
-        float x[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int r = 32 * hf + i;
-            x[i] = (r < L) ? *reinterpret_cast<const float *>(col + sw(r, lch)) : 0.f;
-        }
-#pragma unroll
-        for (int i = 1; i < 32; ++i) x[i] += x[i - 1];
-        if (hf == 0) {
-            float gmid = 0.f;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) gmid = (i == rm) ? x[i] : gmid;
-            s_half[c] = x[31];
-            gm[c] = gmid;
-            egm[c] = expf(gmid);
-        }
-        if (tid < C) beta[tid] = bval;
-        __syncthreads();
-        if (hf == 1) {
-            const float off = s_half[c];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] += off;
-            ecm[c] = expf(x[31] - gm[c]);
-        }
-#pragma unroll
-        for (int i = 0; i < 32; ++i) *reinterpret_cast<float *>(col + sw(32 * hf + i, lch)) = x[i];
-    };
-
-    // Thread <-> TMEM mapping for the epilogues: warp w reads lanes 32*(w%4)...,
-    // its column half is w/4.  `row` is the TMEM lane = value column j.
-    const int qd = warp & 3, half = warp >> 2;
-    const int row = qd * 32 + lane;
-    const uint32_t tl = tbase + (uint32_t(qd * 32) << 16);
-    const size_t unit = size_t(seq) * H + h;
-
-    // beta of a chunk is read from global memory one chunk ahead (a register)
-    auto load_beta = [&](int ci) {
-        const int s = bos + ci * C;
-        return (tid < C && ci < nchunks && s + tid < eos) ? a.beta[size_t(s + tid) * H + h] : 0.f;
-    };
-    if (nchunks > 0) scan(0, load_beta(0));
-    __syncthreads();
-
-    // Initial state: R = S0^T (fp32).
-    {
-        uint32_t v[32];
-        for (int p = 0; p < 2; ++p) {
-            for (int e = 0; e < 32; ++e) {
-                const int c = 64 * half + 32 * p + e;
-                const float x = a.S0 ? a.S0[(unit * D + c) * D + row] : 0.f;
-                v[e] = __float_as_uint(x);
+    // Wait for phase `phase` of mbarrier b (bounded, gives up on an abort).
+    // `leader` records the wait for the drain on abort.
+    auto mwait = [&](int b, uint32_t phase, bool leader) {
+        const long long t0 = clock64();
+        while (!ptx::mbar_try_wait(bars + b, phase & 1u)) {
+            if (*reinterpret_cast<volatile int *>(s_abort) || clock64() - t0 > kWaitCycles) {
+                fail();
+                return false;
             }
-            ptx::tmem_st32(tl + TS + 64 * half + 32 * p, v);
         }
-        ptx::tmem_wait_st();
-    }
-    ptx::tc_fence_before();
-    __syncthreads();
+        if (leader) wt[b] = phase + 1;
+        return true;
+    };
+    // Wait until progress counter i reaches `target` (bounded, gives up on an abort).
+    auto cwait = [&](int i, uint32_t target) {
+        if (ptx::ld_acquire(cnt + i) >= target) return true;
+        const long long t0 = clock64();
+        while (ptx::ld_acquire(cnt + i) < target) {
+            if (*reinterpret_cast<volatile int *>(s_abort) || clock64() - t0 > kWaitCycles) {
+                fail();
+                return false;
+            }
+            __nanosleep(20);
+        }
+        return true;
+    };
 
-    for (int ci = 0; ci < nchunks; ++ci) {
-        const int s = bos + ci * C;
-        const int L = min(C, eos - s);
-        const bool has_next = ci + 1 < nchunks;
-        const int s_next = s + C;
-        const int par = ci & 1;
-        const float *gm = vec(par, VEC_GM);
-        const float *beta = vec(par, VEC_BETA);
-        const float beta_next = load_beta(ci + 1);
-
-        // ---- E0: R *= e^{g_L - g_m}(previous chunk) e^{g_m}, giving S^T Diag(e^{g_m}),
-        // and its fp16 copy Sop, the A operand of M2 (one pass over R).
-        {
-            const float *egm = vec(par, VEC_EGM);
-            const float *ecm_prev = vec(par ^ 1, VEC_ECM);
-            uint32_t v[32], pk[32];
-            for (int p = 0; p < 2; ++p) {
-                const uint32_t col = TS + 64 * half + 32 * p;
-                ptx::tmem_ld32(tl + col, v);
-                ptx::tmem_wait_ld();
-#pragma unroll
+    if (warp < 4) {
+        // =================================================================== state group
+        const int row = tid;  // TMEM lane = value column j
+        const uint32_t tl = tbase + (uint32_t(warp * 32) << 16);
+        const bool leader = tid == 0;
+        if (leader && nchunks > 0) load_v(bos);
+        {  // R = S0^T
+            uint32_t v[32];
+            for (int p = 0; p < 4; ++p) {
                 for (int e = 0; e < 32; ++e) {
-                    const int c = 64 * half + 32 * p + e;
-                    const float f = ci > 0 ? ecm_prev[c] * egm[c] : egm[c];
-                    v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+                    const int c = 32 * p + e;
+                    v[e] = __float_as_uint(a.S0 ? a.S0[(unit * D + c) * D + row] : 0.f);
                 }
-                ptx::tmem_st32(tl + col, v);
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pk[16 * p + e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                ptx::tmem_st32(tl + TS + 32 * p, v);
             }
-            ptx::tmem_st32(tl + TSOP + 32 * half, pk);
             ptx::tmem_wait_st();
         }
-        ptx::tc_fence_before();
+        for (int ci = 0; ci < nchunks; ++ci) {
+            const int s = bos + ci * C;
+            const int L = min(C, eos - s);
+            const bool has_next = ci + 1 < nchunks;
+            const int par = ci & 1;
 
-        // ---- P2: Kt, Qt (in place over the raw k|q rows) and Kb; one (token row,
-        // 32-channel quarter) per thread.
-        wait_on(bar_qk, w_qk);
-        {
-            const int r = tid & 63, part = tid >> 6, kb = part >> 1;
-            const bool valid = r < L;
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const int ch = (part & 1) * 4 + qq;
-                const uint32_t ph16 = sw(r, ch);
-                const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + OFF_QK + kb * 16384 + ph16);
-                const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + OFF_QK + kb * 16384 + 8192 + ph16);
-                const int c0 = 64 * kb + 8 * ch;
-                const int box = c0 >> 5, lch = (c0 & 31) >> 2;
-                const float4 ga = *reinterpret_cast<const float4 *>(sm + OFF_LA + box * 8192 + sw(r, lch));
-                const float4 gb = *reinterpret_cast<const float4 *>(sm + OFF_LA + box * 8192 + sw(r, lch + 1));
-                const float4 m0 = *reinterpret_cast<const float4 *>(gm + c0);
-                const float4 m1 = *reinterpret_cast<const float4 *>(gm + c0 + 4);
-                const float dg[8] = {ga.x - m0.x, ga.y - m0.y, ga.z - m0.z, ga.w - m0.w,
-                                     gb.x - m1.x, gb.y - m1.y, gb.z - m1.z, gb.w - m1.w};
-                const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
-                const uint32_t qw[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
-                uint32_t o_kt[4], o_qt[4], o_kb[4];
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                    float kt[2], qt[2], kbv[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int e = 2 * e2 + u;
-                        const float kv = u ? bf16_hi(kw[e2]) : bf16_lo(kw[e2]);
-                        const float qv = u ? bf16_hi(qw[e2]) : bf16_lo(qw[e2]);
-                        const float up = __expf(dg[e]);
-                        const float dn = __expf(-dg[e]);
-                        kt[u] = valid ? kv * up : 0.f;
-                        qt[u] = valid ? qv * up : 0.f;
-                        kbv[u] = valid ? kv * dn : 0.f;
-                    }
-                    o_kt[e2] = pack_h2(kt[0], kt[1]);
-                    o_qt[e2] = pack_h2(qt[0], qt[1]);
-                    o_kb[e2] = pack_h2(kbv[0], kbv[1]);
-                }
-                *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + ph16) = make_uint4(o_kt[0], o_kt[1], o_kt[2], o_kt[3]);
-                *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + 8192 + ph16) = make_uint4(o_qt[0], o_qt[1], o_qt[2], o_qt[3]);
-                *reinterpret_cast<uint4 *>(sm + OFF_KB + kb * 8192 + ph16) = make_uint4(o_kb[0], o_kb[1], o_kb[2], o_kb[3]);
-            }
-        }
-        ptx::fence_proxy_async_smem();
-        __syncthreads();
-        if (*s_abort) break;
-
-        // ---- M1 and M2; then the next chunk's log alpha (g of this chunk is done).
-        if (tid == 0) {
-            ptx::tc_fence_after();
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t ka = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
-                const uint32_t kbo = uint32_t(ks >> 2) * 8192u + uint32_t(ks & 3) * 32u;
-                ptx::mma_ss(tbase + TAP, ptx::sdesc_sw128(sb + OFF_QK + ka), ptx::sdesc_sw128(sb + OFF_KB + kbo),
-                            IDESC_N64, ks > 0);
-            }
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint32_t kq = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
-                ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_QK + kq), IDESC_N128,
-                            ks > 0);
-            }
-            ptx::mma_commit(bar_mma);
-            ++n_mma;
-            if (has_next) {
-                load_la(s_next);
-                ++n_la;
-            }
-        }
-        wait_on(bar_mma, w_mma);
-        ptx::tc_fence_after();
-        if (tid == 0 && has_next) {  // M1 and M2 have read the [Kt; Qt] tile
-            load_qk(s_next);
-            ++n_qk;
-        }
-        wait_on(bar_v, w_v);
-
-        // ---- E1: A rows -> fp32 scratch, P rows -> fp16 operand.
-        // ---- E2: Y^T = V^T - Z[:, :64] -> fp16 operand.
-        {
-            uint32_t v[32];
-            ptx::tmem_ld32(tl + TAP + 32 * half, v);
-            ptx::tmem_wait_ld();
-            if (qd < 2) {
-                const int r = row;
-                const float br = beta[r];
-                float *af = reinterpret_cast<float *>(sm + OFF_AF) + r * LDF + 32 * half;
-                for (int e = 0; e < 32; e += 4) {
-                    float4 x;
-                    const int i = 32 * half + e;
-                    x.x = (i + 0 < r) ? br * __uint_as_float(v[e + 0]) : 0.f;
-                    x.y = (i + 1 < r) ? br * __uint_as_float(v[e + 1]) : 0.f;
-                    x.z = (i + 2 < r) ? br * __uint_as_float(v[e + 2]) : 0.f;
-                    x.w = (i + 3 < r) ? br * __uint_as_float(v[e + 3]) : 0.f;
-                    *reinterpret_cast<float4 *>(af + e) = x;
-                }
-            } else {
-                const int r = row - 64;
-                for (int qq = 0; qq < 4; ++qq) {
-                    uint32_t pk[4];
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        const int e = 8 * qq + 2 * e2, i = 32 * half + e;
-                        pk[e2] = pack_h2(i <= r ? __uint_as_float(v[e]) : 0.f,
-                                         i + 1 <= r ? __uint_as_float(v[e + 1]) : 0.f);
-                    }
-                    *reinterpret_cast<uint4 *>(sm + OFF_P + sw(r, 4 * half + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-            }
-            ptx::tmem_ld32(tl + TZ + 32 * half, v);
-            ptx::tmem_wait_ld();
+            // ---- E0: R *= e^{g_L - g_m}(previous chunk) e^{g_m}; Sop = fp16(R).
+            cwait(CNT_ROWS, ci + 1);
             {
+                const float *egm = vec(par, VEC_EGM);
+                const float *ecm_prev = vec(par ^ 1, VEC_ECM);
+                uint32_t v[32], pk[32];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    ptx::tmem_ld32(tl + TS + 32 * p, v);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int c = 32 * p + e;
+                        const float f = ci > 0 ? ecm_prev[c] * egm[c] : egm[c];
+                        v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+                    }
+                    ptx::tmem_st32(tl + TS + 32 * p, v);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[16 * (p & 1) + e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                    if (p & 1) ptx::tmem_st32(tl + TSOP + 32 * (p >> 1), pk);
+                }
+                ptx::tmem_wait_st();
+            }
+            ptx::tc_fence_before();
+            if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
+            if (leader) {
+                ptx::st_release(cnt + CNT_E0, ci + 1);
+                ptx::tc_fence_after();
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t kq = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
+                    ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_QK + kq), IDESC_N128,
+                                ks > 0);
+                }
+                commit(B_M2);
+            }
+            mwait(B_M2, ci, leader);
+            ptx::tc_fence_after();
+            if (leader) {
+                ptx::st_release(cnt + CNT_M2, ci + 1);
+                // the [Kt; Qt] tile is free once M1 of this chunk has read it too
+                if (has_next && mwait(B_M1, ci, false)) load_qk(s + C);
+            }
+            mwait(B_V, ci, leader);
+
+            // ---- E2: Y^T = V^T - Z[:, :64] -> fp16 operand (rows i >= L of V are
+            // never used: T's columns i >= L are zero).
+            {
+                uint32_t v[32];
                 const int j = row, vbox = j >> 6, jj = j & 63, vch = jj >> 3;
                 const uint8_t *vcol = sm + OFF_V + vbox * 8192 + (jj & 7) * 2;
-                for (int qq = 0; qq < 4; ++qq) {
-                    uint32_t pk[4];
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        float y[2];
-                        for (int u = 0; u < 2; ++u) {
-                            const int e = 8 * qq + 2 * e2 + u, i = 32 * half + e;
-                            const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vcol + sw(i, vch)));
-                            y[u] = (i < L) ? vv - __uint_as_float(v[e]) : 0.f;
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    ptx::tmem_ld32(tl + TZ + 32 * p, v);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            float y[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const int e = 8 * qq + 2 * e2 + u, i = 32 * p + e;
+                                const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vcol + sw(i, vch)));
+                                y[u] = vv - __uint_as_float(v[e]);
+                            }
+                            pk[e2] = pack_h2(y[0], y[1]);
                         }
-                        pk[e2] = pack_h2(y[0], y[1]);
+                        *reinterpret_cast<uint4 *>(sm + OFF_Y + sw(j, 4 * p + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     }
-                    *reinterpret_cast<uint4 *>(sm + OFF_Y + sw(j, 4 * half + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
+            if (leader && has_next) load_v(s + C);  // V has been read
+
+            // ---- M3: U^T = Y^T T^T  (T of this chunk from the prep group).
+            cwait(CNT_TP, ci + 1);
+            if (leader) {
+                ptx::tc_fence_after();
+                for (int ks = 0; ks < 4; ++ks)
+                    ptx::mma_ss(tbase + TU, ptx::sdesc_sw128(sb + OFF_Y + 32 * ks), ptx::sdesc_sw128(sb + OFF_T + 32 * ks),
+                                IDESC_N64, ks > 0);
+                commit(B_M3);
+            }
+            mwait(B_M3, ci, leader);
+            ptx::tc_fence_after();
+            if (leader) ptx::st_release(cnt + CNT_M3, ci + 1);
+            {  // E3: U^T -> fp16 operand
+                uint32_t v[32];
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    ptx::tmem_ld32(tl + TU + 32 * p, v);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int e = 8 * qq + 2 * e2;
+                            pk[e2] = pack_h2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                        }
+                        *reinterpret_cast<uint4 *>(sm + OFF_U + sw(row, 4 * p + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
+            if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
+
+            // ---- M4: R += U^T Kb;  M5: O^T = Z[:, 64:] + U^T P^T.
+            if (leader) {
+                ptx::tc_fence_after();
+                const uint32_t kb_base = OFF_KB + par * 16384, p_base = OFF_P + par * 8192;
+                for (int ks = 0; ks < 4; ++ks)
+                    ptx::mma_ss(tbase + TS, ptx::sdesc_sw128(sb + OFF_U + 32 * ks),
+                                ptx::sdesc_sw128_mn(sb + kb_base + 2048 * ks, 8192, 1024), IDESC_N128_BMN, 1u);
+                for (int ks = 0; ks < 4; ++ks)
+                    ptx::mma_ss(tbase + TZ + 64, ptx::sdesc_sw128(sb + OFF_U + 32 * ks),
+                                ptx::sdesc_sw128(sb + p_base + 32 * ks), IDESC_N64, 1u);
+                commit(B_M45);
+            }
+            mwait(B_M45, ci, leader);
+            ptx::tc_fence_after();
+            if (leader) ptx::st_release(cnt + CNT_M45, ci + 1);
+            {  // E4: outputs of this chunk, staged (bf16, row-major) over the Y^T tile
+                uint32_t v[32];
+                __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_Y);
+                for (int p = 0; p < 2; ++p) {
+                    ptx::tmem_ld32(tl + TZ + 64 + 32 * p, v);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) stage[(32 * p + e) * D + row] = __float2bfloat16_rn(__uint_as_float(v[e]));
+                }
+            }
+            ptx::tc_fence_before();
+            if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
+            {  // rows r < L of the staged outputs, 16 bytes per thread
+                const uint4 *src = reinterpret_cast<const uint4 *>(sm + OFF_Y);
+                char *dst = static_cast<char *>(a.o) + (size_t(s) * H + h) * D * 2;
+                for (int t = tid; t < L * 16; t += NS) {
+                    const int r = t >> 4, q = t & 15;
+                    *reinterpret_cast<uint4 *>(dst + size_t(r) * H * D * 2 + q * 16) = src[r * 16 + q];
+                }
+            }
+            // the staged tile is rewritten by the next E2 only after the next E0 barrier
+        }
+        // Final state S_final[c][j] = R[j][c] e^{g_L - g_m}[c] of the last chunk.
+        if (!*reinterpret_cast<volatile int *>(s_abort)) {
+            ptx::tc_fence_after();
+            const float *ecm_last = vec((nchunks - 1) & 1, VEC_ECM);
+            uint32_t v[32];
+            for (int p = 0; p < 4; ++p) {
+                ptx::tmem_ld32(tl + TS + 32 * p, v);
+                ptx::tmem_wait_ld();
+                for (int e = 0; e < 32; ++e) {
+                    const int c = 32 * p + e;
+                    const float f = nchunks > 0 ? ecm_last[c] : 1.f;
+                    a.S_final[(unit * D + c) * D + row] = __uint_as_float(v[e]) * f;
                 }
             }
         }
-        ptx::fence_proxy_async_smem();
-        ptx::tc_fence_before();
-        __syncthreads();
-        if (*s_abort) break;
-        if (tid == 0 && has_next) {  // V has been read
-            load_v(s_next);
-            ++n_v;
+    } else {
+        // =================================================================== prep group
+        const int pt = tid - NS;  // 0..255
+        const int pw = pt >> 5;   // prep warp 0..7
+        const bool leader = pt == 0;
+        const int qd = warp & 3, half = pw >> 2;
+        const int trow = qd * 32 + lane;  // TMEM lane this thread reads in E1
+        const uint32_t tl = tbase + (uint32_t(qd * 32) << 16);
+        if (leader && nchunks > 0) {
+            load_qk(bos);
+            load_la(bos);
         }
-        // ---- T = (I + A)^{-1} Diag(beta).  X = (I + A)^{-1} in 16x16 blocks: the four
-        // diagonal blocks by column substitution in registers (one warp each), then
-        // E_bk = X_bb A_bk for k < b, then the blocks below the diagonal by distance d,
-        // X_{b,b-d} = -sum_{k=b-d}^{b-1} E_bk X_{k,b-d}.
-        {
-            const float *Af = reinterpret_cast<const float *>(sm + OFF_AF);
-            float *X = reinterpret_cast<float *>(sm + OFF_XF);
-            float *E = reinterpret_cast<float *>(sm + OFF_EB);
-            if (warp < 4) {
-                const int b = warp, jj = lane & 15;
-                const float *ab = Af + (16 * b) * LDF + 16 * b;
-                float x[16];
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jj) ? 1.f : 0.f;
-#pragma unroll
-                for (int ss = 0; ss < 16; ++ss) {  // x[ss] is final: eliminate it below
-#pragma unroll
-                    for (int rr = ss + 1; rr < 16; ++rr) x[rr] = fmaf(-ab[rr * LDF + ss], x[ss], x[rr]);
-                }
-                if (lane < 16) {
-#pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) X[(16 * b + rr) * LDF + 16 * b + jj] = x[rr];
-                }
-            }
-            __syncthreads();
-            // E block e = b(b-1)/2 + k holds X_bb A_bk: 0:(1,0) 1:(2,0) 2:(2,1) 3:(3,0) 4:(3,1) 5:(3,2)
-            // one task = one row of a 16x16 block, 8 columns (two per block row)
-            if (tid < 6 * 32) {
-                const int e = tid >> 5, row = (tid & 31) >> 1, c8 = 8 * (tid & 1);
-                const int b = e == 0 ? 1 : (e < 3 ? 2 : 3);
-                const int k = e - b * (b - 1) / 2;
-                float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {  // X_bb is zero above its diagonal
-                    const float xv = X[(16 * b + row) * LDF + 16 * b + m];
-                    const float4 a0 = *reinterpret_cast<const float4 *>(Af + (16 * b + m) * LDF + 16 * k + c8);
-                    const float4 a1 = *reinterpret_cast<const float4 *>(Af + (16 * b + m) * LDF + 16 * k + c8 + 4);
-                    acc[0] = fmaf(xv, a0.x, acc[0]);
-                    acc[1] = fmaf(xv, a0.y, acc[1]);
-                    acc[2] = fmaf(xv, a0.z, acc[2]);
-                    acc[3] = fmaf(xv, a0.w, acc[3]);
-                    acc[4] = fmaf(xv, a1.x, acc[4]);
-                    acc[5] = fmaf(xv, a1.y, acc[5]);
-                    acc[6] = fmaf(xv, a1.z, acc[6]);
-                    acc[7] = fmaf(xv, a1.w, acc[7]);
-                }
-                float *eo = E + (e * 16 + row) * LDE + c8;
-                *reinterpret_cast<float4 *>(eo) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-                *reinterpret_cast<float4 *>(eo + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-            }
-            __syncthreads();
-            for (int d = 1; d <= 3; ++d) {
-                if (tid < (4 - d) * 32) {
-                    const int bj = tid >> 5, b = bj + d, row = (tid & 31) >> 1, c8 = 8 * (tid & 1);
-                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    for (int k = bj; k < b; ++k) {
-                        const float *eb = E + ((b * (b - 1) / 2 + k) * 16 + row) * LDE;
-#pragma unroll
-                        for (int m = 0; m < 16; ++m) {
-                            const float ev = eb[m];
-                            const float *xr = X + (16 * k + m) * LDF + 16 * bj + c8;
-                            const float4 x0 = *reinterpret_cast<const float4 *>(xr);
-                            const float4 x1 = *reinterpret_cast<const float4 *>(xr + 4);
-                            acc[0] = fmaf(ev, x0.x, acc[0]);
-                            acc[1] = fmaf(ev, x0.y, acc[1]);
-                            acc[2] = fmaf(ev, x0.z, acc[2]);
-                            acc[3] = fmaf(ev, x0.w, acc[3]);
-                            acc[4] = fmaf(ev, x1.x, acc[4]);
-                            acc[5] = fmaf(ev, x1.y, acc[5]);
-                            acc[6] = fmaf(ev, x1.z, acc[6]);
-                            acc[7] = fmaf(ev, x1.w, acc[7]);
-                        }
-                    }
-                    float *xo = X + (16 * b + row) * LDF + 16 * bj + c8;
-                    *reinterpret_cast<float4 *>(xo) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-                    *reinterpret_cast<float4 *>(xo + 4) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
-                }
-                __syncthreads();
-            }
-            // T[r][i] = X[r][i] beta_i for i <= r, as an fp16 operand (rows r, K = i).
+        // beta of a chunk is read from global memory one chunk ahead (a register)
+        auto load_beta = [&](int ci) {
+            const int s = bos + ci * C;
+            return (pt < C && ci < nchunks && s + pt < eos) ? a.beta[size_t(s + pt) * H + h] : 0.f;
+        };
+        float beta_cur = load_beta(0);
+        for (int ci = 0; ci < nchunks; ++ci) {
+            const int s = bos + ci * C;
+            const int L = min(C, eos - s);
+            const bool has_next = ci + 1 < nchunks;
+            const int par = ci & 1;
+            const float beta_next = load_beta(ci + 1);
+            float *gm = vec(par, VEC_GM), *egm = vec(par, VEC_EGM), *ecm = vec(par, VEC_ECM);
+            float *beta = vec(par, VEC_BETA);
+
+            // ---- P1: g = running sum of log alpha per channel, in place, and this
+            // chunk's vectors.  Thread (channel c, half hf) scans tokens
+            // [32 hf, 32 hf + 32); the second half then adds the first half's total.
+            // The vectors of chunk ci - 2 are overwritten: the state group must be
+            // past its pass over R of chunk ci - 1.
+            mwait(B_LA, ci, leader);
+            if (ci >= 2) cwait(CNT_E0, ci);
             {
-                const int rt = tid & 63, part = tid >> 6;
-                for (int qq = 0; qq < 2; ++qq) {
-                    const int ch = 2 * part + qq;
-                    uint32_t pk[4];
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        const int i = 8 * ch + 2 * e2;
-                        const float x0 = (i <= rt) ? X[rt * LDF + i] * beta[i] : 0.f;
-                        const float x1 = (i + 1 <= rt) ? X[rt * LDF + i + 1] * beta[i + 1] : 0.f;
-                        pk[e2] = pack_h2(x0, x1);
-                    }
-                    *reinterpret_cast<uint4 *>(sm + OFF_T + sw(rt, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                }
-            }
-        }
-        ptx::fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---- M3: U^T = Y^T T^T.
-        if (tid == 0) {
-            ptx::tc_fence_after();
-            for (int ks = 0; ks < 4; ++ks)
-                ptx::mma_ss(tbase + TU, ptx::sdesc_sw128(sb + OFF_Y + 32 * ks), ptx::sdesc_sw128(sb + OFF_T + 32 * ks),
-                            IDESC_N64, ks > 0);
-            ptx::mma_commit(bar_mma);
-            ++n_mma;
-        }
-        wait_on(bar_mma, w_mma);
-        ptx::tc_fence_after();
-        {  // E3: U^T -> fp16 operand
-            uint32_t v[32];
-            ptx::tmem_ld32(tl + TU + 32 * half, v);
-            ptx::tmem_wait_ld();
-            for (int qq = 0; qq < 4; ++qq) {
-                uint32_t pk[4];
-                for (int e2 = 0; e2 < 4; ++e2) {
-                    const int e = 8 * qq + 2 * e2;
-                    pk[e2] = pack_h2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                }
-                *reinterpret_cast<uint4 *>(sm + OFF_U + sw(row, 4 * half + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
-        }
-        ptx::fence_proxy_async_smem();
-        ptx::tc_fence_before();
-        __syncthreads();
-        if (*s_abort) break;
-
-        // ---- M4: R += U^T Kb;  M5: O^T = Z[:, 64:] + U^T P^T.  The next chunk's
-        // running sums are formed meanwhile.
-        if (tid == 0) {
-            ptx::tc_fence_after();
-            for (int ks = 0; ks < 4; ++ks)
-                ptx::mma_ss(tbase + TS, ptx::sdesc_sw128(sb + OFF_U + 32 * ks),
-                            ptx::sdesc_sw128_mn(sb + OFF_KB + 2048 * ks, 8192, 1024), IDESC_N128_BMN, 1u);
-            for (int ks = 0; ks < 4; ++ks)
-                ptx::mma_ss(tbase + TZ + 64, ptx::sdesc_sw128(sb + OFF_U + 32 * ks), ptx::sdesc_sw128(sb + OFF_P + 32 * ks),
-                            IDESC_N64, 1u);
-            ptx::mma_commit(bar_mma);
-            ++n_mma;
-        }
-        if (has_next) scan(ci + 1, beta_next);
-        wait_on(bar_mma, w_mma);
-        ptx::tc_fence_after();
-        {  // E4: outputs of this chunk.
-            uint32_t v[32];
-            ptx::tmem_ld32(tl + TZ + 64 + 32 * half, v);
-            ptx::tmem_wait_ld();
-            // stage O[r][j] (bf16, row-major) in the Y^T tile, which M3 has consumed
-            __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_Y);
+                const int c = pt & 127, hf = pt >> 7, box = c >> 5, lc = c & 31, lch = lc >> 2;
+                uint8_t *col = sm + OFF_LA + box * 8192 + (lc & 3) * 4;
+                float *s_half = reinterpret_cast<float *>(sm + OFF_HALF);
+                const int rm = (L - 1) >> 1;
+                float x[32];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) stage[(32 * half + e) * D + row] = __float2bfloat16_rn(__uint_as_float(v[e]));
-        }
-        ptx::tc_fence_before();
-        __syncthreads();
-        if (*s_abort) break;
-        {  // rows r < L of the staged outputs, 16 bytes per thread
-            const uint4 *src = reinterpret_cast<const uint4 *>(sm + OFF_Y);
-            char *dst = static_cast<char *>(a.o) + (size_t(s) * H + h) * D * 2;
-            for (int t = tid; t < L * 16; t += NT) {
-                const int r = t >> 4, q = t & 15;
-                *reinterpret_cast<uint4 *>(dst + size_t(r) * H * D * 2 + q * 16) = src[r * 16 + q];
+                for (int i = 0; i < 32; ++i) {
+                    const int r = 32 * hf + i;
+                    x[i] = (r < L) ? *reinterpret_cast<const float *>(col + sw(r, lch)) : 0.f;
+                }
+#pragma unroll
+                for (int i = 1; i < 32; ++i) x[i] += x[i - 1];
+                if (hf == 0) {
+                    float gmid = 0.f;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) gmid = (i == rm) ? x[i] : gmid;
+                    s_half[c] = x[31];
+                    gm[c] = gmid;
+                    egm[c] = expf(gmid);
+                }
+                if (pt < C) beta[pt] = beta_cur;
+                ptx::named_barrier(BAR_P, NP);
+                if (hf == 1) {
+                    const float off = s_half[c];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) x[i] += off;
+                    ecm[c] = expf(x[31] - gm[c]);
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) *reinterpret_cast<float *>(col + sw(32 * hf + i, lch)) = x[i];
             }
+            beta_cur = beta_next;
+
+            // ---- P2: Kt, Qt (in place over the raw k|q rows) and Kb; one (token row,
+            // 32-channel quarter) per thread.  Kb buffer `par` was last read by M4 of
+            // chunk ci - 2.
+            mwait(B_QK, ci, leader);
+            if (ci >= 2) cwait(CNT_M45, ci - 1);
+            if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
+            {
+                const int r = pt & 63, part = pt >> 6, kb = part >> 1;
+                const bool valid = r < L;
+                uint8_t *kbt = sm + OFF_KB + par * 16384;
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int ch = (part & 1) * 4 + qq;
+                    const uint32_t ph16 = sw(r, ch);
+                    const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + OFF_QK + kb * 16384 + ph16);
+                    const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + OFF_QK + kb * 16384 + 8192 + ph16);
+                    const int c0 = 64 * kb + 8 * ch;
+                    const int box = c0 >> 5, lch = (c0 & 31) >> 2;
+                    const float4 ga = *reinterpret_cast<const float4 *>(sm + OFF_LA + box * 8192 + sw(r, lch));
+                    const float4 gb = *reinterpret_cast<const float4 *>(sm + OFF_LA + box * 8192 + sw(r, lch + 1));
+                    const float4 m0 = *reinterpret_cast<const float4 *>(gm + c0);
+                    const float4 m1 = *reinterpret_cast<const float4 *>(gm + c0 + 4);
+                    const float dg[8] = {ga.x - m0.x, ga.y - m0.y, ga.z - m0.z, ga.w - m0.w,
+                                         gb.x - m1.x, gb.y - m1.y, gb.z - m1.z, gb.w - m1.w};
+                    const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
+                    const uint32_t qw[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
+                    uint32_t o_kt[4], o_qt[4], o_kb[4];
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        float kt[2], qt[2], kbv[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int e = 2 * e2 + u;
+                            const float kv = u ? bf16_hi(kw[e2]) : bf16_lo(kw[e2]);
+                            const float qv = u ? bf16_hi(qw[e2]) : bf16_lo(qw[e2]);
+                            const float up = __expf(dg[e]);
+                            const float dn = __expf(-dg[e]);
+                            kt[u] = valid ? kv * up : 0.f;
+                            qt[u] = valid ? qv * up : 0.f;
+                            kbv[u] = valid ? kv * dn : 0.f;
+                        }
+                        o_kt[e2] = pack_h2(kt[0], kt[1]);
+                        o_qt[e2] = pack_h2(qt[0], qt[1]);
+                        o_kb[e2] = pack_h2(kbv[0], kbv[1]);
+                    }
+                    *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + ph16) = make_uint4(o_kt[0], o_kt[1], o_kt[2], o_kt[3]);
+                    *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + 8192 + ph16) = make_uint4(o_qt[0], o_qt[1], o_qt[2], o_qt[3]);
+                    *reinterpret_cast<uint4 *>(kbt + kb * 8192 + ph16) = make_uint4(o_kb[0], o_kb[1], o_kb[2], o_kb[3]);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
+
+            // ---- M1, then hand the rows to the state group; next chunk's log alpha.
+            if (leader) {
+                ptx::tc_fence_after();
+                const uint32_t kb_base = OFF_KB + par * 16384;
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint32_t ka = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
+                    const uint32_t kbo = uint32_t(ks >> 2) * 8192u + uint32_t(ks & 3) * 32u;
+                    ptx::mma_ss(tbase + TAP, ptx::sdesc_sw128(sb + OFF_QK + ka), ptx::sdesc_sw128(sb + kb_base + kbo),
+                                IDESC_N64, ks > 0);
+                }
+                commit(B_M1);
+                ptx::st_release(cnt + CNT_ROWS, ci + 1);
+                if (has_next) load_la(s + C);  // g of this chunk is no longer read
+            }
+            mwait(B_M1, ci, leader);
+            ptx::tc_fence_after();
+
+            // ---- E1: A rows -> fp32 scratch, P rows -> fp16 operand (buffer `par`,
+            // last read by M5 of chunk ci - 2, already waited for above).
+            {
+                uint32_t v[32];
+                ptx::tmem_ld32(tl + TAP + 32 * half, v);
+                ptx::tmem_wait_ld();
+                if (qd < 2) {
+                    const int r = trow;
+                    const float br = beta[r];
+                    float *af = reinterpret_cast<float *>(sm + OFF_AF) + r * LDF + 32 * half;
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        float4 x;
+                        const int i = 32 * half + e;
+                        x.x = (i + 0 < r) ? br * __uint_as_float(v[e + 0]) : 0.f;
+                        x.y = (i + 1 < r) ? br * __uint_as_float(v[e + 1]) : 0.f;
+                        x.z = (i + 2 < r) ? br * __uint_as_float(v[e + 2]) : 0.f;
+                        x.w = (i + 3 < r) ? br * __uint_as_float(v[e + 3]) : 0.f;
+                        *reinterpret_cast<float4 *>(af + e) = x;
+                    }
+                } else {
+                    const int r = trow - 64;
+                    uint8_t *pt_tile = sm + OFF_P + par * 8192;
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int e = 8 * qq + 2 * e2, i = 32 * half + e;
+                            pk[e2] = pack_h2(i <= r ? __uint_as_float(v[e]) : 0.f,
+                                             i + 1 <= r ? __uint_as_float(v[e + 1]) : 0.f);
+                        }
+                        *reinterpret_cast<uint4 *>(pt_tile + sw(r, 4 * half + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+            }
+            ptx::tc_fence_before();
+            if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
+
+            // ---- T = (I + A)^{-1} Diag(beta).  X = (I + A)^{-1} in 16x16 blocks: the four
+            // diagonal blocks by column substitution in registers (one warp each), then
+            // E_bk = X_bb A_bk for k < b, then the blocks below the diagonal by distance d,
+            // X_{b,b-d} = -sum_{k=b-d}^{b-1} E_bk X_{k,b-d}.
+            {
+                const float *Af = reinterpret_cast<const float *>(sm + OFF_AF);
+                float *X = reinterpret_cast<float *>(sm + OFF_XF);
+                float *E = reinterpret_cast<float *>(sm + OFF_EB);
+                if (pw < 4) {
+                    const int b = pw, jj = lane & 15;
+                    const float *ab = Af + (16 * b) * LDF + 16 * b;
+                    float x[16];
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jj) ? 1.f : 0.f;
+#pragma unroll
+                    for (int ss = 0; ss < 16; ++ss) {  // x[ss] is final: eliminate it below
+#pragma unroll
+                        for (int rr = ss + 1; rr < 16; ++rr) x[rr] = fmaf(-ab[rr * LDF + ss], x[ss], x[rr]);
+                    }
+                    if (lane < 16) {
+#pragma unroll
+                        for (int rr = 0; rr < 16; ++rr) X[(16 * b + rr) * LDF + 16 * b + jj] = x[rr];
+                    }
+                }
+                ptx::named_barrier(BAR_P, NP);
+                // one task = one row of a 16x16 block, 8 columns (two per block row);
+                // E block e = b(b-1)/2 + k holds X_bb A_bk: 0:(1,0) 1:(2,0) 2:(2,1) 3:(3,0) 4:(3,1) 5:(3,2)
+                if (pt < 6 * 32) {
+                    const int e = pt >> 5, rowb = (pt & 31) >> 1, c8 = 8 * (pt & 1);
+                    const int b = e == 0 ? 1 : (e < 3 ? 2 : 3);
+                    const int k = e - b * (b - 1) / 2;
+                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {  // X_bb is zero above its diagonal
+                        const float xv = X[(16 * b + rowb) * LDF + 16 * b + m];
+                        const float4 a0 = *reinterpret_cast<const float4 *>(Af + (16 * b + m) * LDF + 16 * k + c8);
+                        const float4 a1 = *reinterpret_cast<const float4 *>(Af + (16 * b + m) * LDF + 16 * k + c8 + 4);
+                        acc[0] = fmaf(xv, a0.x, acc[0]);
+                        acc[1] = fmaf(xv, a0.y, acc[1]);
+                        acc[2] = fmaf(xv, a0.z, acc[2]);
+                        acc[3] = fmaf(xv, a0.w, acc[3]);
+                        acc[4] = fmaf(xv, a1.x, acc[4]);
+                        acc[5] = fmaf(xv, a1.y, acc[5]);
+                        acc[6] = fmaf(xv, a1.z, acc[6]);
+                        acc[7] = fmaf(xv, a1.w, acc[7]);
+                    }
+                    float *eo = E + (e * 16 + rowb) * LDE + c8;
+                    *reinterpret_cast<float4 *>(eo) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                    *reinterpret_cast<float4 *>(eo + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                }
+                ptx::named_barrier(BAR_P, NP);
+                for (int d = 1; d <= 3; ++d) {
+                    if (pt < (4 - d) * 32) {
+                        const int bj = pt >> 5, b = bj + d, rowb = (pt & 31) >> 1, c8 = 8 * (pt & 1);
+                        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        for (int k = bj; k < b; ++k) {
+                            const float *eb = E + ((b * (b - 1) / 2 + k) * 16 + rowb) * LDE;
+#pragma unroll
+                            for (int m = 0; m < 16; ++m) {
+                                const float ev = eb[m];
+                                const float *xr = X + (16 * k + m) * LDF + 16 * bj + c8;
+                                const float4 x0 = *reinterpret_cast<const float4 *>(xr);
+                                const float4 x1 = *reinterpret_cast<const float4 *>(xr + 4);
+                                acc[0] = fmaf(ev, x0.x, acc[0]);
+                                acc[1] = fmaf(ev, x0.y, acc[1]);
+                                acc[2] = fmaf(ev, x0.z, acc[2]);
+                                acc[3] = fmaf(ev, x0.w, acc[3]);
+                                acc[4] = fmaf(ev, x1.x, acc[4]);
+                                acc[5] = fmaf(ev, x1.y, acc[5]);
+                                acc[6] = fmaf(ev, x1.z, acc[6]);
+                                acc[7] = fmaf(ev, x1.w, acc[7]);
+                            }
+                        }
+                        float *xo = X + (16 * b + rowb) * LDF + 16 * bj + c8;
+                        *reinterpret_cast<float4 *>(xo) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+                        *reinterpret_cast<float4 *>(xo + 4) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
+                    }
+                    ptx::named_barrier(BAR_P, NP);
+                }
+                // T[r][i] = X[r][i] beta_i for i <= r, as an fp16 operand (rows r, K = i);
+                // the T tile was last read by M3 of the previous chunk.
+                if (ci >= 1) cwait(CNT_M3, ci);
+                {
+                    const int rt = pt & 63, part = pt >> 6;
+                    for (int qq = 0; qq < 2; ++qq) {
+                        const int ch = 2 * part + qq;
+                        uint32_t pk[4];
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int i = 8 * ch + 2 * e2;
+                            const float x0 = (i <= rt) ? X[rt * LDF + i] * beta[i] : 0.f;
+                            const float x1 = (i + 1 <= rt) ? X[rt * LDF + i + 1] * beta[i + 1] : 0.f;
+                            pk[e2] = pack_h2(x0, x1);
+                        }
+                        *reinterpret_cast<uint4 *>(sm + OFF_T + sw(rt, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
+            if (leader) ptx::st_release(cnt + CNT_TP, ci + 1);
         }
     }
 
-    if (*s_abort && tid == 0) {  // drain what is still in flight (each wait bounded)
-        while (w_qk < n_qk) ptx::mbar_wait_bounded(bar_qk, uint32_t(w_qk++) & 1u, kWaitCycles);
-        while (w_la < n_la) ptx::mbar_wait_bounded(bar_la, uint32_t(w_la++) & 1u, kWaitCycles);
-        while (w_v < n_v) ptx::mbar_wait_bounded(bar_v, uint32_t(w_v++) & 1u, kWaitCycles);
-        while (w_mma < n_mma) ptx::mbar_wait_bounded(bar_mma, uint32_t(w_mma++) & 1u, kWaitCycles);
-    }
-    // Final state S_final[c][j] = R[j][c] e^{g_L - g_m}[c] of the last chunk.
-    if (!*s_abort) {
-        ptx::tc_fence_after();
-        const float *ecm_last = vec((nchunks - 1) & 1, VEC_ECM);
-        uint32_t v[32];
-        for (int p = 0; p < 2; ++p) {
-            ptx::tmem_ld32(tl + TS + 64 * half + 32 * p, v);
-            ptx::tmem_wait_ld();
-            for (int e = 0; e < 32; ++e) {
-                const int c = 64 * half + 32 * p + e;
-                const float f = nchunks > 0 ? ecm_last[c] : 1.f;
-                a.S_final[(unit * D + c) * D + row] = __uint_as_float(v[e]) * f;
-            }
-        }
+    __syncthreads();
+    if (tid == 0 && *reinterpret_cast<volatile int *>(s_abort)) {
+        // drain what is still in flight (each wait bounded) before TMEM goes away
+        for (int b = 0; b < NBAR; ++b)
+            for (uint32_t ph = wt[b]; ph < iss[b]; ++ph) ptx::mbar_wait_bounded(bars + b, ph & 1u, kWaitCycles);
     }
     ptx::tc_fence_before();
     __syncthreads();
