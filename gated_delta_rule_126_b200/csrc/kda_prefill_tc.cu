@@ -72,18 +72,20 @@ static_assert(OFF_EB + 6 * 16 * LDE * 4 <= OFF_P, "solve scratch overflows");
 constexpr uint32_t OFF_T = OFF_P + 16384;    // T (64 x 64 fp16)
 constexpr uint32_t OFF_Y = OFF_T + 8192;     // Y^T (128 x 64 fp16); later the bf16 output tile
 constexpr uint32_t OFF_U = OFF_Y + 16384;    // U^T (128 x 64 fp16)
-constexpr uint32_t OFF_VEC = OFF_U + 16384;  // per-chunk vectors, two buffers (chunk parity)
+constexpr uint32_t OFF_ID = OFF_U + 16384;   // -I (64 x 64 bf16): loads -V^T into Z with an MMA
+constexpr uint32_t OFF_VEC = OFF_ID + 8192;  // per-chunk vectors, two buffers (chunk parity)
 constexpr uint32_t VEC_GM = 0;        // g_m                  128 f32
 constexpr uint32_t VEC_EGM = 512;     // e^{g_m}
 constexpr uint32_t VEC_ECM = 1024;    // e^{g_L - g_m}
 constexpr uint32_t VEC_BETA = 1536;   // beta                 64 f32
-constexpr uint32_t VEC_BYTES = 1792;
+constexpr uint32_t VEC_FAC = 1792;    // e^{g_L - g_m}(previous chunk) e^{g_m}: the pass over R
+constexpr uint32_t VEC_BYTES = 2304;
 constexpr uint32_t OFF_HALF = OFF_VEC + 2 * VEC_BYTES;  // running sum over the first 32 tokens
 constexpr uint32_t OFF_BAR = OFF_HALF + 512;            // mbarriers
 constexpr int NBAR = 7;
 constexpr int B_QK = 0, B_LA = 1, B_V = 2, B_M1 = 3, B_M2 = 4, B_M3 = 5, B_M45 = 6;
 constexpr uint32_t OFF_CNT = OFF_BAR + 8 * NBAR;        // progress counters
-constexpr int CNT_ROWS = 0, CNT_TP = 1, CNT_E0 = 2, CNT_M2 = 3, CNT_M3 = 4, CNT_M45 = 5;
+constexpr int CNT_ROWS = 0, CNT_TP = 1, CNT_E0 = 2, CNT_M2 = 3, CNT_M3 = 4, CNT_M45 = 5, CNT_TW = 6;
 constexpr uint32_t OFF_ISS = OFF_CNT + 32;              // phases issued / waited per mbarrier
 constexpr uint32_t OFF_WT = OFF_ISS + 4 * NBAR;
 constexpr uint32_t OFF_MISC = OFF_WT + 4 * NBAR;        // tmem base, abort flag
@@ -99,8 +101,9 @@ constexpr uint32_t TSOP = 384;  // Sop fp16           64 cols   state group
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t IDESC_N64 = ptx::idesc_f16_f32(128, 64);
-constexpr uint32_t IDESC_N128 = ptx::idesc_f16_f32(128, 128);
 constexpr uint32_t IDESC_N128_BMN = ptx::idesc_f16_f32(128, 128) | (1u << 16);  // B MN-major
+// bf16 A (MN-major) and B, fp32 D, M = 128, N = 64
+constexpr uint32_t IDESC_BF16_AMN_N64 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (8u << 17) | (8u << 24);
 constexpr long long kWaitCycles = 4000000000LL;  // about two seconds
 
 // byte offset of 16-byte chunk `ch` of row `r` in a 128-byte-row swizzled tile
@@ -218,12 +221,23 @@ __global__ void __launch_bounds__(NT, 1)
         return true;
     };
 
+    // Launched with 384 x 168 registers: the prep group (8 warps) drops to 128, the
+    // state group (4 warps) rises to 240; 4 x 32 x 240 + 8 x 32 x 128 <= 384 x 168.
     if (warp < 4) {
         // =================================================================== state group
+        ptx::regs_inc<240>();
         const int row = tid;  // TMEM lane = value column j
         const uint32_t tl = tbase + (uint32_t(warp * 32) << 16);
         const bool leader = tid == 0;
         if (leader && nchunks > 0) load_v(bos);
+        {  // -I as a K-major bf16 operand (rows r, K = i), for Z[:, :64] = V^T (-I)
+            uint4 *id = reinterpret_cast<uint4 *>(sm + OFF_ID);
+            for (int t = tid; t < 512; t += NS) id[t] = make_uint4(0u, 0u, 0u, 0u);
+            ptx::named_barrier(BAR_S, NS);
+            if (tid < 64) *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_ID + sw(tid, tid >> 3) + (tid & 7) * 2) =
+                __float2bfloat16_rn(-1.f);
+            ptx::fence_proxy_async_smem();
+        }
         {  // R = S0^T
             uint32_t v[32];
             for (int p = 0; p < 4; ++p) {
@@ -244,24 +258,35 @@ __global__ void __launch_bounds__(NT, 1)
             // ---- E0: R *= e^{g_L - g_m}(previous chunk) e^{g_m}; Sop = fp16(R).
             cwait(CNT_ROWS, ci + 1);
             {
-                const float *egm = vec(par, VEC_EGM);
-                const float *ecm_prev = vec(par ^ 1, VEC_ECM);
-                uint32_t v[32], pk[32];
+                const float4 *fac = reinterpret_cast<const float4 *>(vec(par, VEC_FAC));
+                uint32_t r4[4][32], pk[16];
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    ptx::tmem_ld32(tl + TS + 32 * p, v);
-                    ptx::tmem_wait_ld();
+                for (int p = 0; p < 4; ++p) ptx::tmem_ld32(tl + TS + 32 * p, r4[p]);
+                ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int c = 32 * p + e;
-                        const float f = ci > 0 ? ecm_prev[c] * egm[c] : egm[c];
-                        v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+                for (int p = 0; p < 2; ++p) {  // 64 columns at a time
+                    uint32_t(&v)[32] = r4[2 * p];
+                    uint32_t(&w)[32] = r4[2 * p + 1];
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 f0 = fac[16 * p + e4], f1 = fac[16 * p + 8 + e4];
+                        v[4 * e4 + 0] = __float_as_uint(__uint_as_float(v[4 * e4 + 0]) * f0.x);
+                        v[4 * e4 + 1] = __float_as_uint(__uint_as_float(v[4 * e4 + 1]) * f0.y);
+                        v[4 * e4 + 2] = __float_as_uint(__uint_as_float(v[4 * e4 + 2]) * f0.z);
+                        v[4 * e4 + 3] = __float_as_uint(__uint_as_float(v[4 * e4 + 3]) * f0.w);
+                        w[4 * e4 + 0] = __float_as_uint(__uint_as_float(w[4 * e4 + 0]) * f1.x);
+                        w[4 * e4 + 1] = __float_as_uint(__uint_as_float(w[4 * e4 + 1]) * f1.y);
+                        w[4 * e4 + 2] = __float_as_uint(__uint_as_float(w[4 * e4 + 2]) * f1.z);
+                        w[4 * e4 + 3] = __float_as_uint(__uint_as_float(w[4 * e4 + 3]) * f1.w);
                     }
-                    ptx::tmem_st32(tl + TS + 32 * p, v);
+                    ptx::tmem_st32(tl + TS + 64 * p, v);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[16 * (p & 1) + e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-                    if (p & 1) ptx::tmem_st32(tl + TSOP + 32 * (p >> 1), pk);
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                    ptx::tmem_st16(tl + TSOP + 32 * p, pk);
+                    ptx::tmem_st32(tl + TS + 64 * p + 32, w);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_h2(__uint_as_float(w[2 * e]), __uint_as_float(w[2 * e + 1]));
+                    ptx::tmem_st16(tl + TSOP + 32 * p + 16, pk);
                 }
                 ptx::tmem_wait_st();
             }
@@ -269,11 +294,18 @@ __global__ void __launch_bounds__(NT, 1)
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
             if (leader) {
                 ptx::st_release(cnt + CNT_E0, ci + 1);
+                mwait(B_V, ci, true);
                 ptx::tc_fence_after();
+                // Z[:, :64] = -V^T (V read MN-major from its TMA tile), then += Sop Kt^T;
+                // Z[:, 64:] = Sop Qt^T
+                for (int ks = 0; ks < 4; ++ks)
+                    ptx::mma_ss(tbase + TZ, ptx::sdesc_sw128_mn(sb + OFF_V + 2048 * ks, 8192, 1024),
+                                ptx::sdesc_sw128(sb + OFF_ID + 32 * ks), IDESC_BF16_AMN_N64, ks > 0);
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t kq = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
-                    ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_QK + kq), IDESC_N128,
-                                ks > 0);
+                    ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_QK + kq), IDESC_N64, 1u);
+                    ptx::mma_ts(tbase + TZ + 64, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_QK + 8192 + kq),
+                                IDESC_N64, ks > 0);
                 }
                 commit(B_M2);
             }
@@ -281,34 +313,28 @@ __global__ void __launch_bounds__(NT, 1)
             ptx::tc_fence_after();
             if (leader) {
                 ptx::st_release(cnt + CNT_M2, ci + 1);
+                if (has_next) load_v(s + C);  // the V tile has been read by the MMA
                 // the [Kt; Qt] tile is free once M1 of this chunk has read it too
                 if (has_next && mwait(B_M1, ci, false)) load_qk(s + C);
             }
-            mwait(B_V, ci, leader);
 
-            // ---- E2: Y^T = V^T - Z[:, :64] -> fp16 operand (rows i >= L of V are
-            // never used: T's columns i >= L are zero).
+            // ---- E2: Y^T = -Z[:, :64] = V^T - (K e^{g} S)^T -> fp16 operand (rows i >= L
+            // of V are never used: T's columns i >= L are zero).
             {
-                uint32_t v[32];
-                const int j = row, vbox = j >> 6, jj = j & 63, vch = jj >> 3;
-                const uint8_t *vcol = sm + OFF_V + vbox * 8192 + (jj & 7) * 2;
+                uint32_t vz[2][32];
+                const int j = row;
+                ptx::tmem_ld32(tl + TZ, vz[0]);
+                ptx::tmem_ld32(tl + TZ + 32, vz[1]);
+                ptx::tmem_wait_ld();
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
-                    ptx::tmem_ld32(tl + TZ + 32 * p, v);
-                    ptx::tmem_wait_ld();
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq) {
                         uint32_t pk[4];
 #pragma unroll
                         for (int e2 = 0; e2 < 4; ++e2) {
-                            float y[2];
-#pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const int e = 8 * qq + 2 * e2 + u, i = 32 * p + e;
-                                const float vv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(vcol + sw(i, vch)));
-                                y[u] = vv - __uint_as_float(v[e]);
-                            }
-                            pk[e2] = pack_h2(y[0], y[1]);
+                            const int e = 8 * qq + 2 * e2;
+                            pk[e2] = pack_h2(-__uint_as_float(vz[p][e]), -__uint_as_float(vz[p][e + 1]));
                         }
                         *reinterpret_cast<uint4 *>(sm + OFF_Y + sw(j, 4 * p + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     }
@@ -316,11 +342,31 @@ __global__ void __launch_bounds__(NT, 1)
             }
             ptx::fence_proxy_async_smem();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
-            if (leader && has_next) load_v(s + C);  // V has been read
 
             // ---- M3: U^T = Y^T T^T  (T of this chunk from the prep group).
             cwait(CNT_TP, ci + 1);
+            {  // T[r][i] = X[r][i] beta_i for i <= r as an fp16 operand (rows r, K = i)
+                const float *X = reinterpret_cast<const float *>(sm + OFF_XF);
+                const float *beta = vec(par, VEC_BETA);
+                const int rt = tid & 63, part = tid >> 6;
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const int ch = 4 * part + qq;
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const int i = 8 * ch + 2 * e2;
+                        const float x0 = (i <= rt) ? X[rt * LDF + i] * beta[i] : 0.f;
+                        const float x1 = (i + 1 <= rt) ? X[rt * LDF + i + 1] * beta[i + 1] : 0.f;
+                        pk[e2] = pack_h2(x0, x1);
+                    }
+                    *reinterpret_cast<uint4 *>(sm + OFF_T + sw(rt, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+            ptx::fence_proxy_async_smem();
+            if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
             if (leader) {
+                ptx::st_release(cnt + CNT_TW, ci + 1);
                 ptx::tc_fence_after();
                 for (int ks = 0; ks < 4; ++ks)
                     ptx::mma_ss(tbase + TU, ptx::sdesc_sw128(sb + OFF_Y + 32 * ks), ptx::sdesc_sw128(sb + OFF_T + 32 * ks),
@@ -331,11 +377,13 @@ __global__ void __launch_bounds__(NT, 1)
             ptx::tc_fence_after();
             if (leader) ptx::st_release(cnt + CNT_M3, ci + 1);
             {  // E3: U^T -> fp16 operand
-                uint32_t v[32];
+                uint32_t vu[2][32];
+                ptx::tmem_ld32(tl + TU, vu[0]);
+                ptx::tmem_ld32(tl + TU + 32, vu[1]);
+                ptx::tmem_wait_ld();
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
-                    ptx::tmem_ld32(tl + TU + 32 * p, v);
-                    ptx::tmem_wait_ld();
+                    const uint32_t(&v)[32] = vu[p];
 #pragma unroll
                     for (int qq = 0; qq < 4; ++qq) {
                         uint32_t pk[4];
@@ -368,14 +416,16 @@ __global__ void __launch_bounds__(NT, 1)
             ptx::tc_fence_after();
             if (leader) ptx::st_release(cnt + CNT_M45, ci + 1);
             {  // E4: outputs of this chunk, staged (bf16, row-major) over the Y^T tile
-                uint32_t v[32];
+                uint32_t vo[2][32];
                 __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_Y);
-                for (int p = 0; p < 2; ++p) {
-                    ptx::tmem_ld32(tl + TZ + 64 + 32 * p, v);
-                    ptx::tmem_wait_ld();
+                ptx::tmem_ld32(tl + TZ + 64, vo[0]);
+                ptx::tmem_ld32(tl + TZ + 96, vo[1]);
+                ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) stage[(32 * p + e) * D + row] = __float2bfloat16_rn(__uint_as_float(v[e]));
-                }
+                for (int p = 0; p < 2; ++p)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        stage[(32 * p + e) * D + row] = __float2bfloat16_rn(__uint_as_float(vo[p][e]));
             }
             ptx::tc_fence_before();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
@@ -406,6 +456,7 @@ __global__ void __launch_bounds__(NT, 1)
         }
     } else {
         // =================================================================== prep group
+        ptx::regs_dec<128>();
         const int pt = tid - NS;  // 0..255
         const int pw = pt >> 5;   // prep warp 0..7
         const bool leader = pt == 0;
@@ -457,7 +508,9 @@ __global__ void __launch_bounds__(NT, 1)
                     for (int i = 0; i < 32; ++i) gmid = (i == rm) ? x[i] : gmid;
                     s_half[c] = x[31];
                     gm[c] = gmid;
-                    egm[c] = expf(gmid);
+                    const float e = expf(gmid);
+                    egm[c] = e;
+                    vec(par, VEC_FAC)[c] = ci > 0 ? vec(par ^ 1, VEC_ECM)[c] * e : e;
                 }
                 if (pt < C) beta[pt] = beta_cur;
                 ptx::named_barrier(BAR_P, NP);
@@ -589,6 +642,7 @@ __global__ void __launch_bounds__(NT, 1)
                 const float *Af = reinterpret_cast<const float *>(sm + OFF_AF);
                 float *X = reinterpret_cast<float *>(sm + OFF_XF);
                 float *E = reinterpret_cast<float *>(sm + OFF_EB);
+                if (ci >= 1) cwait(CNT_TW, ci);  // the state group has read X of chunk ci - 1
                 if (pw < 4) {
                     const int b = pw, jj = lane & 15;
                     const float *ab = Af + (16 * b) * LDF + 16 * b;
@@ -660,25 +714,8 @@ __global__ void __launch_bounds__(NT, 1)
                     }
                     ptx::named_barrier(BAR_P, NP);
                 }
-                // T[r][i] = X[r][i] beta_i for i <= r, as an fp16 operand (rows r, K = i);
-                // the T tile was last read by M3 of the previous chunk.
-                if (ci >= 1) cwait(CNT_M3, ci);
-                {
-                    const int rt = pt & 63, part = pt >> 6;
-                    for (int qq = 0; qq < 2; ++qq) {
-                        const int ch = 2 * part + qq;
-                        uint32_t pk[4];
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int i = 8 * ch + 2 * e2;
-                            const float x0 = (i <= rt) ? X[rt * LDF + i] * beta[i] : 0.f;
-                            const float x1 = (i + 1 <= rt) ? X[rt * LDF + i + 1] * beta[i + 1] : 0.f;
-                            pk[e2] = pack_h2(x0, x1);
-                        }
-                        *reinterpret_cast<uint4 *>(sm + OFF_T + sw(rt, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    }
-                }
             }
-            ptx::fence_proxy_async_smem();
+            // X (fp32) is handed to the state group, which forms T = X Diag(beta)
             if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
             if (leader) ptx::st_release(cnt + CNT_TP, ci + 1);
         }

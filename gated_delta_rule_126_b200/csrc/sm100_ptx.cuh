@@ -75,6 +75,16 @@ __device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t nthreads,
     return r != 0;
 }
 
+// Per-warp register budget changes for warp-specialised kernels (warpgroup-wide,
+// aligned).  The block's pool is what it was launched with: the increases of some
+// warps must fit in what the others give back.
+template <uint32_t N> __device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N> __device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // Release store / acquire load of a shared-memory word (CTA scope): one group of
 // warps publishes its progress, another reads it.
 __device__ __forceinline__ void st_release(uint32_t *p, uint32_t v) {
@@ -134,6 +144,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32
         "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
         "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
         KDA_W8(0), KDA_W8(8), KDA_W8(16), KDA_W8(24)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        KDA_W8(0), KDA_W8(8)
         : "memory");
 }
 #undef KDA_R8
