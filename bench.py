@@ -227,7 +227,8 @@ def run_reference(args):
 
 
 def run_ours(args):
-    from gated_delta_rule_126_b200 import kda_decode_step, kda_prefill, prefill_workspace_size
+    from gated_delta_rule_126_b200 import (kda_decode_step, kda_decode_tokens, kda_prefill,
+                                           prefill_workspace_size)
     world, rank, local = dist_setup(args)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -339,13 +340,46 @@ def run_ours(args):
         us = d_el / (3 * dw.steps) * 1e6
         dbytes = dw.batch * dw.H * decode_bytes_per_head_step(dw.dk, dw.dv, 2)
         gbs = dbytes / (us * 1e-6) / 1e9
+        # serving form: 4 tokens per call for the same 256 x 32 sequences, states in a
+        # slot pool addressed through a permuted slot table (each state crosses HBM
+        # once per call instead of once per token)
+        n_tok = 4
+        tin = inputs.decode_inputs(dw.batch * n_tok, dw.H, dw.dk, dw.dv, 1, dw.dtype,
+                                   seed=dw.seed + 7, device=dev)
+        tq = {n_: tin[n_][0].reshape(dw.batch, n_tok, dw.H, -1).contiguous()
+              for n_ in ("q", "k", "v", "log_alpha")}
+        tbeta = tin["beta"][0].reshape(dw.batch, n_tok, dw.H).contiguous()
+        pool = tin["S0"][:dw.batch].clone()
+        slots = torch.randperm(dw.batch, generator=torch.Generator().manual_seed(3)).to(
+            torch.int32).to(dev)
+        otok = torch.empty(dw.batch, n_tok, dw.H, dw.dv, dtype=tq["q"].dtype, device=dev)
+
+        def dtok():
+            kda_decode_tokens(tq["q"], tq["k"], tq["v"], tq["log_alpha"], tbeta, pool, slots,
+                              o=otok, stream=stream)
+
+        for _ in range(3):
+            dtok()
+        barrier(world)
+        t_el = max_over_ranks(time_region(dtok, 20, stream), world)
+        us_call = t_el / 20 * 1e6
+        tbytes = dw.batch * dw.H * (2 * 4 * dw.dk * dw.dv +
+                                    n_tok * prefill_bytes_per_head_token(dw.dk, dw.dv, 2))
+        tgbs = tbytes / (us_call * 1e-6) / 1e9
+        decode_tokens = {"tokens_per_call": n_tok, "us_per_call": us_call,
+                         "us_per_token": us_call / n_tok,
+                         "tokens_per_s": world * dw.batch * n_tok / (us_call * 1e-6),
+                         "roofline": {"bound": "hbm", "achieved": tgbs, "peak": hbm_peak,
+                                      "unit": "GB/s", "frac": tgbs / hbm_peak,
+                                      "alg_bytes_per_launch": tbytes}}
+        del tin, tq, pool
         decode = {"workload": dw.name, "us_per_step": us, "batch": dw.batch, "H": dw.H,
                   "steps_per_sequence": dw.steps,
                   "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s",
                                "frac": gbs / hbm_peak, "traffic": None,
                                "alg_bytes_per_launch": dbytes,
                                "peak_source": f"{peak_kind} hbm_gbs (copy, burst)"},
-                  "gpu_launches_per_step": 1}
+                  "gpu_launches_per_step": 1, "multi_token": decode_tokens}
         del dinp, S
 
     cpu = None

@@ -7,13 +7,14 @@ binding over that ABI, with the same names:
 
 * ``kda_prefill``     -- chunked prefill over packed variable-length sequences;
 * ``kda_decode_step`` -- one recurrent decode step for a batch of sequences;
+* ``kda_decode_tokens`` -- n tokens per sequence with states in a slot pool;
 * ``prefill_workspace_size``, ``workspace_status``, ``KdaError``.
 
 ``inputs`` holds the seeded synthetic input generators.  Importing the package
 does not load the CUDA library; the first call does, and raises if it is missing.
 """
-from ._binding import (KdaError, kda_decode_step, kda_prefill, load, prefill_workspace_size,
-                       workspace_status)
+from ._binding import (KdaError, kda_decode_step, kda_decode_tokens, kda_prefill, load,
+                       prefill_workspace_size, workspace_status)
 
-__all__ = ["KdaError", "kda_decode_step", "kda_prefill", "load", "prefill_workspace_size",
-           "workspace_status"]
+__all__ = ["KdaError", "kda_decode_step", "kda_decode_tokens", "kda_prefill", "load",
+           "prefill_workspace_size", "workspace_status"]

@@ -47,6 +47,9 @@ def _declare(lib):
                                 vp, vp, vp, sz, vp]
     lib.kda_decode_step.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, vp]
+    lib.kda_decode_tokens.restype = i32
+    lib.kda_decode_tokens.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                      vp, vp]
     lib.kda_workspace_status.restype = i32
     lib.kda_workspace_status.argtypes = [vp, vp]
     return lib
@@ -176,6 +179,39 @@ def kda_decode_step(q, k, v, log_alpha, beta, S, o=None, stream=None):
                                  _ptr(beta), _ptr(S), B, H, dk, dv, _ptr(o),
                                  _stream_handle(stream))
     _check(st, "kda_decode_step")
+    return o
+
+
+def kda_decode_tokens(q, k, v, log_alpha, beta, S_pool, slot_idx=None, o=None, stream=None):
+    """n tokens for B sequences with states in a slot pool (see ``kda_decode_tokens`` in kda.h).
+
+    q, k [B,n,H,d_k], v [B,n,H,d_v], log_alpha [B,n,H,d_k] f32, beta [B,n,H] f32,
+    S_pool [num_slots,H,d_k,d_v] f32 (updated in place), slot_idx [B] int32 on the
+    device or None (slot b).  Returns o [B,n,H,d_v].
+    """
+    lib = load()
+    dev = q.device
+    dt = q.dtype
+    if dt not in DTYPE_CODE:
+        raise ValueError("q/k/v dtype must be float32 or bfloat16")
+    _need(q, "q", dt)
+    B, n, H, dk = q.shape
+    _need(k, "k", dt, dev)
+    _need(v, "v", dt, dev)
+    dv = v.shape[3]
+    _need(log_alpha, "log_alpha", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(S_pool, "S_pool", torch.float32, dev)
+    if slot_idx is not None:
+        _need(slot_idx, "slot_idx", torch.int32, dev)
+    if o is None:
+        o = torch.empty(B, n, H, dv, dtype=dt, device=dev)
+    _need(o, "o", dt, dev)
+    with torch.cuda.device(dev):
+        st = lib.kda_decode_tokens(_ptr(q), _ptr(k), _ptr(v), DTYPE_CODE[dt], _ptr(log_alpha),
+                                   _ptr(beta), _ptr(S_pool), _ptr(slot_idx), S_pool.shape[0], B,
+                                   n, H, dk, dv, _ptr(o), _stream_handle(stream))
+    _check(st, "kda_decode_tokens")
     return o
 
 

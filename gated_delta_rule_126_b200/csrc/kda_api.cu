@@ -108,6 +108,24 @@ kda_status_t kda_decode_step(const void *q, const void *k, const void *v, kda_dt
     return from_cuda(kda::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+kda_status_t kda_decode_tokens(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                               const float *log_alpha, const float *beta, float *S_pool,
+                               const int32_t *slot_idx, int num_slots, int B, int n, int H, int d_k,
+                               int d_v, void *o, kda_stream_t stream) {
+    if (B < 0 || n < 0 || H < 1 || d_k < 1 || d_v < 1 || num_slots < 0 || !dtype_ok(qkv_dtype))
+        return KDA_ERR_INVALID_ARG;
+    if (d_k > 128 || d_v > 128 || (d_v % 4) != 0) return KDA_ERR_UNSUPPORTED;
+    if (!slot_idx && num_slots < B) return KDA_ERR_INVALID_ARG;
+    if (B == 0 || n == 0) return KDA_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !S_pool || !o) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(S_pool)) return KDA_ERR_INVALID_ARG;
+    kda::DecodeTokensArgs a;
+    a.q = q; a.k = k; a.v = v; a.dtype = qkv_dtype;
+    a.log_alpha = log_alpha; a.beta = beta; a.S_pool = S_pool; a.slot_idx = slot_idx;
+    a.num_slots = num_slots; a.B = B; a.n = n; a.H = H; a.dk = d_k; a.dv = d_v; a.o = o;
+    return from_cuda(kda::launch_decode_tokens(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 kda_status_t kda_workspace_status(const void *workspace, kda_stream_t stream) {
     if (!workspace) return KDA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

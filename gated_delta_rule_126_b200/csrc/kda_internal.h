@@ -56,7 +56,18 @@ struct DecodeArgs {
     void *o;
 };
 
+struct DecodeTokensArgs {
+    const void *q, *k, *v;
+    kda_dtype_t dtype;
+    const float *log_alpha, *beta;
+    float *S_pool;
+    const int32_t *slot_idx;  // [B] or NULL (slot = b)
+    int num_slots, B, n, H, dk, dv;
+    void *o;
+};
+
 cudaError_t launch_order_by_length(const PrefillArgs &a, cudaStream_t stream);
+cudaError_t launch_decode_tokens(const DecodeTokensArgs &a, cudaStream_t stream);
 cudaError_t launch_prefill_simt(const PrefillArgs &a, cudaStream_t stream);
 bool prefill_tc_supported(const PrefillArgs &a);
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream);

@@ -167,6 +167,28 @@ KDA_API kda_status_t kda_prefill_noalloc(const void *q, const void *k, const voi
                                  void *o, float *S_final, kda_stream_t stream);
 
 /*
+ * kda_decode_tokens -- n consecutive tokens for B sequences whose states live in a
+ * pool of state slots (serving-style decode, and the multi-token form of the
+ * recurrence used to check several drafted tokens at once).
+ *
+ * For every b with 0 <= slot_idx[b] < num_slots and every head, the state in
+ * that slot is advanced through tokens 0 .. n-1 of sequence b by the same
+ * equation as kda_decode_step (o written for every token) and written back.  The
+ * state crosses HBM once per call instead of once per token.
+ *
+ *   q, k, log_alpha  [B, n, H, d_k]    v, o  [B, n, H, d_v]    beta  [B, n, H]
+ *   S_pool    [num_slots, H, d_k, d_v] float32, 16-byte aligned, read and updated
+ *   slot_idx  [B] int32 device array, or NULL for slot b (then num_slots >= B);
+ *             a slot outside [0, num_slots) skips sequence b (no output written);
+ *             two sequences of one call must not share a slot (their updates race)
+ * Supported: 1 <= d_k <= 128, d_v in {4, 8, ..., 128}; B = 0 or n = 0 is a no-op.
+ */
+KDA_API kda_status_t kda_decode_tokens(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                               const float *log_alpha, const float *beta, float *S_pool,
+                               const int32_t *slot_idx, int num_slots, int B, int n, int H,
+                               int d_k, int d_v, void *o, kda_stream_t stream);
+
+/*
  * kda_workspace_status -- waits for `stream`, then reports whether a kernel of
  * the last kda_prefill call that used `workspace` flagged an internal error
  * (KDA_ERR_DEVICE_FAULT, e.g. a bounded wait that ran out) and clears the flag.

@@ -29,8 +29,8 @@ def declared_symbols():
 
 def test_header_declares_the_abi():
     assert declared_symbols() == sorted([
-        "kda_decode_step", "kda_prefill", "kda_prefill_noalloc", "kda_prefill_workspace_size",
-        "kda_status_string", "kda_version", "kda_workspace_status"])
+        "kda_decode_step", "kda_decode_tokens", "kda_prefill", "kda_prefill_noalloc",
+        "kda_prefill_workspace_size", "kda_status_string", "kda_version", "kda_workspace_status"])
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -98,6 +98,23 @@ def test_decode_rejects_bad_arguments(lib):
     assert f(FAKE, FAKE, FAKE, 1, FAKE, FAKE, ctypes.c_void_p((1 << 20) + 4), 4, 2, 128, 128,
              FAKE, None) == INVALID
     assert f(None, None, None, 1, None, None, None, 0, 2, 128, 128, None, None) == 0  # B = 0
+
+
+def test_decode_tokens_rejects_bad_arguments(lib):
+    f = lib.kda_decode_tokens
+    args = lambda **kw: [kw.get("q", FAKE), FAKE, FAKE, kw.get("dt", 1), FAKE, FAKE, kw.get("S", FAKE),
+                         kw.get("slots", FAKE), kw.get("ns", 8), kw.get("B", 4), kw.get("n", 2),
+                         kw.get("H", 2), 128, kw.get("dv", 128), FAKE, None]
+    assert f(*args(B=-1)) == INVALID
+    assert f(*args(n=-1)) == INVALID
+    assert f(*args(H=0)) == INVALID
+    assert f(*args(ns=-1)) == INVALID
+    assert f(*args(dt=3)) == INVALID
+    assert f(*args(dv=126)) == UNSUPPORTED
+    assert f(*args(slots=None, ns=2)) == INVALID          # identity slots need num_slots >= B
+    assert f(*args(q=None)) == INVALID
+    assert f(*args(S=ctypes.c_void_p((1 << 20) + 4))) == INVALID
+    assert f(*args(n=0)) == 0 and f(*args(B=0)) == 0
 
 
 def test_binding_raises_without_library(tmp_path):
