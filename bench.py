@@ -126,14 +126,16 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def dist_setup(args):
+def dist_setup(backend="nccl"):
+    """Join the process group that torchrun describes in the environment (one rank
+    per GPU); a single process needs none.  Returns (world, rank, local_rank)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local))
+        kw = {"device_id": torch.device("cuda", local)} if backend == "nccl" else {}
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
@@ -150,18 +152,25 @@ def time_region(fn, steps, stream):
     return start.elapsed_time(end) / 1e3
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """The largest of every rank's x (the job's time is its slowest rank's)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
 
-def barrier(world):
+def barrier(world, cuda=True):
     if world > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if cuda:
+        torch.cuda.synchronize()
+
+
+def weak_scaling_value(tokens_per_rank, steps, max_elapsed_s, world):
+    """Whole-job tokens/s: every rank runs its own copy of the workload."""
+    return world * tokens_per_rank * steps / max_elapsed_s
 
 
 def oracle_sample(w, budget_head_tokens, seed_device="cpu"):
@@ -229,7 +238,7 @@ def run_reference(args):
 def run_ours(args):
     from gated_delta_rule_126_b200 import (kda_decode_step, kda_decode_tokens, kda_prefill,
                                            prefill_workspace_size)
-    world, rank, local = dist_setup(args)
+    world, rank, local = dist_setup("nccl")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
@@ -259,7 +268,7 @@ def run_ours(args):
     barrier(world)
     elapsed = max_over_ranks(elapsed, world)
     ms = elapsed / args.steps * 1e3
-    value = world * T * args.steps / elapsed
+    value = weak_scaling_value(T, args.steps, elapsed, world)
 
     # roofline of the prefill kernel (one launch per step; events above bracket the
     # call, which also holds a one-thread-block ordering kernel of a few microseconds)
