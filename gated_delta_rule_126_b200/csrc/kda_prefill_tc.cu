@@ -27,11 +27,12 @@
 //   R at the start of each chunk, which also packs Sop, so no K e^{g}, Q e^{g} or
 //   (K e^{g_L - g})^T tile is built.
 // * Two warp groups work on different chunks at once.  The prep group (warps
-//   4-11) builds chunk c + 1 -- running sums, decayed rows, M1, A and P, the
-//   triangular solve for T -- while the state group (warps 0-3) runs chunk c --
-//   the pass over R, M2, Y, M3, U, M4/M5 and the outputs.  They hand buffers over
-//   through release/acquire progress counters in shared memory; the decayed-row
-//   (Kb) and P tiles are double-buffered by chunk parity.
+//   4-11) builds chunk c + 1 -- decayed rows, M1, A and P, the triangular solve
+//   for T -- while the state group (warps 0-3) runs chunk c -- the pass over R,
+//   M2, Y, M3, U, M4/M5 and the outputs -- and, while it waits for T, the
+//   running sums of chunk c + 1.  They hand buffers over through release/acquire
+//   progress counters in shared memory; the decayed-row (Kb) and P tiles and the
+//   per-chunk vectors are double-buffered by chunk parity.
 // * Operands are fp16 (fp32 accumulation): the S-dependent chain keeps the
 //   relative error near fp16's 2^-11, which the parity bounds need (bf16 operands
 //   do not meet them).  Sop lives in TMEM (fp16 pairs per column).
@@ -80,12 +81,11 @@ constexpr uint32_t VEC_ECM = 1024;    // e^{g_L - g_m}
 constexpr uint32_t VEC_BETA = 1536;   // beta                 64 f32
 constexpr uint32_t VEC_FAC = 1792;    // e^{g_L - g_m}(previous chunk) e^{g_m}: the pass over R
 constexpr uint32_t VEC_BYTES = 2304;
-constexpr uint32_t OFF_HALF = OFF_VEC + 2 * VEC_BYTES;  // running sum over the first 32 tokens
-constexpr uint32_t OFF_BAR = OFF_HALF + 512;            // mbarriers
+constexpr uint32_t OFF_BAR = OFF_VEC + 2 * VEC_BYTES;   // mbarriers
 constexpr int NBAR = 7;
 constexpr int B_QK = 0, B_LA = 1, B_V = 2, B_M1 = 3, B_M2 = 4, B_M3 = 5, B_M45 = 6;
 constexpr uint32_t OFF_CNT = OFF_BAR + 8 * NBAR;        // progress counters
-constexpr int CNT_ROWS = 0, CNT_TP = 1, CNT_E0 = 2, CNT_M2 = 3, CNT_M3 = 4, CNT_M45 = 5, CNT_TW = 6;
+constexpr int CNT_ROWS = 0, CNT_TP = 1, CNT_SCAN = 2, CNT_M45 = 3, CNT_TW = 4;
 constexpr uint32_t OFF_ISS = OFF_CNT + 32;              // phases issued / waited per mbarrier
 constexpr uint32_t OFF_WT = OFF_ISS + 4 * NBAR;
 constexpr uint32_t OFF_MISC = OFF_WT + 4 * NBAR;        // tmem base, abort flag
@@ -249,6 +249,48 @@ __global__ void __launch_bounds__(NT, 1)
             }
             ptx::tmem_wait_st();
         }
+        // ---- P1 of chunk cj: g = running sum of log alpha per channel, in place over
+        // the log alpha tile, and the chunk's vectors (buffer cj & 1): g_m, e^{g_m},
+        // e^{g_L - g_m}, the factors of the pass over R and beta.  One channel per
+        // thread; beta is read from global memory one chunk ahead (a register).
+        auto load_beta = [&](int cj) {
+            const int s = bos + cj * C;
+            return (tid < C && cj < nchunks && s + tid < eos) ? a.beta[size_t(s + tid) * H + h] : 0.f;
+        };
+        float beta_reg = load_beta(0);
+        float ecm_prev = 1.f;  // e^{g_L - g_m} of the previous chunk, channel tid
+        auto scan = [&](int cj) {
+            const int L = min(C, eos - (bos + cj * C));
+            const int par = cj & 1;
+            const int c = tid, lch = (c & 31) >> 2;
+            uint8_t *col = sm + OFF_LA + (c >> 5) * 8192 + (c & 3) * 4;
+            const int rm = (L - 1) >> 1;
+            mwait(B_LA, cj, leader);
+            float x[C];
+#pragma unroll
+            for (int i = 0; i < C; ++i) x[i] = (i < L) ? *reinterpret_cast<const float *>(col + sw(i, lch)) : 0.f;
+#pragma unroll
+            for (int i = 1; i < C; ++i) x[i] += x[i - 1];
+            float gmid = 0.f;
+#pragma unroll
+            for (int i = 0; i < C; ++i) gmid = (i == rm) ? x[i] : gmid;
+#pragma unroll
+            for (int i = 0; i < C; ++i) *reinterpret_cast<float *>(col + sw(i, lch)) = x[i];
+            const float e = expf(gmid), ecm = expf(x[C - 1] - gmid);  // rows >= L add 0
+            vec(par, VEC_GM)[c] = gmid;
+            vec(par, VEC_EGM)[c] = e;
+            vec(par, VEC_ECM)[c] = ecm;
+            vec(par, VEC_FAC)[c] = ecm_prev * e;
+            ecm_prev = ecm;
+            if (tid < C) vec(par, VEC_BETA)[tid] = beta_reg;
+            beta_reg = load_beta(cj + 1);
+            ptx::fence_proxy_async_smem();  // the next log alpha tile overwrites g by TMA
+        };
+        if (nchunks > 0) {
+            scan(0);
+            ptx::named_barrier(BAR_S, NS);
+            if (leader) ptx::st_release(cnt + CNT_SCAN, 1u);
+        }
         for (int ci = 0; ci < nchunks; ++ci) {
             const int s = bos + ci * C;
             const int L = min(C, eos - s);
@@ -256,7 +298,6 @@ __global__ void __launch_bounds__(NT, 1)
             const int par = ci & 1;
 
             // ---- E0: R *= e^{g_L - g_m}(previous chunk) e^{g_m}; Sop = fp16(R).
-            cwait(CNT_ROWS, ci + 1);
             {
                 const float4 *fac = reinterpret_cast<const float4 *>(vec(par, VEC_FAC));
                 uint32_t r4[4][32], pk[16];
@@ -293,7 +334,7 @@ __global__ void __launch_bounds__(NT, 1)
             ptx::tc_fence_before();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
             if (leader) {
-                ptx::st_release(cnt + CNT_E0, ci + 1);
+                cwait(CNT_ROWS, ci + 1);  // [Kt; Qt] of this chunk
                 mwait(B_V, ci, true);
                 ptx::tc_fence_after();
                 // Z[:, :64] = -V^T (V read MN-major from its TMA tile), then += Sop Kt^T;
@@ -312,7 +353,6 @@ __global__ void __launch_bounds__(NT, 1)
             mwait(B_M2, ci, leader);
             ptx::tc_fence_after();
             if (leader) {
-                ptx::st_release(cnt + CNT_M2, ci + 1);
                 if (has_next) load_v(s + C);  // the V tile has been read by the MMA
                 // the [Kt; Qt] tile is free once M1 of this chunk has read it too
                 if (has_next && mwait(B_M1, ci, false)) load_qk(s + C);
@@ -341,7 +381,11 @@ __global__ void __launch_bounds__(NT, 1)
                 }
             }
             ptx::fence_proxy_async_smem();
+            // P1 of the next chunk.  Its vectors go to the buffer of chunk ci - 1, which the
+            // prep group last read in E1 of chunk ci - 1, before its rows of chunk ci.
+            if (has_next) scan(ci + 1);
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
+            if (leader && has_next) ptx::st_release(cnt + CNT_SCAN, ci + 2);
 
             // ---- M3: U^T = Y^T T^T  (T of this chunk from the prep group).
             cwait(CNT_TP, ci + 1);
@@ -375,7 +419,6 @@ __global__ void __launch_bounds__(NT, 1)
             }
             mwait(B_M3, ci, leader);
             ptx::tc_fence_after();
-            if (leader) ptx::st_release(cnt + CNT_M3, ci + 1);
             {  // E3: U^T -> fp16 operand
                 uint32_t vu[2][32];
                 ptx::tmem_ld32(tl + TU, vu[0]);
@@ -467,67 +510,17 @@ __global__ void __launch_bounds__(NT, 1)
             load_qk(bos);
             load_la(bos);
         }
-        // beta of a chunk is read from global memory one chunk ahead (a register)
-        auto load_beta = [&](int ci) {
-            const int s = bos + ci * C;
-            return (pt < C && ci < nchunks && s + pt < eos) ? a.beta[size_t(s + pt) * H + h] : 0.f;
-        };
-        float beta_cur = load_beta(0);
         for (int ci = 0; ci < nchunks; ++ci) {
             const int s = bos + ci * C;
             const int L = min(C, eos - s);
             const bool has_next = ci + 1 < nchunks;
             const int par = ci & 1;
-            const float beta_next = load_beta(ci + 1);
-            float *gm = vec(par, VEC_GM), *egm = vec(par, VEC_EGM), *ecm = vec(par, VEC_ECM);
-            float *beta = vec(par, VEC_BETA);
-
-            // ---- P1: g = running sum of log alpha per channel, in place, and this
-            // chunk's vectors.  Thread (channel c, half hf) scans tokens
-            // [32 hf, 32 hf + 32); the second half then adds the first half's total.
-            // The vectors of chunk ci - 2 are overwritten: the state group must be
-            // past its pass over R of chunk ci - 1.
-            mwait(B_LA, ci, leader);
-            if (ci >= 2) cwait(CNT_E0, ci);
-            {
-                const int c = pt & 127, hf = pt >> 7, box = c >> 5, lc = c & 31, lch = lc >> 2;
-                uint8_t *col = sm + OFF_LA + box * 8192 + (lc & 3) * 4;
-                float *s_half = reinterpret_cast<float *>(sm + OFF_HALF);
-                const int rm = (L - 1) >> 1;
-                float x[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int r = 32 * hf + i;
-                    x[i] = (r < L) ? *reinterpret_cast<const float *>(col + sw(r, lch)) : 0.f;
-                }
-#pragma unroll
-                for (int i = 1; i < 32; ++i) x[i] += x[i - 1];
-                if (hf == 0) {
-                    float gmid = 0.f;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) gmid = (i == rm) ? x[i] : gmid;
-                    s_half[c] = x[31];
-                    gm[c] = gmid;
-                    const float e = expf(gmid);
-                    egm[c] = e;
-                    vec(par, VEC_FAC)[c] = ci > 0 ? vec(par ^ 1, VEC_ECM)[c] * e : e;
-                }
-                if (pt < C) beta[pt] = beta_cur;
-                ptx::named_barrier(BAR_P, NP);
-                if (hf == 1) {
-                    const float off = s_half[c];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) x[i] += off;
-                    ecm[c] = expf(x[31] - gm[c]);
-                }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) *reinterpret_cast<float *>(col + sw(32 * hf + i, lch)) = x[i];
-            }
-            beta_cur = beta_next;
+            const float *gm = vec(par, VEC_GM), *beta = vec(par, VEC_BETA);
 
             // ---- P2: Kt, Qt (in place over the raw k|q rows) and Kb; one (token row,
             // 32-channel quarter) per thread.  Kb buffer `par` was last read by M4 of
-            // chunk ci - 2.
+            // chunk ci - 2.  g and g_m come from the state group's P1.
+            cwait(CNT_SCAN, ci + 1);
             mwait(B_QK, ci, leader);
             if (ci >= 2) cwait(CNT_M45, ci - 1);
             if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
