@@ -101,6 +101,7 @@ constexpr uint32_t TSOP = 384;  // Sop fp16           64 cols   state group
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t IDESC_N64 = ptx::idesc_f16_f32(128, 64);
+constexpr uint32_t IDESC_N128 = ptx::idesc_f16_f32(128, 128);
 constexpr uint32_t IDESC_N128_BMN = ptx::idesc_f16_f32(128, 128) | (1u << 16);  // B MN-major
 // bf16 A (MN-major) and B, fp32 D, M = 128, N = 64
 constexpr uint32_t IDESC_BF16_AMN_N64 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (8u << 17) | (8u << 24);
@@ -335,19 +336,20 @@ __global__ void __launch_bounds__(NT, 1)
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
             if (leader) {
                 cwait(CNT_ROWS, ci + 1);  // [Kt; Qt] of this chunk
-                mwait(B_V, ci, true);
                 ptx::tc_fence_after();
-                // Z[:, :64] = -V^T (V read MN-major from its TMA tile), then += Sop Kt^T;
-                // Z[:, 64:] = Sop Qt^T
-                for (int ks = 0; ks < 4; ++ks)
-                    ptx::mma_ss(tbase + TZ, ptx::sdesc_sw128_mn(sb + OFF_V + 2048 * ks, 8192, 1024),
-                                ptx::sdesc_sw128(sb + OFF_ID + 32 * ks), IDESC_BF16_AMN_N64, ks > 0);
+                // Z = Sop [Kt; Qt]^T (the k and q boxes of a channel block are rows 0-63 and
+                // 64-127 of one 128-row operand), then Z[:, :64] += V^T (-I), V read MN-major
+                // from its TMA tile
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t kq = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
-                    ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_QK + kq), IDESC_N64, 1u);
-                    ptx::mma_ts(tbase + TZ + 64, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_QK + 8192 + kq),
-                                IDESC_N64, ks > 0);
+                    ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_QK + kq), IDESC_N128,
+                                ks > 0);
                 }
+                mwait(B_V, ci, true);
+                ptx::tc_fence_after();
+                for (int ks = 0; ks < 4; ++ks)
+                    ptx::mma_ss(tbase + TZ, ptx::sdesc_sw128_mn(sb + OFF_V + 2048 * ks, 8192, 1024),
+                                ptx::sdesc_sw128(sb + OFF_ID + 32 * ks), IDESC_BF16_AMN_N64, 1u);
                 commit(B_M2);
             }
             mwait(B_M2, ci, leader);
