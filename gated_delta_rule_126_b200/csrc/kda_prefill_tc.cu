@@ -67,13 +67,13 @@ constexpr int LDF = 68;
 constexpr int LDE = 20;
 constexpr uint32_t OFF_AF = OFF_SCR;
 constexpr uint32_t OFF_XF = OFF_AF + 64 * LDF * 4;
-constexpr uint32_t OFF_EB = OFF_XF + 64 * LDF * 4;  // six 16x16 blocks X_bb A_bk
+constexpr uint32_t OFF_EB = OFF_XF + 64 * LDF * 4;  // X_11 A_10 and X_33 A_32; then X_H1 A_21
+constexpr int LDG = 33;
 constexpr uint32_t OFF_P = 157696;    // P (64 x 64 fp16), two buffers
-static_assert(OFF_EB + 6 * 16 * LDE * 4 <= OFF_P, "solve scratch overflows");
+static_assert(OFF_EB + 32 * LDE * 4 <= OFF_P && OFF_EB + 32 * LDG * 4 <= OFF_P, "solve scratch overflows");
 constexpr uint32_t OFF_T = OFF_P + 16384;    // T (64 x 64 fp16)
-constexpr uint32_t OFF_Y = OFF_T + 8192;     // Y^T (128 x 64 fp16); later the bf16 output tile
-constexpr uint32_t OFF_U = OFF_Y + 16384;    // U^T (128 x 64 fp16)
-constexpr uint32_t OFF_ID = OFF_U + 16384;   // -I (64 x 64 bf16): loads -V^T into Z with an MMA
+constexpr uint32_t OFF_Y = OFF_T + 8192;     // the bf16 output tile (two 64 x 64 boxes)
+constexpr uint32_t OFF_ID = OFF_Y + 16384;   // -I (64 x 64 bf16): loads -V^T into Z with an MMA
 constexpr uint32_t OFF_VEC = OFF_ID + 8192;  // per-chunk vectors, two buffers (chunk parity)
 constexpr uint32_t VEC_GM = 0;        // g_m                  128 f32
 constexpr uint32_t VEC_EGM = 512;     // e^{g_m}
@@ -98,6 +98,8 @@ constexpr uint32_t TZ = 128;    // Z fp32            128 cols   state group
 constexpr uint32_t TU = 256;    // U^T fp32           64 cols   state group
 constexpr uint32_t TAP = 320;   // [A; P] raw fp32    64 cols   prep group
 constexpr uint32_t TSOP = 384;  // Sop fp16           64 cols   state group
+constexpr uint32_t TY16 = TSOP;       // Y^T fp16, 32 cols, over Sop once M2 has read it
+constexpr uint32_t TU16 = TSOP + 32;  // U^T fp16, 32 cols
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t IDESC_N64 = ptx::idesc_f16_f32(128, 64);
@@ -106,6 +108,7 @@ constexpr uint32_t IDESC_N128_BMN = ptx::idesc_f16_f32(128, 128) | (1u << 16);  
 // bf16 A (MN-major) and B, fp32 D, M = 128, N = 64
 constexpr uint32_t IDESC_BF16_AMN_N64 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (8u << 17) | (8u << 24);
 constexpr long long kWaitCycles = 4000000000LL;  // about two seconds
+constexpr float kLog2e = 1.4426950408889634f;
 
 // byte offset of 16-byte chunk `ch` of row `r` in a 128-byte-row swizzled tile
 __device__ __forceinline__ uint32_t sw(int r, int ch) { return uint32_t(r) * 128u + (uint32_t((ch ^ (r & 7))) << 4); }
@@ -118,7 +121,7 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 struct TcMaps {
-    CUtensorMap q, k, v, la;
+    CUtensorMap q, k, v, la, o;
 };
 
 __global__ void __launch_bounds__(NT, 1)
@@ -162,6 +165,7 @@ __global__ void __launch_bounds__(NT, 1)
         ptx::prefetch_tmap(&maps.k);
         ptx::prefetch_tmap(&maps.v);
         ptx::prefetch_tmap(&maps.la);
+        ptx::prefetch_tmap(&maps.o);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -250,8 +254,9 @@ __global__ void __launch_bounds__(NT, 1)
             }
             ptx::tmem_wait_st();
         }
-        // ---- P1 of chunk cj: g = running sum of log alpha per channel, in place over
-        // the log alpha tile, and the chunk's vectors (buffer cj & 1): g_m, e^{g_m},
+        // ---- P1 of chunk cj: g = running sum of log alpha per channel, in base 2 (g log2 e)
+        // in place over the log alpha tile, and the chunk's vectors (buffer cj & 1): g_m
+        // (base 2), e^{g_m},
         // e^{g_L - g_m}, the factors of the pass over R and beta.  One channel per
         // thread; beta is read from global memory one chunk ahead (a register).
         auto load_beta = [&](int cj) {
@@ -270,14 +275,15 @@ __global__ void __launch_bounds__(NT, 1)
             float x[C];
 #pragma unroll
             for (int i = 0; i < C; ++i) x[i] = (i < L) ? *reinterpret_cast<const float *>(col + sw(i, lch)) : 0.f;
+            x[0] *= kLog2e;
 #pragma unroll
-            for (int i = 1; i < C; ++i) x[i] += x[i - 1];
+            for (int i = 1; i < C; ++i) x[i] = fmaf(x[i], kLog2e, x[i - 1]);
             float gmid = 0.f;
 #pragma unroll
             for (int i = 0; i < C; ++i) gmid = (i == rm) ? x[i] : gmid;
 #pragma unroll
             for (int i = 0; i < C; ++i) *reinterpret_cast<float *>(col + sw(i, lch)) = x[i];
-            const float e = expf(gmid), ecm = expf(x[C - 1] - gmid);  // rows >= L add 0
+            const float e = exp2f(gmid), ecm = exp2f(x[C - 1] - gmid);  // rows >= L add 0
             vec(par, VEC_GM)[c] = gmid;
             vec(par, VEC_EGM)[c] = e;
             vec(par, VEC_ECM)[c] = ecm;
@@ -333,6 +339,7 @@ __global__ void __launch_bounds__(NT, 1)
                 ptx::tmem_wait_st();
             }
             ptx::tc_fence_before();
+            if (leader) ptx::bulk_wait_read0();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
             if (leader) {
                 cwait(CNT_ROWS, ci + 1);  // [Kt; Qt] of this chunk
@@ -360,29 +367,23 @@ __global__ void __launch_bounds__(NT, 1)
                 if (has_next && mwait(B_M1, ci, false)) load_qk(s + C);
             }
 
-            // ---- E2: Y^T = -Z[:, :64] = V^T - (K e^{g} S)^T -> fp16 operand (rows i >= L
-            // of V are never used: T's columns i >= L are zero).
+            // ---- E2: Y^T = -Z[:, :64] = V^T - (K e^{g} S)^T -> fp16 pairs in TMEM, the A
+            // operand of M3 (rows i >= L of V are never used: T's columns i >= L are zero).
             {
-                uint32_t vz[2][32];
-                const int j = row;
+                uint32_t vz[2][32], pk[16];
                 ptx::tmem_ld32(tl + TZ, vz[0]);
                 ptx::tmem_ld32(tl + TZ + 32, vz[1]);
                 ptx::tmem_wait_ld();
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
 #pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        uint32_t pk[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int e = 8 * qq + 2 * e2;
-                            pk[e2] = pack_h2(-__uint_as_float(vz[p][e]), -__uint_as_float(vz[p][e + 1]));
-                        }
-                        *reinterpret_cast<uint4 *>(sm + OFF_Y + sw(j, 4 * p + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    }
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_h2(-__uint_as_float(vz[p][2 * e]), -__uint_as_float(vz[p][2 * e + 1]));
+                    ptx::tmem_st16(tl + TY16 + 16 * p, pk);
                 }
+                ptx::tmem_wait_st();
             }
-            ptx::fence_proxy_async_smem();
+            ptx::tc_fence_before();
             // P1 of the next chunk.  Its vectors go to the buffer of chunk ci - 1, which the
             // prep group last read in E1 of chunk ci - 1, before its rows of chunk ci.
             if (has_next) scan(ci + 1);
@@ -415,33 +416,26 @@ __global__ void __launch_bounds__(NT, 1)
                 ptx::st_release(cnt + CNT_TW, ci + 1);
                 ptx::tc_fence_after();
                 for (int ks = 0; ks < 4; ++ks)
-                    ptx::mma_ss(tbase + TU, ptx::sdesc_sw128(sb + OFF_Y + 32 * ks), ptx::sdesc_sw128(sb + OFF_T + 32 * ks),
-                                IDESC_N64, ks > 0);
+                    ptx::mma_ts(tbase + TU, tbase + TY16 + 8 * ks, ptx::sdesc_sw128(sb + OFF_T + 32 * ks), IDESC_N64,
+                                ks > 0);
                 commit(B_M3);
             }
             mwait(B_M3, ci, leader);
             ptx::tc_fence_after();
-            {  // E3: U^T -> fp16 operand
-                uint32_t vu[2][32];
+            {  // E3: U^T -> fp16 pairs in TMEM, the A operand of M4 and M5
+                uint32_t vu[2][32], pk[16];
                 ptx::tmem_ld32(tl + TU, vu[0]);
                 ptx::tmem_ld32(tl + TU + 32, vu[1]);
                 ptx::tmem_wait_ld();
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
-                    const uint32_t(&v)[32] = vu[p];
 #pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        uint32_t pk[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int e = 8 * qq + 2 * e2;
-                            pk[e2] = pack_h2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-                        }
-                        *reinterpret_cast<uint4 *>(sm + OFF_U + sw(row, 4 * p + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    }
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_h2(__uint_as_float(vu[p][2 * e]), __uint_as_float(vu[p][2 * e + 1]));
+                    ptx::tmem_st16(tl + TU16 + 16 * p, pk);
                 }
+                ptx::tmem_wait_st();
             }
-            ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
 
@@ -450,19 +444,21 @@ __global__ void __launch_bounds__(NT, 1)
                 ptx::tc_fence_after();
                 const uint32_t kb_base = OFF_KB + par * 16384, p_base = OFF_P + par * 8192;
                 for (int ks = 0; ks < 4; ++ks)
-                    ptx::mma_ss(tbase + TS, ptx::sdesc_sw128(sb + OFF_U + 32 * ks),
-                                ptx::sdesc_sw128_mn(sb + kb_base + 2048 * ks, 8192, 1024), IDESC_N128_BMN, 1u);
+                    ptx::mma_ts(tbase + TS, tbase + TU16 + 8 * ks, ptx::sdesc_sw128_mn(sb + kb_base + 2048 * ks, 8192, 1024),
+                                IDESC_N128_BMN, 1u);
                 for (int ks = 0; ks < 4; ++ks)
-                    ptx::mma_ss(tbase + TZ + 64, ptx::sdesc_sw128(sb + OFF_U + 32 * ks),
-                                ptx::sdesc_sw128(sb + p_base + 32 * ks), IDESC_N64, 1u);
+                    ptx::mma_ts(tbase + TZ + 64, tbase + TU16 + 8 * ks, ptx::sdesc_sw128(sb + p_base + 32 * ks), IDESC_N64,
+                                1u);
                 commit(B_M45);
             }
             mwait(B_M45, ci, leader);
             ptx::tc_fence_after();
             if (leader) ptx::st_release(cnt + CNT_M45, ci + 1);
-            {  // E4: outputs of this chunk, staged (bf16, row-major) over the Y^T tile
+            {  // E4: outputs of this chunk, staged over the Y^T tile as two 128-byte swizzled
+               // boxes (columns 0-63, 64-127)
                 uint32_t vo[2][32];
-                __nv_bfloat16 *stage = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_Y);
+                uint8_t *stage = sm + OFF_Y + (row >> 6) * 8192 + (row & 7) * 2;
+                const int ch = (row & 63) >> 3;
                 ptx::tmem_ld32(tl + TZ + 64, vo[0]);
                 ptx::tmem_ld32(tl + TZ + 96, vo[1]);
                 ptx::tmem_wait_ld();
@@ -470,19 +466,28 @@ __global__ void __launch_bounds__(NT, 1)
                 for (int p = 0; p < 2; ++p)
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
-                        stage[(32 * p + e) * D + row] = __float2bfloat16_rn(__uint_as_float(vo[p][e]));
+                        *reinterpret_cast<__nv_bfloat16 *>(stage + sw(32 * p + e, ch)) =
+                            __float2bfloat16_rn(__uint_as_float(vo[p][e]));
             }
+            ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
-            {  // rows r < L of the staged outputs, 16 bytes per thread
-                const uint4 *src = reinterpret_cast<const uint4 *>(sm + OFF_Y);
+            if (L == C) {  // a full chunk: two TMA tile stores
+                if (leader) {
+                    ptx::tma_store_3d(&maps.o, sm + OFF_Y, 0, h, s);
+                    ptx::tma_store_3d(&maps.o, sm + OFF_Y + 8192, 64, h, s);
+                    ptx::bulk_commit_group();
+                }
+            } else {  // rows r < L (the later rows belong to the next sequence), 16 bytes per thread
                 char *dst = static_cast<char *>(a.o) + (size_t(s) * H + h) * D * 2;
                 for (int t = tid; t < L * 16; t += NS) {
                     const int r = t >> 4, q = t & 15;
-                    *reinterpret_cast<uint4 *>(dst + size_t(r) * H * D * 2 + q * 16) = src[r * 16 + q];
+                    *reinterpret_cast<uint4 *>(dst + size_t(r) * H * D * 2 + q * 16) =
+                        *reinterpret_cast<const uint4 *>(sm + OFF_Y + (q >> 3) * 8192 + sw(r, q & 7));
                 }
             }
-            // the staged tile is rewritten by the next E2 only after the next E0 barrier
+            // the staged tile is rewritten by the next E2 only after the next E0 barrier, before
+            // which the leader waits for the tile stores' reads
         }
         // Final state S_final[c][j] = R[j][c] e^{g_L - g_m}[c] of the last chunk.
         if (!*reinterpret_cast<volatile int *>(s_abort)) {
@@ -499,6 +504,7 @@ __global__ void __launch_bounds__(NT, 1)
                 }
             }
         }
+        if (leader) ptx::bulk_wait0();
     } else {
         // =================================================================== prep group
         ptx::regs_dec<128>();
@@ -542,28 +548,30 @@ __global__ void __launch_bounds__(NT, 1)
                     const float4 gb = *reinterpret_cast<const float4 *>(sm + OFF_LA + box * 8192 + sw(r, lch + 1));
                     const float4 m0 = *reinterpret_cast<const float4 *>(gm + c0);
                     const float4 m1 = *reinterpret_cast<const float4 *>(gm + c0 + 4);
-                    const float dg[8] = {ga.x - m0.x, ga.y - m0.y, ga.z - m0.z, ga.w - m0.w,
-                                         gb.x - m1.x, gb.y - m1.y, gb.z - m1.z, gb.w - m1.w};
-                    const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
-                    const uint32_t qw[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
-                    uint32_t o_kt[4], o_qt[4], o_kb[4];
+                    uint32_t o_kt[4] = {0u, 0u, 0u, 0u}, o_qt[4] = {0u, 0u, 0u, 0u}, o_kb[4] = {0u, 0u, 0u, 0u};
+                    if (valid) {  // rows >= L stay zero
+                        const float dg[8] = {ga.x - m0.x, ga.y - m0.y, ga.z - m0.z, ga.w - m0.w,
+                                             gb.x - m1.x, gb.y - m1.y, gb.z - m1.z, gb.w - m1.w};  // base 2
+                        const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
+                        const uint32_t qw[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
 #pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        float kt[2], qt[2], kbv[2];
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            float kt[2], qt[2], kbv[2];
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int e = 2 * e2 + u;
-                            const float kv = u ? bf16_hi(kw[e2]) : bf16_lo(kw[e2]);
-                            const float qv = u ? bf16_hi(qw[e2]) : bf16_lo(qw[e2]);
-                            const float up = __expf(dg[e]);
-                            const float dn = __expf(-dg[e]);
-                            kt[u] = valid ? kv * up : 0.f;
-                            qt[u] = valid ? qv * up : 0.f;
-                            kbv[u] = valid ? kv * dn : 0.f;
+                            for (int u = 0; u < 2; ++u) {
+                                const int e = 2 * e2 + u;
+                                const float kv = u ? bf16_hi(kw[e2]) : bf16_lo(kw[e2]);
+                                const float qv = u ? bf16_hi(qw[e2]) : bf16_lo(qw[e2]);
+                                const float up = ptx::ex2_approx(dg[e]);
+                                const float dn = ptx::ex2_approx(-dg[e]);
+                                kt[u] = kv * up;
+                                qt[u] = qv * up;
+                                kbv[u] = kv * dn;
+                            }
+                            o_kt[e2] = pack_h2(kt[0], kt[1]);
+                            o_qt[e2] = pack_h2(qt[0], qt[1]);
+                            o_kb[e2] = pack_h2(kbv[0], kbv[1]);
                         }
-                        o_kt[e2] = pack_h2(kt[0], kt[1]);
-                        o_qt[e2] = pack_h2(qt[0], qt[1]);
-                        o_kb[e2] = pack_h2(kbv[0], kbv[1]);
                     }
                     *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + ph16) = make_uint4(o_kt[0], o_kt[1], o_kt[2], o_kt[3]);
                     *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + 8192 + ph16) = make_uint4(o_qt[0], o_qt[1], o_qt[2], o_qt[3]);
@@ -629,10 +637,12 @@ __global__ void __launch_bounds__(NT, 1)
             ptx::tc_fence_before();
             if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
 
-            // ---- T = (I + A)^{-1} Diag(beta).  X = (I + A)^{-1} in 16x16 blocks: the four
-            // diagonal blocks by column substitution in registers (one warp each), then
-            // E_bk = X_bb A_bk for k < b, then the blocks below the diagonal by distance d,
-            // X_{b,b-d} = -sum_{k=b-d}^{b-1} E_bk X_{k,b-d}.
+            // ---- T = (I + A)^{-1} Diag(beta).  X = (I + A)^{-1} by block doubling: the four
+            // diagonal 16x16 blocks by column substitution in registers (one warp each); then
+            // the two 32x32 diagonal halves, X_10 = -(X_11 A_10) X_00 and X_32 = -(X_33 A_32) X_22;
+            // then the lower-left half, X_21 = -(X_H1 A_21) X_H0 over 32x32 halves.  The
+            // inverse of a unit lower-triangular block matrix [[L0, 0], [B, L1]] is
+            // [[L0^-1, 0], [-L1^-1 B L0^-1, L1^-1]].
             {
                 const float *Af = reinterpret_cast<const float *>(sm + OFF_AF);
                 float *X = reinterpret_cast<float *>(sm + OFF_XF);
@@ -655,60 +665,91 @@ __global__ void __launch_bounds__(NT, 1)
                     }
                 }
                 ptx::named_barrier(BAR_P, NP);
-                // one task = one row of a 16x16 block, 8 columns (two per block row);
-                // E block e = b(b-1)/2 + k holds X_bb A_bk: 0:(1,0) 1:(2,0) 2:(2,1) 3:(3,0) 4:(3,1) 5:(3,2)
-                if (pt < 6 * 32) {
-                    const int e = pt >> 5, rowb = (pt & 31) >> 1, c8 = 8 * (pt & 1);
-                    const int b = e == 0 ? 1 : (e < 3 ? 2 : 3);
-                    const int k = e - b * (b - 1) / 2;
-                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                {  // E_h = X_{b1 b1} A_{b1 b0} (16x16, h = 0: b = 1, 0; h = 1: b = 3, 2); two columns a thread.
+                   // Diagonal blocks of X hold zeros above their diagonal.
+                    const int hh = pt >> 7, r = (pt >> 3) & 15, c2 = 2 * (pt & 7);
+                    const int b1 = 2 * hh + 1, b0 = 2 * hh;
+                    float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) {  // X_bb is zero above its diagonal
-                        const float xv = X[(16 * b + rowb) * LDF + 16 * b + m];
-                        const float4 a0 = *reinterpret_cast<const float4 *>(Af + (16 * b + m) * LDF + 16 * k + c8);
-                        const float4 a1 = *reinterpret_cast<const float4 *>(Af + (16 * b + m) * LDF + 16 * k + c8 + 4);
-                        acc[0] = fmaf(xv, a0.x, acc[0]);
-                        acc[1] = fmaf(xv, a0.y, acc[1]);
-                        acc[2] = fmaf(xv, a0.z, acc[2]);
-                        acc[3] = fmaf(xv, a0.w, acc[3]);
-                        acc[4] = fmaf(xv, a1.x, acc[4]);
-                        acc[5] = fmaf(xv, a1.y, acc[5]);
-                        acc[6] = fmaf(xv, a1.z, acc[6]);
-                        acc[7] = fmaf(xv, a1.w, acc[7]);
+                    for (int m = 0; m < 16; ++m) {
+                        const float xv = X[(16 * b1 + r) * LDF + 16 * b1 + m];
+                        const float2 av = *reinterpret_cast<const float2 *>(Af + (16 * b1 + m) * LDF + 16 * b0 + c2);
+                        a0 = fmaf(xv, av.x, a0);
+                        a1 = fmaf(xv, av.y, a1);
                     }
-                    float *eo = E + (e * 16 + rowb) * LDE + c8;
-                    *reinterpret_cast<float4 *>(eo) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-                    *reinterpret_cast<float4 *>(eo + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                    *reinterpret_cast<float2 *>(E + (16 * hh + r) * LDE + c2) = make_float2(a0, a1);
                 }
                 ptx::named_barrier(BAR_P, NP);
-                for (int d = 1; d <= 3; ++d) {
-                    if (pt < (4 - d) * 32) {
-                        const int bj = pt >> 5, b = bj + d, rowb = (pt & 31) >> 1, c8 = 8 * (pt & 1);
-                        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                        for (int k = bj; k < b; ++k) {
-                            const float *eb = E + ((b * (b - 1) / 2 + k) * 16 + rowb) * LDE;
+                {  // X_{b1 b0} = -E_h X_{b0 b0}
+                    const int hh = pt >> 7, r = (pt >> 3) & 15, c2 = 2 * (pt & 7);
+                    const int b1 = 2 * hh + 1, b0 = 2 * hh;
+                    float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-                            for (int m = 0; m < 16; ++m) {
-                                const float ev = eb[m];
-                                const float *xr = X + (16 * k + m) * LDF + 16 * bj + c8;
-                                const float4 x0 = *reinterpret_cast<const float4 *>(xr);
-                                const float4 x1 = *reinterpret_cast<const float4 *>(xr + 4);
-                                acc[0] = fmaf(ev, x0.x, acc[0]);
-                                acc[1] = fmaf(ev, x0.y, acc[1]);
-                                acc[2] = fmaf(ev, x0.z, acc[2]);
-                                acc[3] = fmaf(ev, x0.w, acc[3]);
-                                acc[4] = fmaf(ev, x1.x, acc[4]);
-                                acc[5] = fmaf(ev, x1.y, acc[5]);
-                                acc[6] = fmaf(ev, x1.z, acc[6]);
-                                acc[7] = fmaf(ev, x1.w, acc[7]);
-                            }
-                        }
-                        float *xo = X + (16 * b + rowb) * LDF + 16 * bj + c8;
-                        *reinterpret_cast<float4 *>(xo) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-                        *reinterpret_cast<float4 *>(xo + 4) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
+                    for (int m = 0; m < 16; ++m) {
+                        const float ev = E[(16 * hh + r) * LDE + m];
+                        const float2 xv = *reinterpret_cast<const float2 *>(X + (16 * b0 + m) * LDF + 16 * b0 + c2);
+                        a0 = fmaf(ev, xv.x, a0);
+                        a1 = fmaf(ev, xv.y, a1);
                     }
-                    ptx::named_barrier(BAR_P, NP);
+                    *reinterpret_cast<float2 *>(X + (16 * b1 + r) * LDF + 16 * b0 + c2) = make_float2(-a0, -a1);
                 }
+                ptx::named_barrier(BAR_P, NP);
+                {  // F = X_H1 A_21 (32x32; X_H1 = X[32:64, 32:64] is zero above its diagonal, and
+                   // its upper-right 16x16 block is never read); F[r][c] at E[r * LDG + c]
+                    const int r = pt >> 3, c4 = 4 * (pt & 7);
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    const float *xr = X + (32 + r) * LDF + 32;
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        const float xv = xr[m];
+                        const float4 av = *reinterpret_cast<const float4 *>(Af + (32 + m) * LDF + c4);
+                        acc[0] = fmaf(xv, av.x, acc[0]);
+                        acc[1] = fmaf(xv, av.y, acc[1]);
+                        acc[2] = fmaf(xv, av.z, acc[2]);
+                        acc[3] = fmaf(xv, av.w, acc[3]);
+                    }
+                    if (r >= 16) {  // uniform over a warp
+#pragma unroll
+                        for (int m = 16; m < 32; ++m) {
+                            const float xv = xr[m];
+                            const float4 av = *reinterpret_cast<const float4 *>(Af + (32 + m) * LDF + c4);
+                            acc[0] = fmaf(xv, av.x, acc[0]);
+                            acc[1] = fmaf(xv, av.y, acc[1]);
+                            acc[2] = fmaf(xv, av.z, acc[2]);
+                            acc[3] = fmaf(xv, av.w, acc[3]);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) E[r * LDG + c4 + q] = acc[q];
+                }
+                ptx::named_barrier(BAR_P, NP);
+                {  // X_21 = -F X_H0 (X_H0 = X[0:32, 0:32]; its upper-right block is never read)
+                    const int r = pt & 31, c4 = 4 * (pt >> 5);
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    const float *fr = E + r * LDG;
+                    if (c4 < 16) {  // uniform over a warp
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) {
+                            const float fv = fr[m];
+                            const float4 xv = *reinterpret_cast<const float4 *>(X + m * LDF + c4);
+                            acc[0] = fmaf(fv, xv.x, acc[0]);
+                            acc[1] = fmaf(fv, xv.y, acc[1]);
+                            acc[2] = fmaf(fv, xv.z, acc[2]);
+                            acc[3] = fmaf(fv, xv.w, acc[3]);
+                        }
+                    }
+#pragma unroll
+                    for (int m = 16; m < 32; ++m) {
+                        const float fv = fr[m];
+                        const float4 xv = *reinterpret_cast<const float4 *>(X + m * LDF + c4);
+                        acc[0] = fmaf(fv, xv.x, acc[0]);
+                        acc[1] = fmaf(fv, xv.y, acc[1]);
+                        acc[2] = fmaf(fv, xv.z, acc[2]);
+                        acc[3] = fmaf(fv, xv.w, acc[3]);
+                    }
+                    *reinterpret_cast<float4 *>(X + (32 + r) * LDF + c4) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+                }
+                ptx::named_barrier(BAR_P, NP);
             }
             // X (fp32) is handed to the state group, which forms T = X Diag(beta)
             if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
@@ -771,7 +812,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
     if (!make_map(&maps.q, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens) ||
         !make_map(&maps.k, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens) ||
         !make_map(&maps.v, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens) ||
-        !make_map(&maps.la, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.H, a.total_tokens))
+        !make_map(&maps.la, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.H, a.total_tokens) ||
+        !make_map(&maps.o, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens))
         return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            int(SMEM_ALLOC));
