@@ -399,13 +399,17 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll
                 for (int qq = 0; qq < 4; ++qq) {
                     const int ch = 4 * part + qq;
+                    const float4 x0 = *reinterpret_cast<const float4 *>(X + rt * LDF + 8 * ch);
+                    const float4 x1 = *reinterpret_cast<const float4 *>(X + rt * LDF + 8 * ch + 4);
+                    const float4 b0 = *reinterpret_cast<const float4 *>(beta + 8 * ch);
+                    const float4 b1 = *reinterpret_cast<const float4 *>(beta + 8 * ch + 4);
+                    const float xs[8] = {x0.x * b0.x, x0.y * b0.y, x0.z * b0.z, x0.w * b0.w,
+                                         x1.x * b1.x, x1.y * b1.y, x1.z * b1.z, x1.w * b1.w};
                     uint32_t pk[4];
 #pragma unroll
                     for (int e2 = 0; e2 < 4; ++e2) {
                         const int i = 8 * ch + 2 * e2;
-                        const float x0 = (i <= rt) ? X[rt * LDF + i] * beta[i] : 0.f;
-                        const float x1 = (i + 1 <= rt) ? X[rt * LDF + i + 1] * beta[i + 1] : 0.f;
-                        pk[e2] = pack_h2(x0, x1);
+                        pk[e2] = pack_h2(i <= rt ? xs[2 * e2] : 0.f, i + 1 <= rt ? xs[2 * e2 + 1] : 0.f);
                     }
                     *reinterpret_cast<uint4 *>(sm + OFF_T + sw(rt, ch)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
@@ -653,11 +657,17 @@ __global__ void __launch_bounds__(NT, 1)
                     const float *ab = Af + (16 * b) * LDF + 16 * b;
                     float x[16];
 #pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == jj) ? 1.f : 0.f;
+                    for (int rr = 0; rr < 16; ++rr) {  // x_rr = [rr == jj] - sum_{ss < rr} A_bb[rr][ss] x_ss
+                        float acc = (rr == jj) ? 1.f : 0.f;
 #pragma unroll
-                    for (int ss = 0; ss < 16; ++ss) {  // x[ss] is final: eliminate it below
+                        for (int s4 = 0; s4 < rr; s4 += 4) {
+                            const float4 a4 = *reinterpret_cast<const float4 *>(ab + rr * LDF + s4);
+                            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                        for (int rr = ss + 1; rr < 16; ++rr) x[rr] = fmaf(-ab[rr * LDF + ss], x[ss], x[rr]);
+                            for (int u = 0; u < 4; ++u)
+                                if (s4 + u < rr) acc = fmaf(-av[u], x[s4 + u], acc);
+                        }
+                        x[rr] = acc;
                     }
                     if (lane < 16) {
 #pragma unroll
