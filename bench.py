@@ -19,6 +19,7 @@ has) on the host cores over a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -54,6 +55,32 @@ def prefill_bytes_per_head_token(dk, dv, qkv_bytes):
 
 def decode_bytes_per_head_step(dk, dv, qkv_bytes):
     return 2 * 4 * dk * dv + prefill_bytes_per_head_token(dk, dv, qkv_bytes)
+
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one ncu capture per
+# kernel, with the SHA-256 of the kernel's source file at capture time.  A launch's
+# traffic is the capture's bytes scaled by the units (head-tokens) the launch
+# processes, and is reported as null once the source differs from the captured one.
+# Prefill: one launch on 2 x 8192 tokens x 32 heads (524,288 head-tokens).
+MEASURED_TRAFFIC = {
+    "prefill_tc": {"source": "gated_delta_rule_126_b200/csrc/kda_prefill_tc.cu",
+                   "sha256": "92c410c3acb0b10e4ea05ba53d7a7f6af863449f41b8e51563394789b9d86fde",
+                   "units": 2 * 8192 * 32, "dram_bytes": 673498112 + 121482752},
+}
+
+
+def measured_traffic(kernel, units):
+    rec = MEASURED_TRAFFIC.get(kernel)
+    if rec is None:
+        return None
+    try:
+        with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    if digest != rec["sha256"]:
+        return None
+    return rec["dram_bytes"] * units / rec["units"]
 
 
 def load_peaks():
@@ -283,8 +310,9 @@ def run_ours(args):
     achieved_gbs = alg_bytes / t_launch / 1e9
     achieved_tf = alg_flops / t_launch / 1e12
     t_roof = max(alg_bytes / (hbm_peak * 1e9), alg_flops / (tc_peak * 1e12))
+    traffic = measured_traffic("prefill_tc", head_tokens) if w.dtype == "bf16" else None
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved_gbs / hbm_peak, "traffic": None,
+                "frac": achieved_gbs / hbm_peak, "traffic": traffic,
                 "peak_source": f"{peak_kind} hbm_gbs (copy, burst)",
                 "alg_bytes_per_launch": alg_bytes, "alg_flops_per_launch": alg_flops,
                 "tensor": {"achieved": achieved_tf, "peak": tc_peak, "unit": "TFLOP/s",
