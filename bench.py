@@ -264,7 +264,7 @@ def run_reference(args):
 
 def run_ours(args):
     from gated_delta_rule_126_b200 import (kda_decode_step, kda_decode_tokens, kda_prefill,
-                                           prefill_workspace_size)
+                                           kda_prefill_gated, prefill_workspace_size)
     world, rank, local = dist_setup("nccl")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -358,6 +358,33 @@ def run_ours(args):
                "d2h_bytes_per_step": d2h, "steps": e_steps}
         del host, dbuf, h_o, h_S
 
+    # the same prefill with the layer's output epilogue (sigmoid gate + RMSNorm) fused
+    # into the output store: one more bf16 read (the gate) per head-token, same launches
+    gated = None
+    if not args.no_gated and w.dtype == "bf16" and w.dk == 128 and w.dv == 128 and w.chunk == 64:
+        gate, g_w = inputs.gate_inputs(T, w.H, w.dv, w.dtype, seed=w.seed + 7 + 1000 * rank, device=dev)
+        y = torch.empty_like(o)
+
+        def gstep():
+            kda_prefill_gated(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                              inp["cu_seqlens"], gate, g_w, 1e-6, cu_seqlens_host=cu_host,
+                              S0=inp["S0"], chunk=w.chunk, y=y, S_final=S_final, workspace=ws,
+                              stream=stream)
+
+        for _ in range(args.warmup):
+            gstep()
+        barrier(world)
+        g_el = max_over_ranks(time_region(gstep, args.steps, stream), world)
+        g_t = g_el / args.steps
+        g_bytes = alg_bytes + head_tokens * w.dv * qkv_bytes
+        g_gbs = g_bytes / g_t / 1e9
+        gated = {"value": weak_scaling_value(T, args.steps, g_el, world), "unit": UNIT,
+                 "ms_per_step": g_t * 1e3, "epilogue": "y = o / sqrt(mean(o^2) + 1e-6) * w * sigmoid(gate)",
+                 "gpu_launches_per_step": 2,
+                 "roofline": {"bound": "hbm", "achieved": g_gbs, "peak": hbm_peak, "unit": "GB/s",
+                              "frac": g_gbs / hbm_peak, "alg_bytes_per_launch": g_bytes}}
+        del gate, g_w, y
+
     # decode: 256 sequences x 32 heads, 64 consecutive one-token steps
     decode = None
     if not args.no_decode:
@@ -436,7 +463,8 @@ def run_ours(args):
                     "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                     "l2": "inputs larger than L2 (no flush)"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": 2 * args.steps, "clocks": clk.summary(), "decode": decode}
+                "gpu_launches": 2 * args.steps, "clocks": clk.summary(), "decode": decode,
+                "gated_epilogue": gated}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -455,6 +483,7 @@ def main():
                     help="size of the oracle's timed sample in head-tokens")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-gated", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps

@@ -6,6 +6,8 @@ in ``include/kda.h`` (library ``lib/libkda_b200.so``, built by
 binding over that ABI, with the same names:
 
 * ``kda_prefill``     -- chunked prefill over packed variable-length sequences;
+* ``kda_prefill_gated`` -- the same with the layer's output epilogue (sigmoid gate
+  and RMSNorm) applied to o;
 * ``kda_decode_step`` -- one recurrent decode step for a batch of sequences;
 * ``kda_decode_tokens`` -- n tokens per sequence with states in a slot pool;
 * ``prefill_workspace_size``, ``workspace_status``, ``KdaError``.
@@ -13,8 +15,8 @@ binding over that ABI, with the same names:
 ``inputs`` holds the seeded synthetic input generators.  Importing the package
 does not load the CUDA library; the first call does, and raises if it is missing.
 """
-from ._binding import (KdaError, kda_decode_step, kda_decode_tokens, kda_prefill, load,
-                       prefill_workspace_size, workspace_status)
+from ._binding import (KdaError, kda_decode_step, kda_decode_tokens, kda_prefill,
+                       kda_prefill_gated, load, prefill_workspace_size, workspace_status)
 
-__all__ = ["KdaError", "kda_decode_step", "kda_decode_tokens", "kda_prefill", "load",
-           "prefill_workspace_size", "workspace_status"]
+__all__ = ["KdaError", "kda_decode_step", "kda_decode_tokens", "kda_prefill", "kda_prefill_gated",
+           "load", "prefill_workspace_size", "workspace_status"]

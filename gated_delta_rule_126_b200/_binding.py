@@ -45,6 +45,9 @@ def _declare(lib):
     lib.kda_prefill.restype = i32
     lib.kda_prefill.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                 vp, vp, vp, sz, vp]
+    lib.kda_prefill_gated.restype = i32
+    lib.kda_prefill_gated.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                      vp, vp, c.c_float, vp, vp, vp, sz, vp]
     lib.kda_decode_step.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, vp]
     lib.kda_decode_tokens.restype = i32
@@ -150,6 +153,58 @@ def kda_prefill(q, k, v, log_alpha, beta, cu_seqlens, cu_seqlens_host=None, S0=N
                              _stream_handle(stream))
     _check(st, "kda_prefill")
     return o, S_final
+
+
+def kda_prefill_gated(q, k, v, log_alpha, beta, cu_seqlens, gate, norm_weight, eps=1e-6,
+                      cu_seqlens_host=None, S0=None, chunk=64, y=None, S_final=None, workspace=None,
+                      stream=None):
+    """Chunked prefill with the output epilogue (see ``kda_prefill_gated`` in kda.h).
+
+    As ``kda_prefill``, plus gate [T,H,d_v] (dtype of q), norm_weight [d_v] float32 and
+    eps > 0; returns ``(y, S_final)`` with y = o / sqrt(mean(o^2) + eps) * w * sigmoid(gate).
+    """
+    lib = load()
+    dev = q.device
+    dt = q.dtype
+    if dt not in DTYPE_CODE:
+        raise ValueError("q/k/v dtype must be float32 or bfloat16")
+    _need(q, "q", dt)
+    T, H, dk = q.shape
+    _need(k, "k", dt, dev)
+    _need(v, "v", dt, dev)
+    dv = v.shape[2]
+    _need(log_alpha, "log_alpha", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    _need(gate, "gate", dt, dev)
+    _need(norm_weight, "norm_weight", torch.float32, dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu()
+    cu_h = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
+    N = cu_h.numel() - 1
+    if cu_seqlens.numel() != N + 1:
+        raise ValueError("cu_seqlens and cu_seqlens_host differ in length")
+    if y is None:
+        y = torch.empty(T, H, dv, dtype=dt, device=dev)
+    if S_final is None:
+        S_final = torch.empty(N, H, dk, dv, dtype=torch.float32, device=dev)
+    _need(y, "y", dt, dev)
+    _need(S_final, "S_final", torch.float32, dev)
+    ws_bytes = prefill_workspace_size(N, T, H, dk, dv, chunk, dt)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = lib.kda_prefill_gated(_ptr(q), _ptr(k), _ptr(v), DTYPE_CODE[dt], _ptr(log_alpha),
+                                   _ptr(beta), _ptr(S0), _ptr(cu_seqlens),
+                                   ctypes.c_void_p(cu_h.data_ptr()), N, H, dk, dv, int(chunk),
+                                   _ptr(gate), _ptr(norm_weight), float(eps), _ptr(y),
+                                   _ptr(S_final), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(),
+                                   _stream_handle(stream))
+    _check(st, "kda_prefill_gated")
+    return y, S_final
 
 
 def kda_decode_step(q, k, v, log_alpha, beta, S, o=None, stream=None):

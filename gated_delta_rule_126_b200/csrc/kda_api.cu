@@ -1,5 +1,6 @@
 // C-ABI entry points of the KDA library: argument checks on the host, then
 // kernel launches on the caller's stream.  See include/kda.h for the contract.
+#include <cmath>
 #include <cstring>
 
 #include "kda_internal.h"
@@ -19,6 +20,52 @@ kda_status_t check_prefill_shape(int num_seqs, int H, int d_k, int d_v, int chun
     if (num_seqs < 0 || H < 1 || d_k < 1 || d_v < 1 || !dtype_ok(dt)) return KDA_ERR_INVALID_ARG;
     if (chunk != 16 && chunk != 32 && chunk != 64) return KDA_ERR_UNSUPPORTED;
     if (d_k > 128 || d_v > 128) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+// Checks shared by kda_prefill and kda_prefill_gated; fills `a` (o = out).  Sets
+// *empty when there is nothing to launch (num_seqs == 0).
+kda_status_t prepare_prefill(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                             const float *log_alpha, const float *beta, const float *S0,
+                             const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int num_seqs, int H,
+                             int d_k, int d_v, int chunk, void *out, float *S_final, void *workspace,
+                             size_t workspace_bytes, kda::PrefillArgs &a, bool *empty) {
+    const kda_status_t shape = check_prefill_shape(num_seqs, H, d_k, d_v, chunk, qkv_dtype);
+    if (shape != KDA_OK) return shape;
+    if (!cu_seqlens_host || !cu_seqlens_dev || !S_final) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens_host[0] != 0) return KDA_ERR_INVALID_ARG;
+    int max_len = 0;
+    for (int n = 0; n < num_seqs; ++n) {
+        const int64_t len = int64_t(cu_seqlens_host[n + 1]) - cu_seqlens_host[n];
+        if (len < 0) return KDA_ERR_INVALID_ARG;
+        if (len > max_len) max_len = int(len);
+    }
+    const int64_t T = cu_seqlens_host[num_seqs];
+    if (T > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(S_final) || (S0 && !aligned16(S0))) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+                  !aligned16(log_alpha)))
+        return KDA_ERR_INVALID_ARG;
+    const kda::WorkspaceLayout wl = kda::workspace_layout(num_seqs);
+    if (!workspace || workspace_bytes < wl.total) return KDA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_WORKSPACE;
+
+    a.q = q; a.k = k; a.v = v; a.dtype = qkv_dtype;
+    a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0;
+    a.cu_seqlens = cu_seqlens_dev;
+    a.num_seqs = num_seqs; a.H = H; a.dk = d_k; a.dv = d_v; a.chunk = chunk;
+    a.total_tokens = T; a.max_seqlen = max_len;
+    a.o = out; a.S_final = S_final;
+    a.status = static_cast<kda::DeviceStatus *>(workspace);
+    a.order = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + wl.order_offset);
+    *empty = num_seqs == 0;
+    return KDA_OK;
+}
+
+// Status reset and the length ordering every prefill launch starts with.
+kda_status_t launch_prefill_prologue(const kda::PrefillArgs &a, cudaStream_t st) {
+    if (cudaMemsetAsync(a.status, 0, sizeof(kda::DeviceStatus), st) != cudaSuccess) return KDA_ERR_CUDA;
+    if (kda::launch_order_by_length(a, st) != cudaSuccess) return KDA_ERR_CUDA;
     return KDA_OK;
 }
 
@@ -53,44 +100,46 @@ kda_status_t kda_prefill(const void *q, const void *k, const void *v, kda_dtype_
                          int num_seqs, int H, int d_k, int d_v, int chunk, void *o,
                          float *S_final, void *workspace, size_t workspace_bytes,
                          kda_stream_t stream) {
-    const kda_status_t shape = check_prefill_shape(num_seqs, H, d_k, d_v, chunk, qkv_dtype);
-    if (shape != KDA_OK) return shape;
-    if (!cu_seqlens_host || !cu_seqlens_dev || !S_final) return KDA_ERR_INVALID_ARG;
-    if (cu_seqlens_host[0] != 0) return KDA_ERR_INVALID_ARG;
-    int max_len = 0;
-    for (int n = 0; n < num_seqs; ++n) {
-        const int64_t len = int64_t(cu_seqlens_host[n + 1]) - cu_seqlens_host[n];
-        if (len < 0) return KDA_ERR_INVALID_ARG;
-        if (len > max_len) max_len = int(len);
-    }
-    const int64_t T = cu_seqlens_host[num_seqs];
-    if (T > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_INVALID_ARG;
-    if (!aligned16(S_final) || (S0 && !aligned16(S0))) return KDA_ERR_INVALID_ARG;
-    if (T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-                  !aligned16(log_alpha)))
-        return KDA_ERR_INVALID_ARG;
-    const kda::WorkspaceLayout wl = kda::workspace_layout(num_seqs);
-    if (!workspace || workspace_bytes < wl.total) return KDA_ERR_WORKSPACE;
-    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_WORKSPACE;
-
     kda::PrefillArgs a;
-    a.q = q; a.k = k; a.v = v; a.dtype = qkv_dtype;
-    a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0;
-    a.cu_seqlens = cu_seqlens_dev;
-    a.num_seqs = num_seqs; a.H = H; a.dk = d_k; a.dv = d_v; a.chunk = chunk;
-    a.total_tokens = T; a.max_seqlen = max_len;
-    a.o = o; a.S_final = S_final;
-    a.status = static_cast<kda::DeviceStatus *>(workspace);
-    a.order = reinterpret_cast<int32_t *>(static_cast<char *>(workspace) + wl.order_offset);
-
+    bool empty = false;
+    const kda_status_t st0 = prepare_prefill(q, k, v, qkv_dtype, log_alpha, beta, S0, cu_seqlens_dev,
+                                             cu_seqlens_host, num_seqs, H, d_k, d_v, chunk, o, S_final,
+                                             workspace, workspace_bytes, a, &empty);
+    if (st0 != KDA_OK || empty) return st0;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (num_seqs == 0) return KDA_OK;
-    cudaError_t err = cudaMemsetAsync(a.status, 0, sizeof(kda::DeviceStatus), st);
-    if (err != cudaSuccess) return KDA_ERR_CUDA;
-    err = kda::launch_order_by_length(a, st);
-    if (err != cudaSuccess) return KDA_ERR_CUDA;
+    const kda_status_t pro = launch_prefill_prologue(a, st);
+    if (pro != KDA_OK) return pro;
     if (kda::prefill_tc_supported(a)) return from_cuda(kda::launch_prefill_tc(a, st));
     return from_cuda(kda::launch_prefill_simt(a, st));
+}
+
+kda_status_t kda_prefill_gated(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                               const float *log_alpha, const float *beta, const float *S0,
+                               const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                               int num_seqs, int H, int d_k, int d_v, int chunk, const void *gate,
+                               const float *norm_weight, float eps, void *y, float *S_final,
+                               void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+    kda::PrefillArgs a;
+    bool empty = false;
+    const kda_status_t st0 = prepare_prefill(q, k, v, qkv_dtype, log_alpha, beta, S0, cu_seqlens_dev,
+                                             cu_seqlens_host, num_seqs, H, d_k, d_v, chunk, y, S_final,
+                                             workspace, workspace_bytes, a, &empty);
+    if (st0 != KDA_OK) return st0;
+    if (!(eps > 0.f) || !std::isfinite(eps)) return KDA_ERR_INVALID_ARG;
+    if (a.total_tokens > 0 && (!gate || !norm_weight || !aligned16(gate))) return KDA_ERR_INVALID_ARG;
+    a.gate = gate;
+    a.norm_weight = norm_weight;
+    a.eps = eps;
+    const bool fused = kda::prefill_tc_supported(a);
+    if (!fused && qkv_dtype != KDA_DTYPE_F32 && a.total_tokens > 0) return KDA_ERR_UNSUPPORTED;
+    if (empty) return KDA_OK;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const kda_status_t pro = launch_prefill_prologue(a, st);
+    if (pro != KDA_OK) return pro;
+    if (fused) return from_cuda(kda::launch_prefill_tc(a, st));
+    const cudaError_t err = kda::launch_prefill_simt(a, st);  // o into y, then the epilogue in place
+    if (err != cudaSuccess) return KDA_ERR_CUDA;
+    return from_cuda(kda::launch_gated_rmsnorm(a, st));
 }
 
 kda_status_t kda_decode_step(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,

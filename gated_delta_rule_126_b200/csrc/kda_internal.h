@@ -45,6 +45,10 @@ struct PrefillArgs {
     float *S_final;
     DeviceStatus *status;
     int32_t *order;       // sequence order (longest first), num_seqs entries
+    // output epilogue (kda_prefill_gated): o is replaced by o / sqrt(mean(o^2) + eps) * w * sigmoid(gate)
+    const void *gate = nullptr;          // [T, H, d_v], dtype; nullptr = plain prefill
+    const float *norm_weight = nullptr;  // [d_v]
+    float eps = 0.f;
 };
 
 struct DecodeArgs {
@@ -70,7 +74,9 @@ cudaError_t launch_order_by_length(const PrefillArgs &a, cudaStream_t stream);
 cudaError_t launch_decode_tokens(const DecodeTokensArgs &a, cudaStream_t stream);
 cudaError_t launch_prefill_simt(const PrefillArgs &a, cudaStream_t stream);
 bool prefill_tc_supported(const PrefillArgs &a);
-cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream);
+cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream);  // fuses the epilogue when a.gate is set
+// The output epilogue in place over a.o (after a prefill that does not fuse it).
+cudaError_t launch_gated_rmsnorm(const PrefillArgs &a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 
 }  // namespace kda

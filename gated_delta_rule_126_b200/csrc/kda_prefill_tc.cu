@@ -82,15 +82,21 @@ constexpr uint32_t VEC_BETA = 1536;   // beta                 64 f32
 constexpr uint32_t VEC_FAC = 1792;    // e^{g_L - g_m}(previous chunk) e^{g_m}: the pass over R
 constexpr uint32_t VEC_BYTES = 2304;
 constexpr uint32_t OFF_BAR = OFF_VEC + 2 * VEC_BYTES;   // mbarriers
-constexpr int NBAR = 7;
-constexpr int B_QK = 0, B_LA = 1, B_V = 2, B_M1 = 3, B_M2 = 4, B_M3 = 5, B_M45 = 6;
+constexpr int NBAR = 8;
+constexpr int B_QK = 0, B_LA = 1, B_V = 2, B_M1 = 3, B_M2 = 4, B_M3 = 5, B_M45 = 6, B_G = 7;
 constexpr uint32_t OFF_CNT = OFF_BAR + 8 * NBAR;        // progress counters
 constexpr int CNT_ROWS = 0, CNT_TP = 1, CNT_SCAN = 2, CNT_M45 = 3, CNT_TW = 4;
 constexpr uint32_t OFF_ISS = OFF_CNT + 32;              // phases issued / waited per mbarrier
 constexpr uint32_t OFF_WT = OFF_ISS + 4 * NBAR;
 constexpr uint32_t OFF_MISC = OFF_WT + 4 * NBAR;        // tmem base, abort flag
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
-constexpr uint32_t SMEM_ALLOC = SMEM_USED + 1024;  // + alignment slack
+// The gated output epilogue adds the gate tile (bf16, two 64 x 64 boxes) and the
+// per-token reduction of o^2 (4 x 64 partial sums, then 64 reciprocal RMS values).
+constexpr uint32_t OFF_G = (SMEM_USED + 1023) / 1024 * 1024;
+constexpr uint32_t OFF_RED = OFF_G + 16384;
+constexpr uint32_t SMEM_USED_G = OFF_RED + 320 * 4;
+constexpr uint32_t smem_alloc(bool gated) { return (gated ? SMEM_USED_G : SMEM_USED) + 1024; }  // + alignment slack
+static_assert(smem_alloc(true) <= 232448, "shared memory");
 
 // Tensor memory columns.
 constexpr uint32_t TS = 0;      // R (fp32)          128 cols   state group
@@ -121,9 +127,13 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 struct TcMaps {
-    CUtensorMap q, k, v, la, o;
+    CUtensorMap q, k, v, la, o, g;  // g: the output gate (gated epilogue only)
 };
 
+// kGated: the output store applies the layer's output epilogue, y = o / sqrt(mean_j o_j^2 + eps)
+// * w * sigmoid(gate) per token and head (the KDA layer's sigmoid output gate and RMSNorm,
+// section "模型架构" of the same page), instead of storing o.
+template <bool kGated>
 __global__ void __launch_bounds__(NT, 1)
     prefill_tc_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -166,6 +176,7 @@ __global__ void __launch_bounds__(NT, 1)
         ptx::prefetch_tmap(&maps.v);
         ptx::prefetch_tmap(&maps.la);
         ptx::prefetch_tmap(&maps.o);
+        if (kGated) ptx::prefetch_tmap(&maps.g);
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -190,6 +201,12 @@ __global__ void __launch_bounds__(NT, 1)
         ptx::tma_load_3d(sm + OFF_V, &maps.v, bars + B_V, 0, h, s);
         ptx::tma_load_3d(sm + OFF_V + 8192, &maps.v, bars + B_V, 64, h, s);
         ++iss[B_V];
+    };
+    auto load_g = [&](int s) {
+        ptx::mbar_arrive_expect_tx(bars + B_G, 2 * 8192);
+        ptx::tma_load_3d(sm + OFF_G, &maps.g, bars + B_G, 0, h, s);
+        ptx::tma_load_3d(sm + OFF_G + 8192, &maps.g, bars + B_G, 64, h, s);
+        ++iss[B_G];
     };
     auto commit = [&](int b) {
         ptx::mma_commit(bars + b);
@@ -234,7 +251,11 @@ __global__ void __launch_bounds__(NT, 1)
         const int row = tid;  // TMEM lane = value column j
         const uint32_t tl = tbase + (uint32_t(warp * 32) << 16);
         const bool leader = tid == 0;
-        if (leader && nchunks > 0) load_v(bos);
+        if (leader && nchunks > 0) {
+            load_v(bos);
+            if (kGated) load_g(bos);
+        }
+        const float w_row = kGated ? a.norm_weight[row] : 0.f;  // RMSNorm weight of value channel `row`
         {  // -I as a K-major bf16 operand (rows r, K = i), for Z[:, :64] = V^T (-I)
             uint4 *id = reinterpret_cast<uint4 *>(sm + OFF_ID);
             for (int t = tid; t < 512; t += NS) id[t] = make_uint4(0u, 0u, 0u, 0u);
@@ -466,16 +487,69 @@ __global__ void __launch_bounds__(NT, 1)
                 ptx::tmem_ld32(tl + TZ + 64, vo[0]);
                 ptx::tmem_ld32(tl + TZ + 96, vo[1]);
                 ptx::tmem_wait_ld();
+                if constexpr (kGated) {
+                    // this thread's gate column (64 bf16, packed in pairs of tokens), loaded before
+                    // the reduction below so that the loads overlap it
+                    mwait(B_G, ci, leader);
+                    const uint8_t *gt = sm + OFF_G + (row >> 6) * 8192 + (row & 7) * 2;
+                    uint32_t gp[C / 2];
 #pragma unroll
-                for (int p = 0; p < 2; ++p)
+                    for (int i = 0; i < C / 2; ++i)
+                        gp[i] = uint32_t(*reinterpret_cast<const unsigned short *>(gt + sw(2 * i, ch))) |
+                                (uint32_t(*reinterpret_cast<const unsigned short *>(gt + sw(2 * i + 1, ch))) << 16);
+                    // sum over the 128 value channels (one per thread) of o^2 for each of the 64
+                    // tokens: a transposed butterfly leaves lane l holding tokens 2l and 2l + 1 of
+                    // its warp's 32 channels; the four warps' partial sums meet in shared memory
+                    float sq[C];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        *reinterpret_cast<__nv_bfloat16 *>(stage + sw(32 * p + e, ch)) =
-                            __float2bfloat16_rn(__uint_as_float(vo[p][e]));
+                    for (int p = 0; p < 2; ++p)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) sq[32 * p + e] = __uint_as_float(vo[p][e]) * __uint_as_float(vo[p][e]);
+#pragma unroll
+                    for (int m = 16; m >= 1; m >>= 1) {  // 4m partial sums -> 2m
+                        const bool hi = (lane & m) != 0;
+#pragma unroll
+                        for (int i = 0; i < 2 * m; ++i) {
+                            const float send = hi ? sq[i] : sq[2 * m + i];
+                            const float keep = hi ? sq[2 * m + i] : sq[i];
+                            sq[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+                        }
+                    }
+                    float *red = reinterpret_cast<float *>(sm + OFF_RED);
+                    red[warp * 64 + 2 * lane] = sq[0];
+                    red[warp * 64 + 2 * lane + 1] = sq[1];
+                    ptx::named_barrier(BAR_S, NS);
+                    if (tid < C)
+                        red[256 + tid] = rsqrtf((red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid]) * (1.f / D) + a.eps);
+                    ptx::named_barrier(BAR_S, NS);
+#pragma unroll
+                    for (int p = 0; p < 2; ++p)
+#pragma unroll
+                        for (int e4 = 0; e4 < 8; ++e4) {
+                            const float4 rs = *reinterpret_cast<const float4 *>(red + 256 + 32 * p + 4 * e4);
+                            const float rsv[4] = {rs.x, rs.y, rs.z, rs.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int r = 32 * p + 4 * e4 + u;
+                                const float gv = (r & 1) ? bf16_hi(gp[r >> 1]) : bf16_lo(gp[r >> 1]);
+                                const float sg = fmaf(0.5f, ptx::tanh_approx(0.5f * gv), 0.5f);  // sigmoid
+                                *reinterpret_cast<__nv_bfloat16 *>(stage + sw(r, ch)) =
+                                    __float2bfloat16_rn(__uint_as_float(vo[p][4 * e4 + u]) * rsv[u] * w_row * sg);
+                            }
+                        }
+                } else {
+#pragma unroll
+                    for (int p = 0; p < 2; ++p)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            *reinterpret_cast<__nv_bfloat16 *>(stage + sw(32 * p + e, ch)) =
+                                __float2bfloat16_rn(__uint_as_float(vo[p][e]));
+                }
             }
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
+            if (kGated && leader && has_next) load_g(s + C);  // the gate tile has been read
             if (L == C) {  // a full chunk: two TMA tile stores
                 if (leader) {
                     ptx::tma_store_3d(&maps.o, sm + OFF_Y, 0, h, s);
@@ -810,6 +884,16 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <bool kGated>
+cudaError_t launch_tc(const TcMaps &maps, const PrefillArgs &a, cudaStream_t stream) {
+    cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel<kGated>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           int(smem_alloc(kGated)));
+    if (err != cudaSuccess) return err;
+    const unsigned grid = unsigned(a.num_seqs) * unsigned(a.H);
+    prefill_tc_kernel<kGated><<<grid, NT, smem_alloc(kGated), stream>>>(maps, a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 bool prefill_tc_supported(const PrefillArgs &a) {
@@ -825,12 +909,10 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
         !make_map(&maps.la, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.H, a.total_tokens) ||
         !make_map(&maps.o, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens))
         return cudaErrorInvalidValue;
-    cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           int(SMEM_ALLOC));
-    if (err != cudaSuccess) return err;
-    const unsigned grid = unsigned(a.num_seqs) * unsigned(a.H);
-    prefill_tc_kernel<<<grid, NT, SMEM_ALLOC, stream>>>(maps, a);
-    return cudaGetLastError();
+    if (a.gate == nullptr) return launch_tc<false>(maps, a, stream);
+    if (!make_map(&maps.g, a.gate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens))
+        return cudaErrorInvalidValue;
+    return launch_tc<true>(maps, a, stream);
 }
 
 }  // namespace kda

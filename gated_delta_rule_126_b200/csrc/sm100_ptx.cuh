@@ -103,6 +103,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// tanh(x) by the special-function unit (PTX tanh.approx).
+__device__ __forceinline__ float tanh_approx(float x) {
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---------------------------------------------------------------- TMA (tile mode, one CTA)
 __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, uint64_t *bar, int c0, int c1,
                                             int c2) {

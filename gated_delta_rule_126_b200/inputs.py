@@ -143,6 +143,18 @@ def prefill_inputs(seqlens, H, dk, dv, dtype="bf16", s0_std=0.0, seed=0,
                 cu_seqlens_host=cu_host)
 
 
+def gate_inputs(T, H, dv, dtype="bf16", seed=0, device="cpu"):
+    """Synthetic inputs of the output epilogue: the gate pre-activation [T,H,dv]
+    (dtype, ~ N(0, 1)) and the RMSNorm weight [dv] (float32, ~ 1 + 0.1 N(0, 1)).
+    Trained projections do not exist here; these stand in for them."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    f32 = dict(dtype=torch.float32, device=device, generator=gen)
+    gate = torch.randn(T, H, dv, **f32).to(torch_dtype(dtype))
+    weight = 1.0 + 0.1 * torch.randn(dv, **f32)
+    return gate, weight
+
+
 def decode_inputs(batch, H, dk, dv, steps, dtype="bf16", s0_std=S0_STD, seed=0,
                   device="cpu"):
     """Inputs for ``steps`` consecutive one-token decode steps of ``batch`` sequences.

@@ -119,6 +119,39 @@ KDA_API kda_status_t kda_prefill(const void *q, const void *k, const void *v, kd
                          kda_stream_t stream);
 
 /*
+ * kda_prefill_gated -- kda_prefill with the KDA layer's output epilogue applied to o.
+ *
+ * The wiki page "Kimi Linear 高效注意力架构", section "模型架构", lists a sigmoid
+ * output gate and an RMSNorm as the end of the KDA layer, without a formula.  This
+ * call writes, for every token t and head h (the plainest reading of that line),
+ *
+ *   y[t,h,:] = o[t,h,:] / sqrt(mean_j o[t,h,j]^2 + eps) * norm_weight * sigmoid(gate[t,h,:])
+ *
+ * where o is what kda_prefill would write, the mean runs over the d_v value channels
+ * of one head, and norm_weight is shared by the heads.  On the tensor-core path
+ * (bf16, d_k = d_v = 128, chunk = 64) the epilogue is fused into the output store:
+ * o never reaches memory.  With float32 inputs (any shape kda_prefill takes) the
+ * prefill writes o into y and a second kernel applies the epilogue in place.  Other
+ * bf16 shapes return KDA_ERR_UNSUPPORTED (o would be rounded to bf16 twice).
+ *
+ *   gate         [T_total, H, d_v], dtype qkv_dtype: the gate's pre-activation
+ *                (caller-owned, read only; 16-byte aligned)
+ *   norm_weight  [d_v] float32 RMSNorm weight (read only)
+ *   eps          > 0 and finite, added to the mean square inside the root
+ *   y            [T_total, H, d_v] output, dtype qkv_dtype
+ * Every other argument, the workspace rule, S_final and the error behaviour are
+ * kda_prefill's; a bad eps or a NULL gate / norm_weight (with T_total > 0) returns
+ * KDA_ERR_INVALID_ARG.
+ */
+KDA_API kda_status_t kda_prefill_gated(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                               const float *log_alpha, const float *beta, const float *S0,
+                               const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                               int num_seqs, int H, int d_k, int d_v, int chunk,
+                               const void *gate, const float *norm_weight, float eps,
+                               void *y, float *S_final, void *workspace, size_t workspace_bytes,
+                               kda_stream_t stream);
+
+/*
  * kda_decode_step -- one recurrent decode step for B independent sequences.
  *
  * For every (b, h): S <- (I - beta k k^T) Diag(alpha) S + beta k v^T in place,

@@ -29,7 +29,7 @@ def declared_symbols():
 
 def test_header_declares_the_abi():
     assert declared_symbols() == sorted([
-        "kda_decode_step", "kda_decode_tokens", "kda_prefill", "kda_prefill_noalloc",
+        "kda_decode_step", "kda_decode_tokens", "kda_prefill", "kda_prefill_gated", "kda_prefill_noalloc",
         "kda_prefill_workspace_size", "kda_status_string", "kda_version", "kda_workspace_status"])
 
 
@@ -88,6 +88,29 @@ def test_prefill_rejects_bad_arguments(lib):
     assert _prefill(lib, [0, 4], 1, ws=ctypes.c_void_p((1 << 20) + 64)) == WORKSPACE
 
 
+def _gated(lib, cu_host, N, H=2, dk=128, dv=128, chunk=64, dtype=1, gate=FAKE, w=FAKE, eps=1e-6,
+           ws=FAKE):
+    arr = (ctypes.c_int32 * len(cu_host))(*cu_host)
+    return lib.kda_prefill_gated(FAKE, FAKE, FAKE, dtype, FAKE, FAKE, None, FAKE, arr, N, H, dk, dv,
+                                 chunk, gate, w, eps, FAKE, FAKE, ws, 1 << 20, None)
+
+
+def test_prefill_gated_rejects_bad_arguments(lib):
+    assert _gated(lib, [0, 4], 1, H=0) == INVALID                  # kda_prefill's checks come first
+    assert _gated(lib, [0, 4], 1, chunk=48) == UNSUPPORTED
+    assert _gated(lib, [0, 4], 1, ws=None) == WORKSPACE
+    assert _gated(lib, [0, 4], 1, eps=0.0) == INVALID
+    assert _gated(lib, [0, 4], 1, eps=-1.0) == INVALID
+    assert _gated(lib, [0, 4], 1, eps=float("inf")) == INVALID
+    assert _gated(lib, [0, 4], 1, eps=float("nan")) == INVALID
+    assert _gated(lib, [0, 4], 1, gate=None) == INVALID
+    assert _gated(lib, [0, 4], 1, w=None) == INVALID
+    assert _gated(lib, [0, 4], 1, gate=ctypes.c_void_p((1 << 20) + 4)) == INVALID  # misaligned
+    assert _gated(lib, [0, 4], 1, dk=64, dv=64) == UNSUPPORTED    # bf16 off the fused path
+    assert _gated(lib, [0, 4], 1, chunk=32) == UNSUPPORTED
+    assert _gated(lib, [0], 0) == 0                                 # nothing to do
+
+
 def test_decode_rejects_bad_arguments(lib):
     f = lib.kda_decode_step
     assert f(FAKE, FAKE, FAKE, 1, FAKE, FAKE, FAKE, -1, 2, 128, 128, FAKE, None) == INVALID
@@ -131,3 +154,5 @@ def test_binding_raises_without_library(tmp_path):
 def test_valid_call_without_gpu_reports_cuda_error(lib):
     # arguments pass the host checks, then the first CUDA call fails: KDA_ERR_CUDA, no crash
     assert _prefill(lib, [0, 4], 1) == 4
+    assert _gated(lib, [0, 4], 1) == 4
+    assert _gated(lib, [0, 4], 1, dtype=0, dk=16, dv=16, chunk=16) == 4
