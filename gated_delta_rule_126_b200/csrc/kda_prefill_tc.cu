@@ -90,6 +90,9 @@ constexpr uint32_t OFF_ISS = OFF_CNT + 32;              // phases issued / waite
 constexpr uint32_t OFF_WT = OFF_ISS + 4 * NBAR;
 constexpr uint32_t OFF_MISC = OFF_WT + 4 * NBAR;        // tmem base, abort flag
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
+// Running-sum totals of the 4 token blocks (2 KB): over the output tile, which is idle
+// between the wait for its last TMA store (top of a chunk) and the next E4.
+constexpr uint32_t OFF_PART = OFF_Y;
 // The gated output epilogue adds the gate tile (bf16, two 64 x 64 boxes) and the
 // per-token reduction of o^2 (4 x 64 partial sums, then 64 reciprocal RMS values).
 constexpr uint32_t OFF_G = (SMEM_USED + 1023) / 1024 * 1024;
@@ -277,39 +280,61 @@ __global__ void __launch_bounds__(NT, 1)
         }
         // ---- P1 of chunk cj: g = running sum of log alpha per channel, in base 2 (g log2 e)
         // in place over the log alpha tile, and the chunk's vectors (buffer cj & 1): g_m
-        // (base 2), e^{g_m},
-        // e^{g_L - g_m}, the factors of the pass over R and beta.  One channel per
-        // thread; beta is read from global memory one chunk ahead (a register).
+        // (base 2), e^{g_m}, e^{g_L - g_m}, the factors of the pass over R and beta.  Warp w
+        // sums tokens 16w .. 16w + 15 for four channels a lane (float4 rows); the warps'
+        // totals meet in shared memory.  beta is read from global memory one chunk ahead.
         auto load_beta = [&](int cj) {
             const int s = bos + cj * C;
             return (tid < C && cj < nchunks && s + tid < eos) ? a.beta[size_t(s + tid) * H + h] : 0.f;
         };
         float beta_reg = load_beta(0);
-        float ecm_prev = 1.f;  // e^{g_L - g_m} of the previous chunk, channel tid
         auto scan = [&](int cj) {
             const int L = min(C, eos - (bos + cj * C));
             const int par = cj & 1;
-            const int c = tid, lch = (c & 31) >> 2;
-            uint8_t *col = sm + OFF_LA + (c >> 5) * 8192 + (c & 3) * 4;
+            const int wq = warp, c0 = 4 * lane, lch = lane & 7;
+            uint8_t *tile = sm + OFF_LA + (lane >> 3) * 8192;  // box holding channels c0 .. c0 + 3
             const int rm = (L - 1) >> 1;
             mwait(B_LA, cj, leader);
-            float x[C];
+            float4 x[16];
 #pragma unroll
-            for (int i = 0; i < C; ++i) x[i] = (i < L) ? *reinterpret_cast<const float *>(col + sw(i, lch)) : 0.f;
-            x[0] *= kLog2e;
+            for (int i = 0; i < 16; ++i) {
+                const int r = 16 * wq + i;
+                x[i] = r < L ? *reinterpret_cast<const float4 *>(tile + sw(r, lch)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            x[0] = make_float4(x[0].x * kLog2e, x[0].y * kLog2e, x[0].z * kLog2e, x[0].w * kLog2e);
 #pragma unroll
-            for (int i = 1; i < C; ++i) x[i] = fmaf(x[i], kLog2e, x[i - 1]);
-            float gmid = 0.f;
+            for (int i = 1; i < 16; ++i)
+                x[i] = make_float4(fmaf(x[i].x, kLog2e, x[i - 1].x), fmaf(x[i].y, kLog2e, x[i - 1].y),
+                                   fmaf(x[i].z, kLog2e, x[i - 1].z), fmaf(x[i].w, kLog2e, x[i - 1].w));
+            float4 *part = reinterpret_cast<float4 *>(sm + OFF_PART);
+            part[wq * 32 + lane] = x[15];
+            ptx::named_barrier(BAR_S, NS);
+            float4 off = make_float4(0.f, 0.f, 0.f, 0.f), tot = off;
 #pragma unroll
-            for (int i = 0; i < C; ++i) gmid = (i == rm) ? x[i] : gmid;
+            for (int w = 0; w < 4; ++w) {
+                const float4 p = part[w * 32 + lane];
+                if (w < wq) off = make_float4(off.x + p.x, off.y + p.y, off.z + p.z, off.w + p.w);
+                tot = make_float4(tot.x + p.x, tot.y + p.y, tot.z + p.z, tot.w + p.w);
+            }
 #pragma unroll
-            for (int i = 0; i < C; ++i) *reinterpret_cast<float *>(col + sw(i, lch)) = x[i];
-            const float e = exp2f(gmid), ecm = exp2f(x[C - 1] - gmid);  // rows >= L add 0
-            vec(par, VEC_GM)[c] = gmid;
-            vec(par, VEC_EGM)[c] = e;
-            vec(par, VEC_ECM)[c] = ecm;
-            vec(par, VEC_FAC)[c] = ecm_prev * e;
-            ecm_prev = ecm;
+            for (int i = 0; i < 16; ++i) {
+                x[i] = make_float4(x[i].x + off.x, x[i].y + off.y, x[i].z + off.z, x[i].w + off.w);
+                *reinterpret_cast<float4 *>(tile + sw(16 * wq + i, lch)) = x[i];
+            }
+            if (wq == (rm >> 4)) {  // the warp holding token rm writes the chunk's vectors
+                const float4 gm = *reinterpret_cast<const float4 *>(tile + sw(rm, lch));  // stored above by this thread
+                const float4 e = make_float4(exp2f(gm.x), exp2f(gm.y), exp2f(gm.z), exp2f(gm.w));
+                // g_L = tot: rows >= L add 0
+                const float4 ecm = make_float4(exp2f(tot.x - gm.x), exp2f(tot.y - gm.y), exp2f(tot.z - gm.z),
+                                               exp2f(tot.w - gm.w));
+                const float4 prev = cj > 0 ? *reinterpret_cast<const float4 *>(vec(par ^ 1, VEC_ECM) + c0)
+                                           : make_float4(1.f, 1.f, 1.f, 1.f);
+                *reinterpret_cast<float4 *>(vec(par, VEC_GM) + c0) = gm;
+                *reinterpret_cast<float4 *>(vec(par, VEC_EGM) + c0) = e;
+                *reinterpret_cast<float4 *>(vec(par, VEC_ECM) + c0) = ecm;
+                *reinterpret_cast<float4 *>(vec(par, VEC_FAC) + c0) =
+                    make_float4(prev.x * e.x, prev.y * e.y, prev.z * e.z, prev.w * e.w);
+            }
             if (tid < C) vec(par, VEC_BETA)[tid] = beta_reg;
             beta_reg = load_beta(cj + 1);
             ptx::fence_proxy_async_smem();  // the next log alpha tile overwrites g by TMA
@@ -521,7 +546,11 @@ __global__ void __launch_bounds__(NT, 1)
                     ptx::named_barrier(BAR_S, NS);
                     if (tid < C)
                         red[256 + tid] = rsqrtf((red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid]) * (1.f / D) + a.eps);
+                    // o again from TMEM (held there until the next M2): fewer registers live across the reduction
+                    ptx::tmem_ld32(tl + TZ + 64, vo[0]);
+                    ptx::tmem_ld32(tl + TZ + 96, vo[1]);
                     ptx::named_barrier(BAR_S, NS);
+                    ptx::tmem_wait_ld();
 #pragma unroll
                     for (int p = 0; p < 2; ++p)
 #pragma unroll
