@@ -264,7 +264,7 @@ def run_reference(args):
 
 def run_ours(args):
     from gated_delta_rule_126_b200 import (kda_decode_step, kda_decode_tokens, kda_prefill,
-                                           kda_prefill_gated, prefill_workspace_size)
+                                           kda_prefill_gated, kda_prologue, prefill_workspace_size)
     world, rank, local = dist_setup("nccl")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -385,6 +385,34 @@ def run_ours(args):
                               "frac": g_gbs / hbm_peak, "alg_bytes_per_launch": g_bytes}}
         del gate, g_w, y
 
+    # the layer's input prologue (short conv + Swish + L2Norm, gates) that makes this
+    # workload's prefill inputs from its projections: one HBM-bound launch
+    prologue = None
+    if not args.no_prologue and w.dk % 4 == 0 and w.dv % 4 == 0:
+        pin = inputs.prologue_inputs(w.seqlens, w.H, w.dk, w.dv, w.dtype, width=4,
+                                     seed=w.seed + 11 + 1000 * rank, device=dev)
+        pout = {n: torch.empty_like(inp[n]) for n in ("q", "k", "v", "log_alpha", "beta")}
+
+        def pstep():
+            kda_prologue(pin["q_pre"], pin["k_pre"], pin["v_pre"], pin["conv_q"], pin["conv_k"],
+                         pin["conv_v"], pin["a_gate"], pin["rate"], pin["b_gate"], pin["cu_seqlens"],
+                         cu_seqlens_host=cu_host, out=pout, stream=stream)
+
+        for _ in range(args.warmup):
+            pstep()
+        barrier(world)
+        p_el = max_over_ranks(time_region(pstep, args.steps, stream), world)
+        p_t = p_el / args.steps
+        # bytes per head-token: q/k/v projections in and q/k/v out (dtype), a_gate in and
+        # log alpha out (f32), b_gate in and beta out (f32)
+        p_bytes = head_tokens * 2 * ((2 * w.dk + w.dv) * qkv_bytes + 4 * w.dk + 4)
+        p_gbs = p_bytes / p_t / 1e9
+        prologue = {"value": weak_scaling_value(T, args.steps, p_el, world), "unit": UNIT,
+                    "ms_per_step": p_t * 1e3, "conv_width": 4, "gpu_launches_per_step": 1,
+                    "roofline": {"bound": "hbm", "achieved": p_gbs, "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": p_gbs / hbm_peak, "alg_bytes_per_launch": p_bytes}}
+        del pin, pout
+
     # decode: 256 sequences x 32 heads, 64 consecutive one-token steps
     decode = None
     if not args.no_decode:
@@ -464,7 +492,7 @@ def run_ours(args):
                     "l2": "inputs larger than L2 (no flush)"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": 2 * args.steps, "clocks": clk.summary(), "decode": decode,
-                "gated_epilogue": gated}
+                "gated_epilogue": gated, "prologue": prologue}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -484,6 +512,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-gated", action="store_true")
+    ap.add_argument("--no-prologue", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps

@@ -8,6 +8,8 @@ binding over that ABI, with the same names:
 * ``kda_prefill``     -- chunked prefill over packed variable-length sequences;
 * ``kda_prefill_gated`` -- the same with the layer's output epilogue (sigmoid gate
   and RMSNorm) applied to o;
+* ``kda_prologue``    -- the layer's input prologue (short conv, Swish, L2Norm, gates)
+  that makes the prefill's inputs from the projections;
 * ``kda_decode_step`` -- one recurrent decode step for a batch of sequences;
 * ``kda_decode_tokens`` -- n tokens per sequence with states in a slot pool;
 * ``prefill_workspace_size``, ``workspace_status``, ``KdaError``.
@@ -16,7 +18,8 @@ binding over that ABI, with the same names:
 does not load the CUDA library; the first call does, and raises if it is missing.
 """
 from ._binding import (KdaError, kda_decode_step, kda_decode_tokens, kda_prefill,
-                       kda_prefill_gated, load, prefill_workspace_size, workspace_status)
+                       kda_prefill_gated, kda_prologue, load, prefill_workspace_size,
+                       workspace_status)
 
 __all__ = ["KdaError", "kda_decode_step", "kda_decode_tokens", "kda_prefill", "kda_prefill_gated",
-           "load", "prefill_workspace_size", "workspace_status"]
+           "kda_prologue", "load", "prefill_workspace_size", "workspace_status"]

@@ -48,6 +48,9 @@ def _declare(lib):
     lib.kda_prefill_gated.restype = i32
     lib.kda_prefill_gated.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                       vp, vp, c.c_float, vp, vp, vp, sz, vp]
+    lib.kda_prologue.restype = i32
+    lib.kda_prologue.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32,
+                                 c.c_float, vp, vp, vp, vp, vp, vp]
     lib.kda_decode_step.restype = i32
     lib.kda_decode_step.argtypes = [vp, vp, vp, i32, vp, vp, vp, i32, i32, i32, i32, vp, vp]
     lib.kda_decode_tokens.restype = i32
@@ -205,6 +208,56 @@ def kda_prefill_gated(q, k, v, log_alpha, beta, cu_seqlens, gate, norm_weight, e
                                    _stream_handle(stream))
     _check(st, "kda_prefill_gated")
     return y, S_final
+
+
+def kda_prologue(q_pre, k_pre, v_pre, conv_q, conv_k, conv_v, a_gate, rate, b_gate, cu_seqlens,
+                 cu_seqlens_host=None, l2_eps=1e-6, out=None, stream=None):
+    """The layer's input prologue (see ``kda_prologue`` in kda.h).
+
+    q_pre, k_pre [T,H,d_k], v_pre [T,H,d_v] (float32 or bfloat16); conv_* [H,d,W] float32;
+    a_gate [T,H,d_k], rate [H], b_gate [T,H] float32.  Returns a dict with q, k, v,
+    log_alpha, beta in kda_prefill's layouts (``out`` may supply them).
+    """
+    lib = load()
+    dev = q_pre.device
+    dt = q_pre.dtype
+    if dt not in DTYPE_CODE:
+        raise ValueError("projection dtype must be float32 or bfloat16")
+    _need(q_pre, "q_pre", dt)
+    T, H, dk = q_pre.shape
+    _need(k_pre, "k_pre", dt, dev)
+    _need(v_pre, "v_pre", dt, dev)
+    dv = v_pre.shape[2]
+    for name, t in (("conv_q", conv_q), ("conv_k", conv_k), ("conv_v", conv_v), ("a_gate", a_gate),
+                    ("rate", rate), ("b_gate", b_gate)):
+        _need(t, name, torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    W = conv_q.shape[-1]
+    if conv_k.shape[-1] != W or conv_v.shape[-1] != W:
+        raise ValueError("the three convolutions must have the same width")
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu()
+    cu_h = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
+    N = cu_h.numel() - 1
+    out = dict(out or {})
+    out.setdefault("q", torch.empty(T, H, dk, dtype=dt, device=dev))
+    out.setdefault("k", torch.empty(T, H, dk, dtype=dt, device=dev))
+    out.setdefault("v", torch.empty(T, H, dv, dtype=dt, device=dev))
+    out.setdefault("log_alpha", torch.empty(T, H, dk, dtype=torch.float32, device=dev))
+    out.setdefault("beta", torch.empty(T, H, dtype=torch.float32, device=dev))
+    for name in ("q", "k", "v"):
+        _need(out[name], name, dt, dev)
+    _need(out["log_alpha"], "log_alpha", torch.float32, dev)
+    _need(out["beta"], "beta", torch.float32, dev)
+    with torch.cuda.device(dev):
+        st = lib.kda_prologue(_ptr(q_pre), _ptr(k_pre), _ptr(v_pre), DTYPE_CODE[dt], _ptr(conv_q),
+                              _ptr(conv_k), _ptr(conv_v), int(W), _ptr(a_gate), _ptr(rate),
+                              _ptr(b_gate), _ptr(cu_seqlens), ctypes.c_void_p(cu_h.data_ptr()), N,
+                              H, dk, dv, float(l2_eps), _ptr(out["q"]), _ptr(out["k"]),
+                              _ptr(out["v"]), _ptr(out["log_alpha"]), _ptr(out["beta"]),
+                              _stream_handle(stream))
+    _check(st, "kda_prologue")
+    return out
 
 
 def kda_decode_step(q, k, v, log_alpha, beta, S, o=None, stream=None):

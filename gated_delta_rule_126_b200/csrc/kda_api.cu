@@ -142,6 +142,38 @@ kda_status_t kda_prefill_gated(const void *q, const void *k, const void *v, kda_
     return from_cuda(kda::launch_gated_rmsnorm(a, st));
 }
 
+kda_status_t kda_prologue(const void *q_pre, const void *k_pre, const void *v_pre, kda_dtype_t dtype,
+                          const float *conv_q, const float *conv_k, const float *conv_v, int conv_width,
+                          const float *a_gate, const float *rate, const float *b_gate,
+                          const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int num_seqs, int H,
+                          int d_k, int d_v, float l2_eps, void *q, void *k, void *v, float *log_alpha,
+                          float *beta, kda_stream_t stream) {
+    if (num_seqs < 0 || H < 1 || d_k < 1 || d_v < 1 || !dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
+    if (!(l2_eps >= 0.f) || !std::isfinite(l2_eps)) return KDA_ERR_INVALID_ARG;
+    if (conv_width < 1 || conv_width > 4) return KDA_ERR_UNSUPPORTED;
+    if (d_k > 128 || d_v > 128 || (d_k % 4) != 0 || (d_v % 4) != 0) return KDA_ERR_UNSUPPORTED;
+    if (!cu_seqlens_host || !cu_seqlens_dev || cu_seqlens_host[0] != 0) return KDA_ERR_INVALID_ARG;
+    for (int n = 0; n < num_seqs; ++n)
+        if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return KDA_ERR_INVALID_ARG;
+    const int64_t T = cu_seqlens_host[num_seqs];
+    if (T == 0) return KDA_OK;
+    const void *ptrs[] = {q_pre, k_pre, v_pre, conv_q, conv_k, conv_v, a_gate, rate, b_gate, q, k, v,
+                          log_alpha, beta};
+    for (const void *p : ptrs)
+        if (!p) return KDA_ERR_INVALID_ARG;
+    const void *rows[] = {q_pre, k_pre, v_pre, a_gate, q, k, v, log_alpha};
+    for (const void *p : rows)
+        if (!aligned16(p)) return KDA_ERR_INVALID_ARG;
+    kda::PrologueArgs a;
+    a.q_pre = q_pre; a.k_pre = k_pre; a.v_pre = v_pre; a.dtype = dtype;
+    a.conv_q = conv_q; a.conv_k = conv_k; a.conv_v = conv_v; a.W = conv_width;
+    a.a = a_gate; a.rate = rate; a.b = b_gate;
+    a.cu_seqlens = cu_seqlens_dev;
+    a.num_seqs = num_seqs; a.H = H; a.dk = d_k; a.dv = d_v; a.total_tokens = T; a.l2_eps = l2_eps;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    return from_cuda(kda::launch_prologue(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 kda_status_t kda_decode_step(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
                              const float *log_alpha, const float *beta, float *S, int B, int H,
                              int d_k, int d_v, void *o, kda_stream_t stream) {

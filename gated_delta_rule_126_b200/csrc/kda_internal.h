@@ -51,6 +51,20 @@ struct PrefillArgs {
     float eps = 0.f;
 };
 
+struct PrologueArgs {
+    const void *q_pre, *k_pre, *v_pre;
+    kda_dtype_t dtype;
+    const float *conv_q, *conv_k, *conv_v;  // [H, d, W]
+    int W;
+    const float *a, *rate, *b;              // [T, H, d_k], [H], [T, H]
+    const int32_t *cu_seqlens;              // device, num_seqs + 1
+    int num_seqs, H, dk, dv;
+    int64_t total_tokens;
+    float l2_eps;
+    void *q, *k, *v;
+    float *log_alpha, *beta;
+};
+
 struct DecodeArgs {
     const void *q, *k, *v;
     kda_dtype_t dtype;
@@ -75,6 +89,7 @@ cudaError_t launch_decode_tokens(const DecodeTokensArgs &a, cudaStream_t stream)
 cudaError_t launch_prefill_simt(const PrefillArgs &a, cudaStream_t stream);
 bool prefill_tc_supported(const PrefillArgs &a);
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream);  // fuses the epilogue when a.gate is set
+cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t stream);
 // The output epilogue in place over a.o (after a prefill that does not fuse it).
 cudaError_t launch_gated_rmsnorm(const PrefillArgs &a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);

@@ -155,6 +155,34 @@ def gate_inputs(T, H, dv, dtype="bf16", seed=0, device="cpu"):
     return gate, weight
 
 
+def prologue_inputs(seqlens, H, dk, dv, dtype="bf16", width=4, seed=0, device="cpu"):
+    """Synthetic inputs of the input prologue, packed like ``prefill_inputs``.
+
+    q_pre, k_pre [T,H,dk], v_pre [T,H,dv] ~ N(0, 1) (dtype); conv_q/conv_k [H,dk,W] and
+    conv_v [H,dv,W] ~ N(0, 1/W) float32; a_gate [T,H,dk] ~ N(0, 1); rate = 0.1 per head;
+    b_gate [T,H] ~ N(0, 1).  With these, log_alpha = -0.1 softplus(N(0, 1)) and
+    beta = sigmoid(N(0, 1)), the gate recipe of ``prefill_inputs``.  Trained weights do
+    not exist here; these stand in for them.
+    """
+    seqlens = [int(x) for x in seqlens]
+    T = sum(seqlens)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    f32 = dict(dtype=torch.float32, device=device, generator=gen)
+    dt = torch_dtype(dtype)
+    cu_host = [0]
+    for L in seqlens:
+        cu_host.append(cu_host[-1] + L)
+    return dict(q_pre=torch.randn(T, H, dk, **f32).to(dt), k_pre=torch.randn(T, H, dk, **f32).to(dt),
+                v_pre=torch.randn(T, H, dv, **f32).to(dt),
+                conv_q=torch.randn(H, dk, width, **f32) / width ** 0.5,
+                conv_k=torch.randn(H, dk, width, **f32) / width ** 0.5,
+                conv_v=torch.randn(H, dv, width, **f32) / width ** 0.5,
+                a_gate=torch.randn(T, H, dk, **f32), rate=torch.full((H,), 0.1, dtype=torch.float32, device=device),
+                b_gate=torch.randn(T, H, **f32),
+                cu_seqlens=torch.tensor(cu_host, dtype=torch.int32, device=device), cu_seqlens_host=cu_host)
+
+
 def decode_inputs(batch, H, dk, dv, steps, dtype="bf16", s0_std=S0_STD, seed=0,
                   device="cpu"):
     """Inputs for ``steps`` consecutive one-token decode steps of ``batch`` sequences.

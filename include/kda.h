@@ -119,6 +119,37 @@ KDA_API kda_status_t kda_prefill(const void *q, const void *k, const void *v, kd
                          kda_stream_t stream);
 
 /*
+ * kda_prologue -- the KDA layer's input prologue: it makes kda_prefill's inputs from
+ * the layer's projections.
+ *
+ * The wiki page "Kimi Linear 高效注意力架构", section "模型架构", lists ShortConv +
+ * Swish + L2Norm (q/k) and a low-rank channel-wise decay gate in the KDA layer,
+ * without formulas.  This call computes, per sequence of cu_seqlens, head h and
+ * channel c (the plainest reading of that line):
+ *
+ *   conv(x)[t] = sum_{w < conv_width} conv[h][c][w] * x[t - w]   (x = 0 before the
+ *                sequence's first token: the convolution never crosses a sequence)
+ *   q = l2norm(swish(conv_q(q_pre))), k = l2norm(swish(conv_k(k_pre))), v = swish(conv_v(v_pre))
+ *   swish(z) = z * sigmoid(z),  l2norm(z) = z / sqrt(sum_c z_c^2 + l2_eps) over the head's channels
+ *   log_alpha = -rate[h] * softplus(a_gate),  beta = sigmoid(b_gate)
+ *
+ *   q_pre, k_pre      [T_total, H, d_k] dtype     v_pre   [T_total, H, d_v] dtype
+ *   conv_q, conv_k    [H, d_k, conv_width] f32    conv_v  [H, d_v, conv_width] f32
+ *   a_gate            [T_total, H, d_k] f32 (the low-rank gate's output)
+ *   rate              [H] f32 (> 0 for log_alpha <= 0)     b_gate [T_total, H] f32
+ *   q, k, v, log_alpha, beta   outputs in kda_prefill's layouts (q/k/v in dtype)
+ * Row pointers (q_pre, k_pre, v_pre, a_gate, q, k, v, log_alpha) are 16-byte aligned.
+ * Supported: 1 <= conv_width <= 4, d_k and d_v multiples of 4 up to 128; otherwise
+ * KDA_ERR_UNSUPPORTED.  l2_eps >= 0 and finite.  HBM-bound; one launch.
+ */
+KDA_API kda_status_t kda_prologue(const void *q_pre, const void *k_pre, const void *v_pre, kda_dtype_t dtype,
+                          const float *conv_q, const float *conv_k, const float *conv_v, int conv_width,
+                          const float *a_gate, const float *rate, const float *b_gate,
+                          const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host, int num_seqs, int H,
+                          int d_k, int d_v, float l2_eps, void *q, void *k, void *v, float *log_alpha,
+                          float *beta, kda_stream_t stream);
+
+/*
  * kda_prefill_gated -- kda_prefill with the KDA layer's output epilogue applied to o.
  *
  * The wiki page "Kimi Linear 高效注意力架构", section "模型架构", lists a sigmoid

@@ -29,7 +29,7 @@ def declared_symbols():
 
 def test_header_declares_the_abi():
     assert declared_symbols() == sorted([
-        "kda_decode_step", "kda_decode_tokens", "kda_prefill", "kda_prefill_gated", "kda_prefill_noalloc",
+        "kda_decode_step", "kda_decode_tokens", "kda_prefill", "kda_prefill_gated", "kda_prefill_noalloc", "kda_prologue",
         "kda_prefill_workspace_size", "kda_status_string", "kda_version", "kda_workspace_status"])
 
 
@@ -111,6 +111,28 @@ def test_prefill_gated_rejects_bad_arguments(lib):
     assert _gated(lib, [0], 0) == 0                                 # nothing to do
 
 
+def _prologue(lib, cu_host, N, H=2, dk=128, dv=128, W=4, dtype=1, ptr=FAKE, eps=1e-6, q=FAKE):
+    arr = (ctypes.c_int32 * len(cu_host))(*cu_host)
+    return lib.kda_prologue(ptr, ptr, ptr, dtype, FAKE, FAKE, FAKE, W, FAKE, FAKE, FAKE, FAKE, arr, N, H, dk,
+                            dv, eps, q, FAKE, FAKE, FAKE, FAKE, None)
+
+
+def test_prologue_rejects_bad_arguments(lib):
+    assert _prologue(lib, [0, 4], 1, H=0) == INVALID
+    assert _prologue(lib, [0, 4], 1, dtype=5) == INVALID
+    assert _prologue(lib, [0, 4], 1, eps=-1.0) == INVALID
+    assert _prologue(lib, [0, 4], 1, eps=float("nan")) == INVALID
+    assert _prologue(lib, [0, 4], 1, W=0) == UNSUPPORTED
+    assert _prologue(lib, [0, 4], 1, W=5) == UNSUPPORTED
+    assert _prologue(lib, [0, 4], 1, dk=130) == UNSUPPORTED
+    assert _prologue(lib, [0, 4], 1, dv=126) == UNSUPPORTED
+    assert _prologue(lib, [1, 4], 1) == INVALID                     # must start at 0
+    assert _prologue(lib, [0, 4, 2], 2) == INVALID                  # decreasing
+    assert _prologue(lib, [0, 4], 1, ptr=None) == INVALID
+    assert _prologue(lib, [0, 4], 1, q=ctypes.c_void_p((1 << 20) + 8)) == INVALID  # misaligned
+    assert _prologue(lib, [0, 0], 1) == 0                           # no tokens
+
+
 def test_decode_rejects_bad_arguments(lib):
     f = lib.kda_decode_step
     assert f(FAKE, FAKE, FAKE, 1, FAKE, FAKE, FAKE, -1, 2, 128, 128, FAKE, None) == INVALID
@@ -156,3 +178,4 @@ def test_valid_call_without_gpu_reports_cuda_error(lib):
     assert _prefill(lib, [0, 4], 1) == 4
     assert _gated(lib, [0, 4], 1) == 4
     assert _gated(lib, [0, 4], 1, dtype=0, dk=16, dv=16, chunk=16) == 4
+    assert _prologue(lib, [0, 4], 1) == 4
