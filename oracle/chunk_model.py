@@ -94,3 +94,74 @@ def prefill(q, k, v, log_alpha, beta, cu_seqlens, S0=None, chunk: int = 64):
                 o[s:e, h] = O
             S_out[n, h] = S
     return o, S_out
+
+
+def chunk_backward_unit(q, k, v, log_alpha, beta, dO, S0, dS_final, chunk: int = 64):
+    """Gradients for one (sequence, head) unit by the chunk form, in fp64.
+
+    The reverse of ``chunk_step`` taken product by product (the derivation is the chain
+    rule through the chunk equations in this module's docstring), with the decay split
+    at the chunk's middle token m as Kt = K e^{g - g_m}, Kb = K e^{g_m - g},
+    Qt = Q e^{g - g_m} (so A = tril(Diag(beta) Kt Kb^T), P = tril_incl(Qt Kb^T)) and
+    Kg = K e^{g}, Qg = Q e^{g}, Kh = K e^{g_L - g}.  q, k, log_alpha [L, d_k]; v, dO
+    [L, d_v]; beta [L]; S0, dS_final [d_k, d_v].  Returns (dq, dk, dv, dlog_alpha, dbeta,
+    dS0).  Pinned to the token adjoint in ``tests/test_backward_pins.py``.
+    """
+    q, k, v, la, b, dO = (np.asarray(x, np.float64) for x in (q, k, v, log_alpha, beta, dO))
+    T, dk = q.shape
+    starts = list(range(0, T, chunk))
+    states = [np.array(S0, np.float64)]
+    for s in starts[:-1] if starts else []:
+        e = min(s + chunk, T)
+        st = chunk_stages(q[s:e], k[s:e], v[s:e], la[s:e], b[s:e])
+        states.append(chunk_step(st, states[-1])[1])
+    dq, dkk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+    dla, db = np.zeros_like(la), np.zeros_like(b)
+    dS = np.array(dS_final, np.float64)
+    for ci in reversed(range(len(starts))):
+        s = starts[ci]
+        e = min(s + chunk, T)
+        L = e - s
+        S = states[ci]
+        K, Q, V, B, dOc = k[s:e], q[s:e], v[s:e], b[s:e], dO[s:e]
+        g = np.cumsum(la[s:e], axis=0)
+        gm = g[(L - 1) // 2]
+        gC = g[-1]
+        Kt, Kb, Qt = K * np.exp(g - gm), K * np.exp(gm - g), Q * np.exp(g - gm)
+        Kg, Qg, Kh = K * np.exp(g), Q * np.exp(g), K * np.exp(gC - g)
+        strict, incl = np.tril(np.ones((L, L)), -1), np.tril(np.ones((L, L)))
+        M = Kt @ Kb.T
+        A = B[:, None] * M * strict
+        X = np.linalg.inv(np.eye(L) + A)
+        Tm = X * B[None, :]
+        Pm = (Qt @ Kb.T) * incl
+        Y = V - Kg @ S
+        U = Tm @ Y
+        # reverse of O = Qg S + Pm U and S_next = Diag(e^{g_C}) S + Kh^T U
+        dU = Kh @ dS + Pm.T @ dOc
+        dKh = U @ dS.T
+        dQg = dOc @ S.T
+        dP = (dOc @ U.T) * incl
+        dQt = dP @ Kb
+        dKb = dP.T @ Qt
+        dT = dU @ Y.T
+        dY = Tm.T @ dU
+        dKg = -dY @ S.T
+        dS_prev = np.exp(gC)[:, None] * dS + Qg.T @ dOc - Kg.T @ dY
+        # T = X Diag(beta), X = (I + A)^{-1}, A = tril(Diag(beta) M)
+        dbeta = np.sum(dT * X, axis=0)
+        dA = -(X.T @ (dT * B[None, :]) @ X.T) * strict
+        dbeta += np.sum(dA * M, axis=1)
+        dM = B[:, None] * dA
+        dKt = dM @ Kb
+        dKb += dM.T @ Kt
+        # back to q, k and the running sums g (g_m is a reference point: its gradient cancels)
+        dq[s:e] = dQt * np.exp(g - gm) + dQg * np.exp(g)
+        dkk[s:e] = dKt * np.exp(g - gm) + dKb * np.exp(gm - g) + dKg * np.exp(g) + dKh * np.exp(gC - g)
+        dg = dKt * Kt - dKb * Kb + dQt * Qt + dKg * Kg + dQg * Qg - dKh * Kh
+        dg[-1] += np.sum(dKh * Kh, axis=0) + np.exp(gC) * np.sum(dS * S, axis=1)
+        dla[s:e] = np.cumsum(dg[::-1], axis=0)[::-1]
+        dv[s:e] = dY
+        db[s:e] = dbeta
+        dS = dS_prev
+    return dq, dkk, dv, dla, db, dS

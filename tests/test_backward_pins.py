@@ -85,3 +85,27 @@ def test_linear_attention_special_case():
     assert np.allclose(g["dq"][:, 0], c["dO"][:, 0] @ S0.T, rtol=1e-12)
     assert np.allclose(g["dS0"][0, 0], c["q"][:, 0].T @ c["dO"][:, 0] + c["dS"][0, 0], rtol=1e-12)
     assert np.array_equal(g["dv"], np.zeros_like(g["dv"]))
+
+
+@pytest.mark.parametrize("T,chunk", [(37, 8), (64, 16), (5, 8), (130, 64)])
+def test_chunk_backward_model_matches_adjoint(T, chunk):
+    """The chunk-form backward (the algorithm the GPU kernel follows) equals the token
+    adjoint to fp64 rounding, with ragged last chunks."""
+    from oracle import chunk_model
+    rng = np.random.default_rng(T)
+    dk, dv = 6, 5
+    q = rng.standard_normal((T, 1, dk))
+    k = rng.standard_normal((T, 1, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((T, 1, dv))
+    la = -0.2 * np.log1p(np.exp(rng.standard_normal((T, 1, dk))))
+    b = 1 / (1 + np.exp(-rng.standard_normal((T, 1))))
+    S0 = rng.standard_normal((1, 1, dk, dv))
+    dO = rng.standard_normal((T, 1, dv))
+    dS = rng.standard_normal((1, 1, dk, dv))
+    g = oracle.backward(q, k, v, la, b, [0, T], dO, S0=S0, dS_final=dS)
+    r = chunk_model.chunk_backward_unit(q[:, 0], k[:, 0], v[:, 0], la[:, 0], b[:, 0], dO[:, 0], S0[0, 0],
+                                        dS[0, 0], chunk=chunk)
+    for name, got in zip(["dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0"], r):
+        ref = g[name][0, 0] if name == "dS0" else g[name][:, 0]
+        assert np.linalg.norm(got - ref) / np.linalg.norm(ref) < 1e-12, name
