@@ -83,6 +83,15 @@ def measured_traffic(kernel, units):
     return rec["dram_bytes"] * units / rec["units"]
 
 
+def prefill_launches(seqlens, H, tc_path):
+    """Kernel launches of one kda_prefill call: the ordering kernel and the prefill; on the
+    tensor-core path a long sequence is split (a sequence of at least 16,384 tokens with
+    2 L 148 > 3 T H), which adds the chain of start states and a second prefill pass."""
+    T = sum(seqlens)
+    split = tc_path and any(L >= 16384 and 2 * L * 148 > 3 * T * H for L in seqlens)
+    return 4 if split else 2
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -491,7 +500,9 @@ def run_ours(args):
                     "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                     "l2": "inputs larger than L2 (no flush)"},
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": 2 * args.steps, "clocks": clk.summary(), "decode": decode,
+                "gpu_launches": prefill_launches(w.seqlens, w.H, w.dtype == "bf16" and w.dk == 128 and w.dv == 128
+                                                 and w.chunk == 64) * args.steps,
+                "clocks": clk.summary(), "decode": decode,
                 "gated_epilogue": gated, "prologue": prologue}
         print(json.dumps(line), flush=True)
     if world > 1:

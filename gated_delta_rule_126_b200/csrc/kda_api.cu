@@ -15,6 +15,11 @@ kda_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_E
 
 bool dtype_ok(kda_dtype_t t) { return t == KDA_DTYPE_F32 || t == KDA_DTYPE_BF16; }
 
+// The shapes the tensor-core prefill takes (it also needs T > 0 and N > 0 at run time).
+bool tc_shape(int d_k, int d_v, int chunk, kda_dtype_t t) {
+    return t == KDA_DTYPE_BF16 && d_k == 128 && d_v == 128 && chunk == 64;
+}
+
 // Shapes every prefill kernel here accepts.
 kda_status_t check_prefill_shape(int num_seqs, int H, int d_k, int d_v, int chunk, kda_dtype_t dt) {
     if (num_seqs < 0 || H < 1 || d_k < 1 || d_v < 1 || !dtype_ok(dt)) return KDA_ERR_INVALID_ARG;
@@ -69,6 +74,82 @@ kda_status_t launch_prefill_prologue(const kda::PrefillArgs &a, cudaStream_t st)
     return KDA_OK;
 }
 
+// Plans the sequence split of the tensor-core prefill (see kda_internal.h) when the
+// workspace has room: sequences with L >= kSplitMinLen whose critical path exceeds 1.5x
+// the even spread of the whole call over the SMs (2 L 148 > 3 T H), longest first.
+// Returns false (no split) otherwise.
+bool plan_split(kda::PrefillArgs &a, const int32_t *cu_host, void *workspace, size_t workspace_bytes) {
+    const kda::WorkspaceLayout wl = kda::workspace_layout(a.num_seqs, a.total_tokens, a.H, true);
+    if (wl.split_offset == 0 || workspace_bytes < wl.total) return false;
+    const int m_max = kda::split_max_seqs(a.total_tokens, a.H);
+    int picked[kda::kMaxSplitSeqs];
+    int m = 0;
+    for (; m < m_max; ++m) {  // the longest qualifying sequences not yet picked
+        int best = -1;
+        int64_t best_len = 0;
+        for (int n = 0; n < a.num_seqs; ++n) {
+            const int64_t len = int64_t(cu_host[n + 1]) - cu_host[n];
+            bool taken = false;
+            for (int i = 0; i < m; ++i) taken |= picked[i] == n;
+            if (taken || len < kda::kSplitMinLen || 2 * len * 148 <= 3 * a.total_tokens * a.H) continue;
+            if (len > best_len) best = n, best_len = len;
+        }
+        if (best < 0) break;
+        picked[m] = best;
+    }
+    if (m == 0) return false;
+    char *base = static_cast<char *>(workspace) + wl.split_offset;
+    a.split.sstart = reinterpret_cast<float *>(base);
+    a.split.lmat = reinterpret_cast<float *>(base + wl.split_array_bytes);
+    a.split.mmat = reinterpret_cast<float *>(base + 2 * wl.split_array_bytes);
+    a.split.num_seqs = m;
+    for (int j = 0; j < m; ++j) a.split.seqs[j] = picked[j];
+    return true;
+}
+
+// Segment p of split sequence j: chunk-aligned thirds (the last one takes the rest).
+void segment_bounds(const int32_t *cu_host, int seq, int p, int32_t *b, int32_t *e) {
+    const int32_t bos = cu_host[seq], eos = cu_host[seq + 1];
+    const int32_t chunks = (eos - bos + 63) / 64;
+    const int32_t seg = (chunks + kda::kSplitP - 1) / kda::kSplitP * 64;
+    *b = bos + p * seg < eos ? bos + p * seg : eos;
+    *e = p == kda::kSplitP - 1 ? eos : (bos + (p + 1) * seg < eos ? bos + (p + 1) * seg : eos);
+}
+
+// Pass A, the chain of start states, pass B (kda_internal.h), on one stream.
+cudaError_t launch_prefill_tc_split(kda::PrefillArgs a, const int32_t *cu_host, cudaStream_t st) {
+    using namespace kda;
+    int n = 0;
+    for (int j = 0; j < a.split.num_seqs; ++j) {
+        const int seq = a.split.seqs[j];
+        int32_t b, e;
+        segment_bounds(cu_host, seq, 0, &b, &e);
+        a.split.units[n++] = SplitUnit{b, e, seq, UNIT_FIRST, j * kSplitP};
+        for (int p = 1; p + 1 < kSplitP; ++p) {
+            segment_bounds(cu_host, seq, p, &b, &e);
+            a.split.units[n++] = SplitUnit{b, e, seq, UNIT_LOCAL, j * kSplitP + p};
+            a.split.units[n++] = SplitUnit{b, e, seq, UNIT_HOMOG, j * kSplitP + p};
+        }
+    }
+    a.split.num_units = n;
+    a.split.plain_units = true;
+    cudaError_t err = launch_prefill_tc(a, st);
+    for (int p = 2; p < kSplitP && err == cudaSuccess; ++p) err = launch_split_combine(a, p, st);
+    if (err != cudaSuccess) return err;
+    n = 0;
+    for (int j = 0; j < a.split.num_seqs; ++j) {
+        const int seq = a.split.seqs[j];
+        for (int p = 1; p < kSplitP; ++p) {
+            int32_t b, e;
+            segment_bounds(cu_host, seq, p, &b, &e);
+            a.split.units[n++] = SplitUnit{b, e, seq, p + 1 < kSplitP ? UNIT_CONT : UNIT_LAST, j * kSplitP + p};
+        }
+    }
+    a.split.num_units = n;
+    a.split.plain_units = false;
+    return launch_prefill_tc(a, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -91,7 +172,7 @@ size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H, int
                                   int chunk, kda_dtype_t qkv_dtype) {
     if (total_tokens < 0 || total_tokens > INT32_MAX) return 0;
     if (check_prefill_shape(num_seqs, H, d_k, d_v, chunk, qkv_dtype) != KDA_OK) return 0;
-    return kda::workspace_layout(num_seqs).total;
+    return kda::workspace_layout(num_seqs, total_tokens, H, tc_shape(d_k, d_v, chunk, qkv_dtype)).total;
 }
 
 kda_status_t kda_prefill(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
@@ -109,7 +190,11 @@ kda_status_t kda_prefill(const void *q, const void *k, const void *v, kda_dtype_
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const kda_status_t pro = launch_prefill_prologue(a, st);
     if (pro != KDA_OK) return pro;
-    if (kda::prefill_tc_supported(a)) return from_cuda(kda::launch_prefill_tc(a, st));
+    if (kda::prefill_tc_supported(a)) {
+        if (plan_split(a, cu_seqlens_host, workspace, workspace_bytes))
+            return from_cuda(launch_prefill_tc_split(a, cu_seqlens_host, st));
+        return from_cuda(kda::launch_prefill_tc(a, st));
+    }
     return from_cuda(kda::launch_prefill_simt(a, st));
 }
 

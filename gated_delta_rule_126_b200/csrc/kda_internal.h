@@ -12,18 +12,62 @@ namespace kda {
 // Layout of the prefill workspace (all offsets 256-byte aligned).
 //   [0, 256)            device status words (error flag + detail)
 //   [256, 256 + 4*N)    sequence order, longest first (int32)
+// ---- sequence split (tensor-core prefill).  A sequence much longer than the rest
+// would keep H SMs busy long after the others finish; it is cut into kSplitP
+// segments.  The recurrence is affine in the state, S_end = M S_start + L with
+// M (d_k x d_k) the state's transition through a segment and L its end state from a
+// zero start, so: pass A runs segment 0 from S0 and, for each middle segment, L (from
+// zero) and M (from the identity, v = 0) in parallel; a small kernel chains
+// S_start(p) = M(p-1) S_start(p-1) + L(p-1); pass B runs the other segments from
+// their true start states.
+constexpr int kSplitP = 3;
+constexpr int kMaxSplitSeqs = 8;
+constexpr int kSplitMinLen = 16384;
+constexpr int kMaxSplitUnits = kMaxSplitSeqs * (2 * kSplitP - 3);
+enum UnitMode : int32_t { UNIT_FIRST = 1, UNIT_LOCAL = 2, UNIT_HOMOG = 3, UNIT_CONT = 4, UNIT_LAST = 5 };
+struct SplitUnit {
+    int32_t bos, eos, seq, mode;
+    int32_t slot;  // (split sequence j) * kSplitP + segment: the scratch state it reads or writes
+};
+struct SplitPlan {
+    int num_units = 0;  // split units at the front of a launch
+    int num_seqs = 0;   // split sequences, skipped where the plain ordering meets them
+    bool plain_units = true;  // the launch also runs every plain (sequence, head) after the split units
+    int32_t seqs[kMaxSplitSeqs] = {};
+    SplitUnit units[kMaxSplitUnits] = {};
+    float *sstart = nullptr, *lmat = nullptr, *mmat = nullptr;  // [slot][H][128][128] float32 each
+};
+
+// Most sequences a split can take for these sizes (the criterion in kda_api.cu:
+// L >= kSplitMinLen and 2 L 148 > 3 T H, so fewer than 296 / (3 H) sequences qualify).
+inline int split_max_seqs(int64_t total_tokens, int H) {
+    int64_t m = total_tokens / kSplitMinLen;
+    m = m < kMaxSplitSeqs ? m : kMaxSplitSeqs;
+    const int64_t by_h = 296 / (3 * int64_t(H > 0 ? H : 1));
+    return int(m < by_h ? m : by_h);
+}
+
 struct WorkspaceLayout {
     static constexpr size_t kStatusBytes = 256;
     size_t order_offset = kStatusBytes;
+    size_t split_offset = 0;  // three scratch state arrays when a split is possible
+    size_t split_array_bytes = 0;
     size_t total = 0;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-inline WorkspaceLayout workspace_layout(int num_seqs) {
+// split_states: room for a sequence split (tensor-core path only).
+inline WorkspaceLayout workspace_layout(int num_seqs, int64_t total_tokens = 0, int H = 0, bool split_states = false) {
     WorkspaceLayout L;
     L.order_offset = WorkspaceLayout::kStatusBytes;
     L.total = align256(L.order_offset + sizeof(int32_t) * size_t(num_seqs > 0 ? num_seqs : 1));
+    const int m = split_states ? split_max_seqs(total_tokens, H) : 0;
+    if (m > 0) {
+        L.split_offset = L.total;
+        L.split_array_bytes = size_t(m) * kSplitP * size_t(H) * 128 * 128 * sizeof(float);
+        L.total = align256(L.split_offset + 3 * L.split_array_bytes);
+    }
     return L;
 }
 
@@ -45,6 +89,7 @@ struct PrefillArgs {
     float *S_final;
     DeviceStatus *status;
     int32_t *order;       // sequence order (longest first), num_seqs entries
+    SplitPlan split;  // empty: every unit is a plain (sequence, head)
     // output epilogue (kda_prefill_gated): o is replaced by o / sqrt(mean(o^2) + eps) * w * sigmoid(gate)
     const void *gate = nullptr;          // [T, H, d_v], dtype; nullptr = plain prefill
     const float *norm_weight = nullptr;  // [d_v]
@@ -89,6 +134,8 @@ cudaError_t launch_decode_tokens(const DecodeTokensArgs &a, cudaStream_t stream)
 cudaError_t launch_prefill_simt(const PrefillArgs &a, cudaStream_t stream);
 bool prefill_tc_supported(const PrefillArgs &a);
 cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream);  // fuses the epilogue when a.gate is set
+// S_start(p) = M(p-1) S_start(p-1) + L(p-1) for segment p of every split sequence.
+cudaError_t launch_split_combine(const PrefillArgs &a, int p, cudaStream_t stream);
 cudaError_t launch_prologue(const PrologueArgs &a, cudaStream_t stream);
 // The output epilogue in place over a.o (after a prefill that does not fuse it).
 cudaError_t launch_gated_rmsnorm(const PrefillArgs &a, cudaStream_t stream);

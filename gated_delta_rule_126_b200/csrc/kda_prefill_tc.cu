@@ -136,7 +136,9 @@ struct TcMaps {
 // kGated: the output store applies the layer's output epilogue, y = o / sqrt(mean_j o_j^2 + eps)
 // * w * sigmoid(gate) per token and head (the KDA layer's sigmoid output gate and RMSNorm,
 // section "模型架构" of the same page), instead of storing o.
-template <bool kGated>
+// kSplit: the launch runs units of a sequence split (kda_internal.h) before the plain
+// (sequence, head) units; plain launches compile without the per-unit modes.
+template <bool kGated, bool kSplit>
 __global__ void __launch_bounds__(NT, 1)
     prefill_tc_kernel(const __grid_constant__ TcMaps maps, const PrefillArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -148,10 +150,43 @@ __global__ void __launch_bounds__(NT, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.H;
     const int h = blockIdx.x % H;
-    const int seq = a.order[blockIdx.x / H];
-    const int bos = a.cu_seqlens[seq], eos = a.cu_seqlens[seq + 1];
+    // The unit: a split segment (the first a.split.num_units) or a plain sequence.
+    constexpr size_t D2 = size_t(D) * D;
+    const int ui = blockIdx.x / H;
+    int seq, bos, eos, mode = 0;
+    const float *s0 = nullptr;  // initial state [d_k][d_v] (nullptr: zero, or the identity for UNIT_HOMOG)
+    float *sfin = nullptr;      // where the final state goes (nullptr: nowhere)
+    if (kSplit && ui < a.split.num_units) {
+        const SplitUnit u = a.split.units[ui];
+        seq = u.seq;
+        bos = u.bos;
+        eos = u.eos;
+        mode = u.mode;
+        const size_t slot = size_t(u.slot) * H + h;
+        if (mode == UNIT_FIRST) {
+            s0 = a.S0 ? a.S0 + (size_t(seq) * H + h) * D2 : nullptr;
+            sfin = a.split.sstart + (slot + H) * D2;  // the next segment's start state
+        } else if (mode == UNIT_LOCAL) {
+            sfin = a.split.lmat + slot * D2;
+        } else if (mode == UNIT_HOMOG) {
+            sfin = a.split.mmat + slot * D2;
+        } else {  // UNIT_CONT, UNIT_LAST
+            s0 = a.split.sstart + slot * D2;
+            if (mode == UNIT_LAST) sfin = a.S_final + (size_t(seq) * H + h) * D2;
+        }
+    } else {
+        seq = a.order[ui - (kSplit ? a.split.num_units : 0)];
+        if (kSplit)
+            for (int j = 0; j < a.split.num_seqs; ++j)
+                if (a.split.seqs[j] == seq) return;  // run by the split units (the same for the whole block)
+        bos = a.cu_seqlens[seq];
+        eos = a.cu_seqlens[seq + 1];
+        s0 = a.S0 ? a.S0 + (size_t(seq) * H + h) * D2 : nullptr;
+        sfin = a.S_final + (size_t(seq) * H + h) * D2;
+    }
+    const bool v_zero = kSplit && mode == UNIT_HOMOG;                       // the transition runs with v = 0
+    const bool o_skip = kSplit && (mode == UNIT_LOCAL || mode == UNIT_HOMOG);  // only the final state is wanted
     const int nchunks = (eos - bos + C - 1) / C;
-    const size_t unit = size_t(seq) * H + h;
 
     auto vec = [&](int par, uint32_t field) { return reinterpret_cast<float *>(sm + OFF_VEC + par * VEC_BYTES + field); };
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
@@ -174,6 +209,7 @@ __global__ void __launch_bounds__(NT, 1)
         for (int i = 0; i < 8; ++i) cnt[i] = 0;
         ptx::fence_mbar_init();
         *s_abort = 0;
+        *reinterpret_cast<float **>(sm + OFF_MISC + 8) = sfin;  // read back at the end (frees registers)
         ptx::prefetch_tmap(&maps.q);
         ptx::prefetch_tmap(&maps.k);
         ptx::prefetch_tmap(&maps.v);
@@ -255,7 +291,7 @@ __global__ void __launch_bounds__(NT, 1)
         const uint32_t tl = tbase + (uint32_t(warp * 32) << 16);
         const bool leader = tid == 0;
         if (leader && nchunks > 0) {
-            load_v(bos);
+            if (!v_zero) load_v(bos);
             if (kGated) load_g(bos);
         }
         const float w_row = kGated ? a.norm_weight[row] : 0.f;  // RMSNorm weight of value channel `row`
@@ -272,7 +308,10 @@ __global__ void __launch_bounds__(NT, 1)
             for (int p = 0; p < 4; ++p) {
                 for (int e = 0; e < 32; ++e) {
                     const int c = 32 * p + e;
-                    v[e] = __float_as_uint(a.S0 ? a.S0[(unit * D + c) * D + row] : 0.f);
+                    if constexpr (kSplit)
+                        v[e] = __float_as_uint(s0 ? s0[c * D + row] : (v_zero && c == row ? 1.f : 0.f));
+                    else
+                        v[e] = __float_as_uint(a.S0 ? a.S0[((size_t(seq) * H + h) * D + c) * D + row] : 0.f);
                 }
                 ptx::tmem_st32(tl + TS + 32 * p, v);
             }
@@ -398,17 +437,19 @@ __global__ void __launch_bounds__(NT, 1)
                     ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_QK + kq), IDESC_N128,
                                 ks > 0);
                 }
-                mwait(B_V, ci, true);
-                ptx::tc_fence_after();
-                for (int ks = 0; ks < 4; ++ks)
-                    ptx::mma_ss(tbase + TZ, ptx::sdesc_sw128_mn(sb + OFF_V + 2048 * ks, 8192, 1024),
-                                ptx::sdesc_sw128(sb + OFF_ID + 32 * ks), IDESC_BF16_AMN_N64, 1u);
+                if (!v_zero) {
+                    mwait(B_V, ci, true);
+                    ptx::tc_fence_after();
+                    for (int ks = 0; ks < 4; ++ks)
+                        ptx::mma_ss(tbase + TZ, ptx::sdesc_sw128_mn(sb + OFF_V + 2048 * ks, 8192, 1024),
+                                    ptx::sdesc_sw128(sb + OFF_ID + 32 * ks), IDESC_BF16_AMN_N64, 1u);
+                }
                 commit(B_M2);
             }
             mwait(B_M2, ci, leader);
             ptx::tc_fence_after();
             if (leader) {
-                if (has_next) load_v(s + C);  // the V tile has been read by the MMA
+                if (has_next && !v_zero) load_v(s + C);  // the V tile has been read by the MMA
                 // the [Kt; Qt] tile is free once M1 of this chunk has read it too
                 if (has_next && mwait(B_M1, ci, false)) load_qk(s + C);
             }
@@ -504,8 +545,8 @@ __global__ void __launch_bounds__(NT, 1)
             mwait(B_M45, ci, leader);
             ptx::tc_fence_after();
             if (leader) ptx::st_release(cnt + CNT_M45, ci + 1);
-            {  // E4: outputs of this chunk, staged over the Y^T tile as two 128-byte swizzled
-               // boxes (columns 0-63, 64-127)
+            if (!o_skip) {  // E4: outputs of this chunk, staged over the Y^T tile as two 128-byte
+                            // swizzled boxes (columns 0-63, 64-127)
                 uint32_t vo[2][32];
                 uint8_t *stage = sm + OFF_Y + (row >> 6) * 8192 + (row & 7) * 2;
                 const int ch = (row & 63) >> 3;
@@ -579,7 +620,8 @@ __global__ void __launch_bounds__(NT, 1)
             ptx::tc_fence_before();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
             if (kGated && leader && has_next) load_g(s + C);  // the gate tile has been read
-            if (L == C) {  // a full chunk: two TMA tile stores
+            if (o_skip) {
+            } else if (L == C) {  // a full chunk: two TMA tile stores
                 if (leader) {
                     ptx::tma_store_3d(&maps.o, sm + OFF_Y, 0, h, s);
                     ptx::tma_store_3d(&maps.o, sm + OFF_Y + 8192, 64, h, s);
@@ -600,6 +642,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (!*reinterpret_cast<volatile int *>(s_abort)) {
             ptx::tc_fence_after();
             const float *ecm_last = vec((nchunks - 1) & 1, VEC_ECM);
+            float *const sf = *reinterpret_cast<float *const *>(sm + OFF_MISC + 8);
             uint32_t v[32];
             for (int p = 0; p < 4; ++p) {
                 ptx::tmem_ld32(tl + TS + 32 * p, v);
@@ -607,7 +650,11 @@ __global__ void __launch_bounds__(NT, 1)
                 for (int e = 0; e < 32; ++e) {
                     const int c = 32 * p + e;
                     const float f = nchunks > 0 ? ecm_last[c] : 1.f;
-                    a.S_final[(unit * D + c) * D + row] = __uint_as_float(v[e]) * f;
+                    if constexpr (kSplit) {
+                        if (sf) sf[c * D + row] = __uint_as_float(v[e]) * f;
+                    } else {
+                        a.S_final[((size_t(seq) * H + h) * D + c) * D + row] = __uint_as_float(v[e]) * f;
+                    }
                 }
             }
         }
@@ -913,13 +960,15 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool kGated>
+template <bool kGated, bool kSplit>
 cudaError_t launch_tc(const TcMaps &maps, const PrefillArgs &a, cudaStream_t stream) {
-    cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel<kGated>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           int(smem_alloc(kGated)));
+    cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel<kGated, kSplit>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_alloc(kGated)));
     if (err != cudaSuccess) return err;
-    const unsigned grid = unsigned(a.num_seqs) * unsigned(a.H);
-    prefill_tc_kernel<kGated><<<grid, NT, smem_alloc(kGated), stream>>>(maps, a);
+    const unsigned units = unsigned(a.split.num_units) + (a.split.plain_units ? unsigned(a.num_seqs) : 0u);
+    const unsigned grid = units * unsigned(a.H);
+    if (grid == 0) return cudaSuccess;
+    prefill_tc_kernel<kGated, kSplit><<<grid, NT, smem_alloc(kGated), stream>>>(maps, a);
     return cudaGetLastError();
 }
 
@@ -938,10 +987,13 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
         !make_map(&maps.la, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.H, a.total_tokens) ||
         !make_map(&maps.o, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens))
         return cudaErrorInvalidValue;
-    if (a.gate == nullptr) return launch_tc<false>(maps, a, stream);
+    if (a.gate == nullptr) {
+        if (a.split.num_units > 0 || a.split.num_seqs > 0) return launch_tc<false, true>(maps, a, stream);
+        return launch_tc<false, false>(maps, a, stream);
+    }
     if (!make_map(&maps.g, a.gate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens))
         return cudaErrorInvalidValue;
-    return launch_tc<true>(maps, a, stream);
+    return launch_tc<true, false>(maps, a, stream);
 }
 
 }  // namespace kda

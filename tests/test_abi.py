@@ -57,6 +57,11 @@ def test_workspace_size(lib):
     assert ws(-1, 0, 32, 128, 128, 64, 1) == 0
     assert ws(1, -5, 32, 128, 128, 64, 1) == 0
     assert ws(1, 1 << 40, 32, 128, 128, 64, 1) == 0      # more tokens than int32 offsets
+    # the tensor-core shapes reserve room for the sequence split once a call can hold one
+    # (at least 16,384 tokens): three [slot][H][128][128] float32 arrays
+    small, big = ws(2, 8192, 32, 128, 128, 64, 1), ws(2, 1 << 20, 32, 128, 128, 64, 1)
+    assert small < 4096 and big >= 3 * 3 * 3 * 32 * 128 * 128 * 4
+    assert ws(2, 1 << 20, 32, 64, 64, 64, 1) < 4096      # CUDA-core path: no split
 
 
 FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: every case fails on the host
