@@ -64,8 +64,8 @@ def decode_bytes_per_head_step(dk, dv, qkv_bytes):
 # Prefill: one launch on 2 x 8192 tokens x 32 heads (524,288 head-tokens).
 MEASURED_TRAFFIC = {
     "prefill_tc": {"source": "gated_delta_rule_126_b200/csrc/kda_prefill_tc.cu",
-                   "sha256": "92c410c3acb0b10e4ea05ba53d7a7f6af863449f41b8e51563394789b9d86fde",
-                   "units": 2 * 8192 * 32, "dram_bytes": 673498112 + 121482752},
+                   "sha256": "aba0ead2825c75f880c66a0f2a8159bd9f4feb8b9941b462a0047845eb598f77",
+                   "units": 2 * 8192 * 32, "dram_bytes": 673465088 + 120951808},
 }
 
 
