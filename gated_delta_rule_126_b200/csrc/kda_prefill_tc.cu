@@ -19,26 +19,34 @@
 //     M1  [A; P]^raw = [Kt; Qt] Kb^T                 M=128 N=64  K=128
 //     M2  Z          = Sop [Kt; Qt]^T                M=128 N=128 K=128
 //           Z[:, :64] = (K e^{g} S)^T,  Z[:, 64:] = (Q e^{g} S)^T
-//     M3  U^T        = Y^T T^T,  Y^T = V^T - Z[:, :64]   M=128 N=64  K=64
+//     Mv  Z[:, :64] += V^T (-I)     (V read MN-major from its TMA tile)   N=64 K=64
+//     M3  U^T        = Y^T T^T,  Y^T = -Z[:, :64]    M=128 N=64  K=64
 //     M4  R         += U^T Kb      (Kb read as an MN-major operand)  N=128 K=64
 //     M5  Z[:, 64:] += U^T P^T  ( = O^T )                   N=64  K=64
 //   TMEM holds R = S^T Diag(e^{g_m - g_L}) of the previous chunk rather than S^T:
 //   the per-channel factors e^{g_L - g_m} and e^{g_m} then fold into one pass over
 //   R at the start of each chunk, which also packs Sop, so no K e^{g}, Q e^{g} or
-//   (K e^{g_L - g})^T tile is built.
+//   (K e^{g_L - g})^T tile is built.  Y^T and U^T are written back to TMEM as fp16
+//   pairs (over Sop, which M2 has read), so M3-M5 take their A operand from TMEM.
 // * Two warp groups work on different chunks at once.  The prep group (warps
-//   4-11) builds chunk c + 1 -- decayed rows, M1, A and P, the triangular solve
-//   for T -- while the state group (warps 0-3) runs chunk c -- the pass over R,
-//   M2, Y, M3, U, M4/M5 and the outputs -- and, while it waits for T, the
-//   running sums of chunk c + 1.  They hand buffers over through release/acquire
-//   progress counters in shared memory; the decayed-row (Kb) and P tiles and the
-//   per-chunk vectors are double-buffered by chunk parity.
+//   4-11) builds chunk c + 1 -- decayed rows, M1, A and P, and X = (I + A)^{-1} --
+//   while the state group (warps 0-3) runs chunk c -- the pass over R, M2, Y,
+//   T = X Diag(beta), M3, U, M4/M5 and the outputs -- and, while it waits for X,
+//   the running sums of chunk c + 1.  They hand buffers over through
+//   release/acquire progress counters in shared memory; the decayed-row (Kb) and P
+//   tiles and the per-chunk vectors are double-buffered by chunk parity.
 // * Operands are fp16 (fp32 accumulation): the S-dependent chain keeps the
 //   relative error near fp16's 2^-11, which the parity bounds need (bf16 operands
-//   do not meet them).  Sop lives in TMEM (fp16 pairs per column).
+//   do not meet them).
 // * q, k, v and log alpha tiles arrive by TMA in the 128-byte swizzled layout that
-//   the UMMA descriptors use, so the decayed operand rows are built in place.
-// * T is formed in fp32 by a blocked (16x16) forward substitution in shared memory.
+//   the UMMA descriptors use, so the decayed operand rows are built in place.  A
+//   full chunk's outputs leave by two TMA tile stores; a shorter last chunk row by
+//   row (its later rows belong to the next sequence).
+// * X is formed in fp32 in shared memory by block doubling: the four 16x16
+//   diagonal blocks by row substitution, then the two 32x32 halves, then the
+//   lower-left 32x32 block, every stage on all 256 prep threads.
+// * kGated applies the layer's output epilogue (sigmoid gate and RMSNorm) before
+//   the output store; kSplit runs the units of a sequence split (kda_internal.h).
 // * Every wait is bounded: one that runs out sets the workspace error flag and
 //   both groups stop at their next group barrier (decided uniformly by a
 //   barrier-or), drain what they have in flight and free TMEM.
