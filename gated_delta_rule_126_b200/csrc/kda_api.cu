@@ -2,6 +2,7 @@
 // kernel launches on the caller's stream.  See include/kda.h for the contract.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "kda_internal.h"
 
@@ -116,9 +117,54 @@ void segment_bounds(const int32_t *cu_host, int seq, int p, int32_t *b, int32_t 
     *e = p == kda::kSplitP - 1 ? eos : (bos + (p + 1) * seg < eos ? bos + (p + 1) * seg : eos);
 }
 
-// Pass A, the chain of start states, pass B (kda_internal.h), on one stream.
+// A second, high-priority stream and two events per device for the split: it runs the
+// split units, the chain of start states and pass B (the critical path), while the
+// caller's stream runs the plain sequences, which they do not depend on.  Created
+// once, never destroyed.
+struct SideStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+// Held across a split's whole fork / launches / join sequence: the side stream and its
+// events are shared by every caller on the device.
+std::mutex g_side_mu;
+
+bool side_stream(SideStream *out) {  // call with g_side_mu held
+    static SideStream per_device[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    SideStream &s = per_device[dev];
+    if (!s.stream) {
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) greatest = 0;
+        if (cudaStreamCreateWithPriority(&s.stream, cudaStreamNonBlocking, greatest) != cudaSuccess) return false;
+        if (cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess) {
+            s.stream = nullptr;
+            return false;
+        }
+    }
+    *out = s;
+    return true;
+}
+
+// Pass A, the chain of start states and pass B of the split units (kda_internal.h) on
+// a high-priority side stream, issued first; the plain sequences on the caller's
+// stream meanwhile; then the caller's stream waits for the side stream.  Without a
+// side stream, everything runs in order on the caller's stream.
 cudaError_t launch_prefill_tc_split(kda::PrefillArgs a, const int32_t *cu_host, cudaStream_t st) {
     using namespace kda;
+    std::lock_guard<std::mutex> lock(g_side_mu);
+    SideStream side;
+    const bool forked = side_stream(&side);
+    cudaStream_t chain = forked ? side.stream : st;
+    cudaError_t err = cudaSuccess;
+    if (forked) {
+        err = cudaEventRecord(side.fork, st);
+        if (err == cudaSuccess) err = cudaStreamWaitEvent(side.stream, side.fork, 0);
+        if (err != cudaSuccess) return err;
+    }
     int n = 0;
     for (int j = 0; j < a.split.num_seqs; ++j) {
         const int seq = a.split.seqs[j];
@@ -132,22 +178,31 @@ cudaError_t launch_prefill_tc_split(kda::PrefillArgs a, const int32_t *cu_host, 
         }
     }
     a.split.num_units = n;
-    a.split.plain_units = true;
-    cudaError_t err = launch_prefill_tc(a, st);
-    for (int p = 2; p < kSplitP && err == cudaSuccess; ++p) err = launch_split_combine(a, p, st);
+    a.split.plain_units = !forked;
+    err = launch_prefill_tc(a, chain);
+    for (int p = 2; p < kSplitP && err == cudaSuccess; ++p) err = launch_split_combine(a, p, chain);
     if (err != cudaSuccess) return err;
+    PrefillArgs passB = a;
     n = 0;
     for (int j = 0; j < a.split.num_seqs; ++j) {
         const int seq = a.split.seqs[j];
         for (int p = 1; p < kSplitP; ++p) {
             int32_t b, e;
             segment_bounds(cu_host, seq, p, &b, &e);
-            a.split.units[n++] = SplitUnit{b, e, seq, p + 1 < kSplitP ? UNIT_CONT : UNIT_LAST, j * kSplitP + p};
+            passB.split.units[n++] = SplitUnit{b, e, seq, p + 1 < kSplitP ? UNIT_CONT : UNIT_LAST, j * kSplitP + p};
         }
     }
-    a.split.num_units = n;
-    a.split.plain_units = false;
-    return launch_prefill_tc(a, st);
+    passB.split.num_units = n;
+    passB.split.plain_units = false;
+    err = launch_prefill_tc(passB, chain);
+    if (err != cudaSuccess || !forked) return err;
+    PrefillArgs plain = a;  // every plain (sequence, head); split sequences are skipped
+    plain.split.num_units = 0;
+    plain.split.plain_units = true;
+    err = launch_prefill_tc(plain, st);
+    if (err == cudaSuccess) err = cudaEventRecord(side.join, side.stream);
+    if (err == cudaSuccess) err = cudaStreamWaitEvent(st, side.join, 0);
+    return err;
 }
 
 }  // namespace

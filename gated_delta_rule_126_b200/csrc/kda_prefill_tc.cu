@@ -996,6 +996,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
         !make_map(&maps.o, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens))
         return cudaErrorInvalidValue;
     if (a.gate == nullptr) {
+        // a launch that holds split units, or skips split sequences, takes the kSplit form
         if (a.split.num_units > 0 || a.split.num_seqs > 0) return launch_tc<false, true>(maps, a, stream);
         return launch_tc<false, false>(maps, a, stream);
     }

@@ -102,3 +102,31 @@ def test_decode_tokens_full_shape_sampled():
         worst_o = max(worst_o, rel_l2(host64(o[b, :, h]), o_ref))
         worst_S = max(worst_S, rel_l2(host64(inp["S_pool"][slot, h]), S_ref))
     assert worst_o <= TOL["bf16"]["o"] and worst_S <= TOL["bf16"]["S"], (worst_o, worst_S)
+
+
+def test_decode_tokens_unaligned_rows_take_the_other_kernel():
+    """q/k/v/log alpha whose rows start 2 bytes past a 16-byte boundary (a contiguous view
+    one element into a buffer) cannot use the streaming kernel's 16-byte copies; the
+    call must take the per-unit kernel and still match the oracle."""
+    B, n, H, num_slots = 5, 3, 2, 5
+    inp = _tokens_inputs(B, n, H, 128, 128, "bf16", num_slots, seed=25)
+
+    def shifted(t):  # the same values, stored one element past an aligned start
+        buf = torch.empty(t.numel() + 8, dtype=t.dtype, device=DEV)
+        view = buf[1:1 + t.numel()].view(t.shape)
+        view.copy_(t)
+        return view
+
+    q, k, v = shifted(inp["q"]), shifted(inp["k"]), shifted(inp["v"])
+    la = shifted(inp["log_alpha"])
+    assert q.data_ptr() % 16 != 0
+    pool0 = inp["S_pool"].clone()
+    o = kda_decode_tokens(q, k, v, la, inp["beta"], inp["S_pool"])
+    torch.cuda.synchronize()
+    worst_o = worst_S = 0.0
+    for b in range(B):
+        for h in range(H):
+            o_ref, S_ref = _oracle(inp, b, h, b, pool0)
+            worst_o = max(worst_o, rel_l2(host64(o[b, :, h]), o_ref))
+            worst_S = max(worst_S, rel_l2(host64(inp["S_pool"][b, h]), S_ref))
+    assert worst_o <= TOL["bf16"]["o"] and worst_S <= TOL["bf16"]["S"], (worst_o, worst_S)
