@@ -58,6 +58,8 @@ def _declare(lib):
                                       vp, vp]
     lib.kda_workspace_status.restype = i32
     lib.kda_workspace_status.argtypes = [vp, vp]
+    lib.kda_wait_timeout_selftest.restype = i32
+    lib.kda_wait_timeout_selftest.argtypes = [vp, sz, c.c_longlong, vp]
     return lib
 
 
@@ -326,3 +328,13 @@ def kda_decode_tokens(q, k, v, log_alpha, beta, S_pool, slot_idx=None, o=None, s
 def workspace_status(workspace, stream=None):
     """Status flagged by the kernels of the last prefill that used ``workspace``."""
     return int(load().kda_workspace_status(_ptr(workspace), _stream_handle(stream)))
+
+
+def wait_timeout_selftest(workspace, max_cycles, stream=None):
+    """Run the kernel whose bounded waits never see their event (see
+    ``kda_wait_timeout_selftest`` in kda.h); the caller reads the flag it leaves
+    with :func:`workspace_status`."""
+    _need(workspace, "workspace", torch.uint8)
+    st = load().kda_wait_timeout_selftest(_ptr(workspace), workspace.numel(), int(max_cycles),
+                                          _stream_handle(stream))
+    _check(st, "kda_wait_timeout_selftest")

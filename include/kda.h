@@ -266,6 +266,30 @@ KDA_API kda_status_t kda_decode_tokens(const void *q, const void *k, const void 
  */
 KDA_API kda_status_t kda_workspace_status(const void *workspace, kda_stream_t stream);
 
+/*
+ * kda_wait_timeout_selftest -- checks, on the caller's device, the error path that
+ * every bounded wait inside the prefill kernels takes when the event it waits for
+ * never comes.  One small kernel (1 block, 64 threads) waits on an mbarrier phase
+ * that no thread completes and on a shared-memory progress counter that no thread
+ * advances, each for at most `max_cycles` SM clock cycles; both waits run out, the
+ * kernel sets the status word at the start of `workspace` (the same word
+ * kda_prefill's kernels set) and exits normally.  Nothing else is touched, so the
+ * context stays usable and kda_workspace_status(workspace, stream) then returns
+ * KDA_ERR_DEVICE_FAULT (and clears the word).
+ *
+ *   workspace        device buffer of >= 256 bytes, 256-byte aligned
+ *                    (a kda_prefill workspace will do); its first 8 bytes are
+ *                    cleared, then written by the kernel
+ *   max_cycles       1 .. 4e9 (4e9 is the prefill kernels' own limit, about two
+ *                    seconds at the B200's top SM clock)
+ *
+ * Returns KDA_ERR_WORKSPACE for a missing, short or misaligned workspace,
+ * KDA_ERR_INVALID_ARG for max_cycles out of range, KDA_ERR_CUDA if the launch
+ * failed; the launch is asynchronous on `stream`.
+ */
+KDA_API kda_status_t kda_wait_timeout_selftest(void *workspace, size_t workspace_bytes, long long max_cycles,
+                                       kda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

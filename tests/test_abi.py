@@ -30,7 +30,8 @@ def declared_symbols():
 def test_header_declares_the_abi():
     assert declared_symbols() == sorted([
         "kda_decode_step", "kda_decode_tokens", "kda_prefill", "kda_prefill_gated", "kda_prefill_noalloc", "kda_prologue",
-        "kda_prefill_workspace_size", "kda_status_string", "kda_version", "kda_workspace_status"])
+        "kda_prefill_workspace_size", "kda_status_string", "kda_version", "kda_wait_timeout_selftest",
+        "kda_workspace_status"])
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -165,6 +166,15 @@ def test_decode_tokens_rejects_bad_arguments(lib):
     assert f(*args(q=None)) == INVALID
     assert f(*args(S=ctypes.c_void_p((1 << 20) + 4))) == INVALID
     assert f(*args(n=0)) == 0 and f(*args(B=0)) == 0
+
+
+def test_wait_timeout_selftest_rejects_bad_arguments(lib):
+    f = lib.kda_wait_timeout_selftest
+    assert f(None, 256, 1000, None) == WORKSPACE
+    assert f(FAKE, 255, 1000, None) == WORKSPACE                      # shorter than the status block
+    assert f(ctypes.c_void_p((1 << 20) + 16), 256, 1000, None) == WORKSPACE  # not 256-byte aligned
+    assert f(FAKE, 256, 0, None) == INVALID
+    assert f(FAKE, 256, 4000000001, None) == INVALID
 
 
 def test_binding_raises_without_library(tmp_path):
