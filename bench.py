@@ -272,8 +272,9 @@ def run_reference(args):
 
 
 def run_ours(args):
-    from gated_delta_rule_126_b200 import (kda_decode_step, kda_decode_tokens, kda_prefill,
-                                           kda_prefill_gated, kda_prologue, prefill_workspace_size)
+    from gated_delta_rule_126_b200 import (backward_workspace_size, kda_backward, kda_decode_step,
+                                           kda_decode_tokens, kda_prefill, kda_prefill_gated, kda_prologue,
+                                           prefill_workspace_size)
     world, rank, local = dist_setup("nccl")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -422,6 +423,39 @@ def run_ours(args):
                                  "frac": p_gbs / hbm_peak, "alg_bytes_per_launch": p_bytes}}
         del pin, pout
 
+    # the backward pass (training) on the same batch: dO and dS_final given, gradients of
+    # q, k, v, log alpha, beta and S0 out; three launches (forward sweep with checkpoints,
+    # backward sweep, reduction over value-column slices), float32 on CUDA cores
+    backward = None
+    if not args.no_backward:
+        dO, dSf = inputs.grad_inputs(T, N, w.H, w.dk, w.dv, w.dtype, seed=w.seed + 13 + 1000 * rank,
+                                     device=dev)
+        bws = torch.empty(max(256, backward_workspace_size(N, T, w.H, w.dk, w.dv)), dtype=torch.uint8,
+                          device=dev)
+
+        def bstep():
+            kda_backward(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["cu_seqlens"], dO,
+                         cu_seqlens_host=cu_host, S0=inp["S0"], dS_final=dSf, workspace=bws, stream=stream)
+
+        for _ in range(args.warmup):
+            bstep()
+        barrier(world)
+        b_steps = max(1, min(args.steps, 5))
+        b_el = max_over_ranks(time_region(bstep, b_steps, stream), world)
+        b_t = b_el / b_steps
+        # flops per state element and token: forward sweep 5 (decay, P^T k, rank-1 update),
+        # adjoint 18 (P, S_t, G += q do^T, S_t do, G e, G^T k, dP, P du, dP.P, alpha dP)
+        b_flops = head_tokens * w.dk * w.dv * 23
+        b_tf = b_flops / b_t / 1e12
+        alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        backward = {"value": weak_scaling_value(T, b_steps, b_el, world), "unit": UNIT,
+                    "ms_per_step": b_t * 1e3, "steps": b_steps, "gpu_launches_per_step": 3,
+                    "grads": "dq, dk, dv, dlog_alpha, dbeta, dS0 (float32)",
+                    "roofline": {"bound": "alu", "achieved": b_tf, "peak": alu_peak, "unit": "TFLOP/s",
+                                 "frac": b_tf / alu_peak, "alg_flops_per_launch": b_flops,
+                                 "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"}}
+        del dO, dSf, bws
+
     # decode: 256 sequences x 32 heads, 64 consecutive one-token steps
     decode = None
     if not args.no_decode:
@@ -503,7 +537,7 @@ def run_ours(args):
                 "gpu_launches": prefill_launches(w.seqlens, w.H, w.dtype == "bf16" and w.dk == 128 and w.dv == 128
                                                  and w.chunk == 64) * args.steps,
                 "clocks": clk.summary(), "decode": decode,
-                "gated_epilogue": gated, "prologue": prologue}
+                "gated_epilogue": gated, "prologue": prologue, "backward": backward}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -524,6 +558,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-gated", action="store_true")
     ap.add_argument("--no-prologue", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps

@@ -12,16 +12,18 @@ binding over that ABI, with the same names:
   that makes the prefill's inputs from the projections;
 * ``kda_decode_step`` -- one recurrent decode step for a batch of sequences;
 * ``kda_decode_tokens`` -- n tokens per sequence with states in a slot pool;
-* ``prefill_workspace_size``, ``workspace_status``, ``KdaError``;
+* ``kda_backward``    -- gradients of the recurrence with respect to every input;
+* ``prefill_workspace_size``, ``backward_workspace_size``, ``workspace_status``, ``KdaError``;
 * ``wait_timeout_selftest`` -- runs the kernels' bounded-wait error path on events
   that never come, leaving the flag ``workspace_status`` reads.
 
 ``inputs`` holds the seeded synthetic input generators.  Importing the package
 does not load the CUDA library; the first call does, and raises if it is missing.
 """
-from ._binding import (KdaError, kda_decode_step, kda_decode_tokens, kda_prefill,
-                       kda_prefill_gated, kda_prologue, load, prefill_workspace_size,
-                       wait_timeout_selftest, workspace_status)
+from ._binding import (KdaError, backward_workspace_size, kda_backward, kda_decode_step,
+                       kda_decode_tokens, kda_prefill, kda_prefill_gated, kda_prologue, load,
+                       prefill_workspace_size, wait_timeout_selftest, workspace_status)
 
-__all__ = ["KdaError", "kda_decode_step", "kda_decode_tokens", "kda_prefill", "kda_prefill_gated",
-           "kda_prologue", "load", "prefill_workspace_size", "wait_timeout_selftest", "workspace_status"]
+__all__ = ["KdaError", "backward_workspace_size", "kda_backward", "kda_decode_step", "kda_decode_tokens",
+           "kda_prefill", "kda_prefill_gated", "kda_prologue", "load", "prefill_workspace_size",
+           "wait_timeout_selftest", "workspace_status"]

@@ -58,6 +58,11 @@ def _declare(lib):
                                       vp, vp]
     lib.kda_workspace_status.restype = i32
     lib.kda_workspace_status.argtypes = [vp, vp]
+    lib.kda_backward_workspace_size.restype = sz
+    lib.kda_backward_workspace_size.argtypes = [i32, i64, i32, i32, i32]
+    lib.kda_backward.restype = i32
+    lib.kda_backward.argtypes = [vp, vp, vp, i32, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp, vp,
+                                 vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.kda_wait_timeout_selftest.restype = i32
     lib.kda_wait_timeout_selftest.argtypes = [vp, sz, c.c_longlong, vp]
     return lib
@@ -324,6 +329,60 @@ def kda_decode_tokens(q, k, v, log_alpha, beta, S_pool, slot_idx=None, o=None, s
     _check(st, "kda_decode_tokens")
     return o
 
+
+def backward_workspace_size(num_seqs, total_tokens, H, d_k, d_v):
+    return int(load().kda_backward_workspace_size(int(num_seqs), int(total_tokens), int(H), int(d_k),
+                                                  int(d_v)))
+
+
+def kda_backward(q, k, v, log_alpha, beta, cu_seqlens, dO, cu_seqlens_host=None, S0=None,
+                 dS_final=None, want_dS0=True, workspace=None, stream=None):
+    """Gradients of the KDA recurrence (see ``kda_backward`` in kda.h).
+
+    Inputs as ``kda_prefill`` plus dO [T,H,d_v] (dtype of q) and dS_final
+    [N,H,d_k,d_v] f32 or None.  Returns a dict of float32 tensors dq, dk, dv,
+    dlog_alpha, dbeta and dS0 (None unless ``want_dS0``).
+    """
+    lib = load()
+    dev = q.device
+    dt = q.dtype
+    if dt not in DTYPE_CODE:
+        raise ValueError("q/k/v dtype must be float32 or bfloat16")
+    _need(q, "q", dt)
+    T, H, dk = q.shape
+    _need(k, "k", dt, dev)
+    _need(v, "v", dt, dev)
+    _need(dO, "dO", dt, dev)
+    dv = v.shape[2]
+    _need(log_alpha, "log_alpha", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    for t, name in ((S0, "S0"), (dS_final, "dS_final")):
+        if t is not None:
+            _need(t, name, torch.float32, dev)
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu()
+    cu_h = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
+    N = cu_h.numel() - 1
+    if cu_seqlens.numel() != N + 1:
+        raise ValueError("cu_seqlens and cu_seqlens_host differ in length")
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = dict(dq=torch.empty(T, H, dk, **f32), dk=torch.empty(T, H, dk, **f32),
+               dv=torch.empty(T, H, dv, **f32), dlog_alpha=torch.empty(T, H, dk, **f32),
+               dbeta=torch.empty(T, H, **f32),
+               dS0=torch.empty(N, H, dk, dv, **f32) if want_dS0 else None)
+    ws_bytes = backward_workspace_size(N, T, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = lib.kda_backward(_ptr(q), _ptr(k), _ptr(v), DTYPE_CODE[dt], _ptr(log_alpha), _ptr(beta),
+                              _ptr(S0), _ptr(cu_seqlens), ctypes.c_void_p(cu_h.data_ptr()), N, H, dk, dv,
+                              _ptr(dO), _ptr(dS_final), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                              _ptr(out["dlog_alpha"]), _ptr(out["dbeta"]), _ptr(out["dS0"]),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream_handle(stream))
+    _check(st, "kda_backward")
+    return out
 
 def workspace_status(workspace, stream=None):
     """Status flagged by the kernels of the last prefill that used ``workspace``."""

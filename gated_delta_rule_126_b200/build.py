@@ -17,7 +17,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB_PATH = os.path.join(LIB_DIR, "libkda_b200.so")
 SOURCES = ["kda_api.cu", "kda_decode.cu", "kda_prefill_simt.cu", "kda_prefill_tc.cu", "kda_noalloc.cu",
-           "kda_epilogue.cu", "kda_prologue.cu", "kda_split.cu", "kda_selftest.cu"]
+           "kda_epilogue.cu", "kda_prologue.cu", "kda_split.cu", "kda_selftest.cu",
+           "kda_backward.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-fvisibility=hidden",

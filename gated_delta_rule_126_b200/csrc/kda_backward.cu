@@ -1,0 +1,396 @@
+// Backward pass of the KDA recurrence (training): exact gradients of
+// sum <dO, o> + <dS_final, S_final> with respect to q, k, v, log alpha, beta and S0.
+//
+// The forward map is the state-update equation of the wiki page "Kimi Linear
+// 高效注意力架构", section "关键技术方法 > Kimi Delta Attention (KDA)", read out
+// from the post-update state, token by token:
+//   P_t = Diag(alpha_t) S_{t-1},  w_t = v_t - P_t^T k_t,  S_t = P_t + beta_t k_t w_t^T,
+//   o_t = S_t^T q_t,  alpha_t = exp(log alpha_t).
+// Its adjoint, with G = dL/dS_t carried from the last token back to the first:
+//   G += q_t do_t^T;  dq_t = S_t do_t;  de = G^T k_t (de = dL/d(beta_t w_t));
+//   dv_t = beta_t de;  dbeta_t = de . w_t;  du = -beta_t de;
+//   dP = G + k_t du^T;  dk_t = G (beta_t w_t) + P_t du;
+//   dlog_alpha_t[i] = sum_j dP[i][j] P_t[i][j];  G <- Diag(alpha_t) dP;  dS0 = G at the start.
+//
+// Every value column j of the state evolves on its own given (k, alpha, beta): the
+// key-side operators act on rows only.  So the work is cut into slices of 16 value
+// columns, one 128-thread block per (sequence, head, slice), thread i owning key row
+// i of the slice; the reductions over value columns (dq, dk, dlog_alpha, dbeta) are
+// per-slice partial sums that a third kernel adds up.  The one reduction over key
+// rows on the recurrence's critical path (w in the forward sweep, de in the backward
+// sweep) is a transposed warp butterfly plus a 4-warp exchange in shared memory.
+//
+// Three launches:
+//   1. states: the forward sweep, storing w_t for every token and the state before
+//      every 32nd token of each sequence (checkpoints);
+//   2. grads:  the backward sweep, 32-token blocks from the last: the 4-token
+//      sub-blocks (last first) are replayed from the block's checkpoint with the
+//      stored w (no reduction needed), their input states kept in shared memory;
+//   3. reduce: sums the slices' partial dq, dk, dlog_alpha and dbeta.
+// CUDA cores in fp32 throughout; no tensor cores and no waits on other blocks.
+#include <algorithm>
+#include <cmath>
+
+#include "kda_internal.h"
+
+namespace {
+
+constexpr int kCols = 16;  // value columns per slice
+constexpr int kRows = 128; // threads per block = key rows
+constexpr int kBlk = 32;   // tokens between checkpoints
+constexpr int kSub = 4;    // tokens per replayed sub-block
+
+struct BwdArgs {
+    const void *q, *k, *v, *dO;
+    const float *log_alpha, *beta, *S0, *dS_final;
+    const int32_t *cu_seqlens;
+    int num_seqs, H, dk, dv, nsl;
+    int64_t T;
+    float *dq, *dk_out, *dv_out, *dla, *dbeta, *dS0;
+    float4 *ck;            // [blk][H][nsl][4][128] float4: checkpoint slices, row-interleaved
+    float *w;              // [T][H][nsl * 16]
+    float *pq, *pk, *pg;   // [nsl][T][H][dk] partial sums over a slice's columns
+    float *pb;             // [nsl][T][H]
+};
+
+struct BwdLayout {
+    size_t ck_offset = 0, w_offset = 0, p_offset = 0, pb_offset = 0, total = 0;
+    size_t p_bytes = 0;  // one of pq, pk, pg
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Checkpoint slots: sequence n's blocks start at floor(cu[n] / 32) + n, which leaves
+// room for ceil(L_n / 32) blocks before sequence n + 1's first slot.
+BwdLayout bwd_layout(int num_seqs, int64_t T, int H, int dk, int dv) {
+    BwdLayout L;
+    const int nsl = (dv + kCols - 1) / kCols;
+    const size_t nblk = size_t(T / kBlk) + size_t(num_seqs) + 1;
+    L.ck_offset = kda::WorkspaceLayout::kStatusBytes;
+    L.w_offset = L.ck_offset + align256(nblk * size_t(H) * nsl * 4 * kRows * sizeof(float4));
+    L.p_offset = L.w_offset + align256(size_t(T) * H * nsl * kCols * sizeof(float));
+    L.p_bytes = align256(size_t(nsl) * T * H * dk * sizeof(float));
+    L.pb_offset = L.p_offset + 3 * L.p_bytes;
+    L.total = L.pb_offset + align256(size_t(nsl) * T * H * sizeof(float));
+    return L;
+}
+
+__device__ __forceinline__ float ldf(const float *p) { return *p; }
+__device__ __forceinline__ float ldf(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+// Sums c[j] over the block's 128 threads for each of the 16 columns j; every thread
+// gets all 16 sums.  Within a warp a transposed butterfly halves the columns each
+// lane carries at every step (16 shuffles), leaving column (lane >> 1) & 15 summed
+// over the warp in lanes 2m and 2m + 1; the 4 warps then meet in shared memory.
+// `buf` alternates between two halves on consecutive calls, so one barrier a call
+// suffices: a thread's reads of a half come before its next call's barrier.
+__device__ __forceinline__ void column_sums(const float (&c)[kCols], float4 (*buf)[4], int warp, int lane,
+                                            float (&out)[kCols]) {
+    constexpr unsigned kAll = 0xffffffffu;
+    float x8[8], x4[4], x2[2];
+    const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4, u2 = lane & 2;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x8[j] = (u16 ? c[j + 8] : c[j]) + __shfl_xor_sync(kAll, u16 ? c[j] : c[j + 8], 16);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) x4[j] = (u8 ? x8[j + 4] : x8[j]) + __shfl_xor_sync(kAll, u8 ? x8[j] : x8[j + 4], 8);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) x2[j] = (u4 ? x4[j + 2] : x4[j]) + __shfl_xor_sync(kAll, u4 ? x4[j] : x4[j + 2], 4);
+    float x1 = (u2 ? x2[1] : x2[0]) + __shfl_xor_sync(kAll, u2 ? x2[0] : x2[1], 2);
+    x1 += __shfl_xor_sync(kAll, x1, 1);
+    if ((lane & 1) == 0) reinterpret_cast<float *>(buf[warp])[lane >> 1] = x1;
+    __syncthreads();
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+        const float4 a = buf[0][q4], b = buf[1][q4], c2 = buf[2][q4], d = buf[3][q4];
+        out[4 * q4 + 0] = (a.x + b.x) + (c2.x + d.x);
+        out[4 * q4 + 1] = (a.y + b.y) + (c2.y + d.y);
+        out[4 * q4 + 2] = (a.z + b.z) + (c2.z + d.z);
+        out[4 * q4 + 3] = (a.w + b.w) + (c2.w + d.w);
+    }
+}
+
+// x[idx] for a thread-dependent idx < 16, without local memory.
+__device__ __forceinline__ float pick(const float (&x)[kCols], int idx) {
+    float r = 0.f;
+#pragma unroll
+    for (int j = 0; j < kCols; ++j) r = idx == j ? x[j] : r;
+    return r;
+}
+
+// (sequence, head, slice) of this block; slices of one head are adjacent in the grid.
+struct Unit {
+    int s, h, sl, c0;
+    int64_t cs, ce, base;
+};
+__device__ __forceinline__ Unit unit_of(const BwdArgs &a) {
+    Unit u;
+    u.sl = int(blockIdx.x % unsigned(a.nsl));
+    const int64_t sh = blockIdx.x / unsigned(a.nsl);
+    u.h = int(sh % a.H);
+    u.s = int(sh / a.H);
+    u.c0 = u.sl * kCols;
+    u.cs = a.cu_seqlens[u.s];
+    u.ce = a.cu_seqlens[u.s + 1];
+    u.base = u.cs / kBlk + u.s;
+    return u;
+}
+
+// checkpoint slice of block `blk` (relative to the sequence) of unit u
+__device__ __forceinline__ float4 *ck_slice(const BwdArgs &a, const Unit &u, int64_t blk) {
+    return a.ck + (((u.base + blk) * a.H + u.h) * a.nsl + u.sl) * (4 * kRows);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRows) bwd_states_kernel(const BwdArgs a) {
+    __shared__ float4 red[2][4][4];
+    __shared__ float vs[kBlk][kCols];
+    __shared__ float bs[kBlk];
+    const Unit u = unit_of(a);
+    const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+    const int H = a.H, dk = a.dk, dv = a.dv, dvp = a.nsl * kCols;
+    const bool row = i < dk;
+    const T *kp = static_cast<const T *>(a.k);
+    const T *vp = static_cast<const T *>(a.v);
+
+    float S[kCols];
+#pragma unroll
+    for (int j = 0; j < kCols; ++j)
+        S[j] = (a.S0 && row && u.c0 + j < dv) ? a.S0[((int64_t(u.s) * H + u.h) * dk + i) * dv + u.c0 + j] : 0.f;
+    int rp = 0;
+    for (int64_t tb = u.cs; tb < u.ce; tb += kBlk) {
+        const int n = int(min(int64_t(kBlk), u.ce - tb));
+        float4 *ckp = ck_slice(a, u, (tb - u.cs) / kBlk);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4)
+            ckp[q4 * kRows + i] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
+        __syncthreads();  // the previous block's reads of vs and bs are done
+        for (int e = i; e < kBlk * kCols; e += kRows) {
+            const int tt = e / kCols, j = e % kCols;
+            vs[tt][j] = (tt < n && u.c0 + j < dv) ? ldf(vp + ((tb + tt) * H + u.h) * dv + u.c0 + j) : 0.f;
+        }
+        if (i < kBlk) bs[i] = i < n ? a.beta[(tb + i) * H + u.h] : 0.f;
+        __syncthreads();
+        for (int tt = 0; tt < n; ++tt) {
+            const int64_t t = tb + tt, r = (t * H + u.h) * dk + i;
+            const float al = row ? expf(a.log_alpha[r]) : 1.f;
+            const float kk = row ? ldf(kp + r) : 0.f;
+            float c[kCols], ps[kCols];
+#pragma unroll
+            for (int j = 0; j < kCols; ++j) {
+                S[j] *= al;
+                c[j] = S[j] * kk;
+            }
+            column_sums(c, red[rp], warp, lane, ps);  // ps = P_t^T k_t over this slice
+            rp ^= 1;
+            const float b = bs[tt];
+            float wv[kCols];
+#pragma unroll
+            for (int j = 0; j < kCols; ++j) {
+                wv[j] = vs[tt][j] - ps[j];
+                S[j] = fmaf(kk, b * wv[j], S[j]);
+            }
+            if (i < kCols) a.w[(t * H + u.h) * dvp + u.c0 + i] = pick(wv, i);
+        }
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kRows, 4) bwd_grads_kernel(const BwdArgs a) {
+    __shared__ float4 hist[kSub][4][kRows];  // input states of the sub-block's tokens (own rows)
+    __shared__ float4 red[2][4][4];
+    __shared__ float ws[kBlk][kCols], dos[kBlk][kCols];
+    __shared__ float bs[kBlk];
+    const Unit u = unit_of(a);
+    const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+    const int H = a.H, dk = a.dk, dv = a.dv, dvp = a.nsl * kCols;
+    const int64_t nT = a.T;
+    const bool row = i < dk;
+    const T *qp = static_cast<const T *>(a.q);
+    const T *kp = static_cast<const T *>(a.k);
+    const T *dop = static_cast<const T *>(a.dO);
+
+    float G[kCols];  // dL/dS of the current token's output state, this row and slice
+#pragma unroll
+    for (int j = 0; j < kCols; ++j)
+        G[j] = (a.dS_final && row && u.c0 + j < dv) ? a.dS_final[((int64_t(u.s) * H + u.h) * dk + i) * dv + u.c0 + j]
+                                                     : 0.f;
+    int rp = 0;
+    const int64_t nb = (u.ce - u.cs + kBlk - 1) / kBlk;
+    for (int64_t bi = nb - 1; bi >= 0; --bi) {
+        const int64_t t0 = u.cs + bi * kBlk;
+        const int n = int(min(int64_t(kBlk), u.ce - t0));
+        __syncthreads();  // the previous block's reads of ws, dos and bs are done
+        for (int e = i; e < kBlk * kCols; e += kRows) {
+            const int tt = e / kCols, j = e % kCols;
+            const bool in = tt < n;
+            ws[tt][j] = in ? a.w[((t0 + tt) * H + u.h) * dvp + u.c0 + j] : 0.f;
+            dos[tt][j] = (in && u.c0 + j < dv) ? ldf(dop + ((t0 + tt) * H + u.h) * dv + u.c0 + j) : 0.f;
+        }
+        if (i < kBlk) bs[i] = i < n ? a.beta[(t0 + i) * H + u.h] : 0.f;
+        __syncthreads();
+        const float4 *ckp = ck_slice(a, u, bi);
+        const int nsb = (n + kSub - 1) / kSub;
+        for (int sb = nsb - 1; sb >= 0; --sb) {
+            // replay from the checkpoint to the sub-block's first token, then record the
+            // input state of each of its tokens (each thread touches only its own row)
+            float S[kCols];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 x = ckp[q4 * kRows + i];
+                S[4 * q4] = x.x, S[4 * q4 + 1] = x.y, S[4 * q4 + 2] = x.z, S[4 * q4 + 3] = x.w;
+            }
+            const int first = sb * kSub, m_n = min(kSub, n - first);
+            for (int tt = 0; tt < first + m_n - 1; ++tt) {
+                if (tt >= first) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        hist[tt - first][q4][i] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
+                }
+                const int64_t r = ((t0 + tt) * H + u.h) * dk + i;
+                const float al = row ? expf(a.log_alpha[r]) : 1.f;
+                const float kb = row ? ldf(kp + r) * bs[tt] : 0.f;
+#pragma unroll
+                for (int j = 0; j < kCols; ++j) S[j] = fmaf(kb, ws[tt][j], al * S[j]);
+            }
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+                hist[m_n - 1][q4][i] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
+
+            for (int m = m_n - 1; m >= 0; --m) {
+                const int tt = first + m;
+                const int64_t t = t0 + tt, r = (t * H + u.h) * dk + i;
+                const float al = row ? expf(a.log_alpha[r]) : 1.f;
+                const float kk = row ? ldf(kp + r) : 0.f;
+                const float qq = row ? ldf(qp + r) : 0.f;
+                const float b = bs[tt];
+                float P[kCols], c[kCols];
+                float pq = 0.f, dka = 0.f;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 x = hist[m][q4][i];
+                    P[4 * q4] = al * x.x, P[4 * q4 + 1] = al * x.y, P[4 * q4 + 2] = al * x.z, P[4 * q4 + 3] = al * x.w;
+                }
+#pragma unroll
+                for (int j = 0; j < kCols; ++j) {
+                    const float e = b * ws[tt][j], d = dos[tt][j];
+                    G[j] = fmaf(qq, d, G[j]);
+                    pq = fmaf(fmaf(kk, e, P[j]), d, pq);  // (S_t do_t)_i
+                    dka = fmaf(G[j], e, dka);
+                    c[j] = G[j] * kk;
+                }
+                float de[kCols];
+                column_sums(c, red[rp], warp, lane, de);  // de = G^T k_t over this slice
+                rp ^= 1;
+                float db = 0.f, dkb = 0.f, dg = 0.f;
+#pragma unroll
+                for (int j = 0; j < kCols; ++j) {
+                    db = fmaf(de[j], ws[tt][j], db);
+                    const float du = -b * de[j];
+                    const float dP = fmaf(kk, du, G[j]);
+                    dkb = fmaf(P[j], du, dkb);
+                    dg = fmaf(dP, P[j], dg);
+                    G[j] = al * dP;
+                }
+                if (i < kCols && u.c0 + i < dv) a.dv_out[(t * H + u.h) * dv + u.c0 + i] = b * pick(de, i);
+                const int64_t pr = ((int64_t(u.sl) * nT + t) * H + u.h) * dk + i;
+                if (row) {
+                    a.pq[pr] = pq;
+                    a.pk[pr] = dka + dkb;
+                    a.pg[pr] = dg;
+                }
+                if (i == 0) a.pb[(int64_t(u.sl) * nT + t) * H + u.h] = db;
+            }
+        }
+    }
+    if (a.dS0 && row) {
+#pragma unroll
+        for (int j = 0; j < kCols; ++j)
+            if (u.c0 + j < dv) a.dS0[((int64_t(u.s) * H + u.h) * dk + i) * dv + u.c0 + j] = G[j];
+    }
+}
+
+__global__ void __launch_bounds__(256) bwd_reduce_kernel(const BwdArgs a) {
+    const int64_t n = a.T * a.H * a.dk, nb = a.T * a.H;
+    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
+        float sq = 0.f, sk = 0.f, sg = 0.f;
+        for (int sl = 0; sl < a.nsl; ++sl) {
+            sq += a.pq[sl * n + e];
+            sk += a.pk[sl * n + e];
+            sg += a.pg[sl * n + e];
+        }
+        a.dq[e] = sq;
+        a.dk_out[e] = sk;
+        a.dla[e] = sg;
+        if (e < nb) {
+            float sb = 0.f;
+            for (int sl = 0; sl < a.nsl; ++sl) sb += a.pb[sl * nb + e];
+            a.dbeta[e] = sb;
+        }
+    }
+}
+
+template <typename T>
+cudaError_t launch_backward_t(const BwdArgs &a, cudaStream_t st) {
+    const unsigned grid = unsigned(int64_t(a.num_seqs) * a.H * a.nsl);
+    bwd_states_kernel<T><<<grid, kRows, 0, st>>>(a);
+    bwd_grads_kernel<T><<<grid, kRows, 0, st>>>(a);
+    if (a.T > 0) {
+        const int64_t n = a.T * a.H * a.dk;
+        const unsigned rg = unsigned(std::min<int64_t>((n + 255) / 256, 148 * 16));
+        bwd_reduce_kernel<<<rg, 256, 0, st>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t kda_backward_workspace_size(int num_seqs, int64_t total_tokens, int H, int d_k, int d_v) {
+    if (num_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX || H < 1 || d_k < 1 || d_k > 128 || d_v < 1 ||
+        d_v > 128)
+        return 0;
+    return bwd_layout(num_seqs, total_tokens, H, d_k, d_v).total;
+}
+
+kda_status_t kda_backward(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype, const float *log_alpha,
+                          const float *beta, const float *S0, const int32_t *cu_seqlens_dev,
+                          const int32_t *cu_seqlens_host, int num_seqs, int H, int d_k, int d_v, const void *dO,
+                          const float *dS_final, float *dq, float *dk, float *dv, float *dlog_alpha, float *dbeta,
+                          float *dS0, void *workspace, size_t workspace_bytes, kda_stream_t stream) {
+    if (num_seqs < 0 || H < 1 || d_k < 1 || d_v < 1) return KDA_ERR_INVALID_ARG;
+    if (qkv_dtype != KDA_DTYPE_F32 && qkv_dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
+    if (d_k > 128 || d_v > 128) return KDA_ERR_UNSUPPORTED;
+    if (!cu_seqlens_host || !cu_seqlens_dev) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens_host[0] != 0) return KDA_ERR_INVALID_ARG;
+    for (int n = 0; n < num_seqs; ++n)
+        if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return KDA_ERR_INVALID_ARG;
+    const int64_t T = cu_seqlens_host[num_seqs];
+    if (T > 0 && (!q || !k || !v || !log_alpha || !beta || !dO || !dq || !dk || !dv || !dlog_alpha || !dbeta))
+        return KDA_ERR_INVALID_ARG;
+    const BwdLayout L = bwd_layout(num_seqs, T, H, d_k, d_v);
+    if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return KDA_ERR_WORKSPACE;
+    if (num_seqs == 0) return KDA_OK;
+
+    BwdArgs a;
+    a.q = q; a.k = k; a.v = v; a.dO = dO;
+    a.log_alpha = log_alpha; a.beta = beta; a.S0 = S0; a.dS_final = dS_final;
+    a.cu_seqlens = cu_seqlens_dev;
+    a.num_seqs = num_seqs; a.H = H; a.dk = d_k; a.dv = d_v; a.nsl = (d_v + kCols - 1) / kCols;
+    a.T = T;
+    a.dq = dq; a.dk_out = dk; a.dv_out = dv; a.dla = dlog_alpha; a.dbeta = dbeta; a.dS0 = dS0;
+    char *base = static_cast<char *>(workspace);
+    a.ck = reinterpret_cast<float4 *>(base + L.ck_offset);
+    a.w = reinterpret_cast<float *>(base + L.w_offset);
+    a.pq = reinterpret_cast<float *>(base + L.p_offset);
+    a.pk = reinterpret_cast<float *>(base + L.p_offset + L.p_bytes);
+    a.pg = reinterpret_cast<float *>(base + L.p_offset + 2 * L.p_bytes);
+    a.pb = reinterpret_cast<float *>(base + L.pb_offset);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const cudaError_t e = qkv_dtype == KDA_DTYPE_F32 ? launch_backward_t<float>(a, st)
+                                                     : launch_backward_t<__nv_bfloat16>(a, st);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -155,6 +155,18 @@ def gate_inputs(T, H, dv, dtype="bf16", seed=0, device="cpu"):
     return gate, weight
 
 
+def grad_inputs(T, N, H, dk, dv, dtype="bf16", seed=0, device="cpu", ds_std=0.1):
+    """Synthetic incoming gradients of the backward pass: dO [T,H,dv] (dtype,
+    ~ N(0, 1)) and dS_final [N,H,dk,dv] (float32, ~ ds_std N(0, 1); None when
+    ds_std == 0).  No loss exists here; these stand in for its gradients."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    f32 = dict(dtype=torch.float32, device=device, generator=gen)
+    dO = torch.randn(T, H, dv, **f32).to(torch_dtype(dtype))
+    dS = ds_std * torch.randn(N, H, dk, dv, **f32) if ds_std > 0 else None
+    return dO, dS
+
+
 def prologue_inputs(seqlens, H, dk, dv, dtype="bf16", width=4, seed=0, device="cpu"):
     """Synthetic inputs of the input prologue, packed like ``prefill_inputs``.
 

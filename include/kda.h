@@ -267,6 +267,52 @@ KDA_API kda_status_t kda_decode_tokens(const void *q, const void *k, const void 
 KDA_API kda_status_t kda_workspace_status(const void *workspace, kda_stream_t stream);
 
 /*
+ * kda_backward_workspace_size -- bytes of device workspace kda_backward needs for
+ * these sizes (0 when they are unsupported).  About
+ *   (T/32 + N + 1) * H * ceil(d_v/16) * 8 KiB      state checkpoints
+ *   + T * H * 64 * ceil(d_v/16)                    per-token residuals w_t
+ *   + T * H * ceil(d_v/16) * (12 d_k + 4)          per-slice partial sums
+ * (plus 256 bytes and rounding), e.g. 7.8 GB for T = 16384, H = 32, d = 128.
+ */
+KDA_API size_t kda_backward_workspace_size(int num_seqs, int64_t total_tokens, int H, int d_k, int d_v);
+
+/*
+ * kda_backward -- gradients of the KDA recurrence (training).
+ *
+ * The forward map is kda_prefill's (the state-update equation of the wiki page
+ * "Kimi Linear 高效注意力架构", section "关键技术方法 > Kimi Delta Attention (KDA)",
+ * with o_t = S_t^T q_t read from the post-update state).  Given dO = dL/do_t for
+ * every token and dS_final = dL/dS_final, this returns the exact gradients of L
+ * through the recurrence:
+ *
+ *   dq, dk       [T, H, d_k] float32      dlog_alpha [T, H, d_k] float32
+ *   dv           [T, H, d_v] float32      dbeta      [T, H]      float32
+ *   dS0          [N, H, d_k, d_v] float32, or NULL when not wanted
+ *
+ * Inputs are kda_prefill's (q, k, v of qkv_dtype; log_alpha, beta, S0 float32;
+ * S0 NULL = zeros; the same cu_seqlens on the device and the host), plus
+ *   dO        [T, H, d_v] of qkv_dtype
+ *   dS_final  [N, H, d_k, d_v] float32, or NULL for zeros; may alias dS0
+ * All arithmetic is float32 on CUDA cores; the forward states are recomputed
+ * inside the call (no forward output is needed).  Every output element is
+ * written (gradients of empty sequences' tokens do not exist; dS0 of an empty
+ * sequence is dS_final).
+ *
+ * Supported: 1 <= d_k, d_v <= 128, float32 or bfloat16 q/k/v/dO; no alignment
+ * beyond each type's own.  Workspace: kda_backward_workspace_size bytes,
+ * 256-byte aligned (KDA_ERR_WORKSPACE otherwise).  Launches three kernels on
+ * `stream`, asynchronously; the workspace and outputs must not be touched until
+ * they finish.  Argument errors are reported before anything is queued.
+ */
+KDA_API kda_status_t kda_backward(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
+                                  const float *log_alpha, const float *beta, const float *S0,
+                                  const int32_t *cu_seqlens_dev, const int32_t *cu_seqlens_host,
+                                  int num_seqs, int H, int d_k, int d_v, const void *dO,
+                                  const float *dS_final, float *dq, float *dk, float *dv,
+                                  float *dlog_alpha, float *dbeta, float *dS0, void *workspace,
+                                  size_t workspace_bytes, kda_stream_t stream);
+
+/*
  * kda_wait_timeout_selftest -- checks, on the caller's device, the error path that
  * every bounded wait inside the prefill kernels takes when the event it waits for
  * never comes.  One small kernel (1 block, 64 threads) waits on an mbarrier phase

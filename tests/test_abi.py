@@ -29,7 +29,7 @@ def declared_symbols():
 
 def test_header_declares_the_abi():
     assert declared_symbols() == sorted([
-        "kda_decode_step", "kda_decode_tokens", "kda_prefill", "kda_prefill_gated", "kda_prefill_noalloc", "kda_prologue",
+        "kda_backward", "kda_backward_workspace_size", "kda_decode_step", "kda_decode_tokens", "kda_prefill", "kda_prefill_gated", "kda_prefill_noalloc", "kda_prologue",
         "kda_prefill_workspace_size", "kda_status_string", "kda_version", "kda_wait_timeout_selftest",
         "kda_workspace_status"])
 
@@ -168,6 +168,41 @@ def test_decode_tokens_rejects_bad_arguments(lib):
     assert f(*args(n=0)) == 0 and f(*args(B=0)) == 0
 
 
+def test_backward_workspace_size(lib):
+    ws = lib.kda_backward_workspace_size
+    n = ws(2, 16384, 32, 128, 128)
+    # checkpoints (16384/32 + 3 blocks x 32 heads x 8 slices x 8 KiB) + w (16384 x 32 x 128 x 4)
+    # + 3 partial arrays (8 x 16384 x 32 x 128 x 4) + dbeta partials (8 x 16384 x 32 x 4) + status
+    assert n == 256 + 515 * 32 * 8 * 8192 + 16384 * 32 * 128 * 4 + 3 * 8 * 16384 * 32 * 128 * 4 + 8 * 16384 * 32 * 4
+    assert ws(1, 10, 1, 7, 5) > 256
+    assert ws(1, 10, 1, 129, 5) == 0 and ws(1, 10, 1, 7, 129) == 0
+    assert ws(-1, 10, 1, 7, 5) == 0 and ws(1, -1, 1, 7, 5) == 0 and ws(1, 10, 0, 7, 5) == 0
+    assert ws(1, 1 << 40, 1, 7, 5) == 0
+
+
+def _backward(lib, cu, N, dtype=1, H=2, dk=128, dv=128, ws_bytes=None, **kw):
+    arr = (ctypes.c_int32 * len(cu))(*cu)
+    ws = lib.kda_backward_workspace_size(N, cu[-1] if cu else 0, H, dk, dv) if ws_bytes is None else ws_bytes
+    ptr = [kw.get(n, FAKE) for n in ("q", "k", "v")]
+    return lib.kda_backward(*ptr, dtype, FAKE, FAKE, None, FAKE, arr, N, H, dk, dv, kw.get("dO", FAKE), None,
+                            FAKE, FAKE, FAKE, FAKE, FAKE, None, kw.get("ws", FAKE), ws, None)
+
+
+def test_backward_rejects_bad_arguments(lib):
+    assert _backward(lib, [0, 4], 1, dtype=3) == INVALID
+    assert _backward(lib, [0, 4], 1, H=0) == INVALID
+    assert _backward(lib, [0, 4], 1, dk=129) == UNSUPPORTED
+    assert _backward(lib, [0, 4], 1, dv=129) == UNSUPPORTED
+    assert _backward(lib, [1, 4], 1) == INVALID                 # cu_seqlens[0] != 0
+    assert _backward(lib, [0, 4, 2], 2) == INVALID              # decreasing offsets
+    assert _backward(lib, [0, 4], 1, q=None) == INVALID
+    assert _backward(lib, [0, 4], 1, dO=None) == INVALID
+    assert _backward(lib, [0, 4], 1, ws=None) == WORKSPACE
+    assert _backward(lib, [0, 4], 1, ws_bytes=256) == WORKSPACE
+    assert _backward(lib, [0, 4], 1, ws=ctypes.c_void_p((1 << 20) + 16)) == WORKSPACE
+    assert _backward(lib, [0], 0) == 0                          # no sequences: nothing to do
+
+
 def test_wait_timeout_selftest_rejects_bad_arguments(lib):
     f = lib.kda_wait_timeout_selftest
     assert f(None, 256, 1000, None) == WORKSPACE
@@ -194,3 +229,4 @@ def test_valid_call_without_gpu_reports_cuda_error(lib):
     assert _gated(lib, [0, 4], 1) == 4
     assert _gated(lib, [0, 4], 1, dtype=0, dk=16, dv=16, chunk=16) == 4
     assert _prologue(lib, [0, 4], 1) == 4
+    assert _backward(lib, [0, 4], 1) == 4

@@ -76,7 +76,7 @@ def test_long_sequence_crosses_checkpoints():
 
 def test_linear_attention_special_case():
     # alpha = 1, beta = 0: o_t = S0^T q_t, so dq_t = S0 do_t and dS0 = sum_t q_t do_t^T + dS_final;
-    # nothing flows to v
+    # nothing flows to v or k
     c = _case(4, lens=(6,), H=1)
     c["la"][:] = 0.0
     c["b"][:] = 0.0
@@ -85,6 +85,13 @@ def test_linear_attention_special_case():
     assert np.allclose(g["dq"][:, 0], c["dO"][:, 0] @ S0.T, rtol=1e-12)
     assert np.allclose(g["dS0"][0, 0], c["q"][:, 0].T @ c["dO"][:, 0] + c["dS"][0, 0], rtol=1e-12)
     assert np.array_equal(g["dv"], np.zeros_like(g["dv"]))
+    assert np.array_equal(g["dk"], np.zeros_like(g["dk"]))
+    # G_t = dS_final + sum_{tau >= t} q_tau do_tau^T is the gradient of the (unmoving) state
+    # after token t; beta_t scales k_t (v_t - S0^T k_t)^T and log alpha_t scales S0's rows
+    q, k, v, do = c["q"][:, 0], c["k"][:, 0], c["v"][:, 0], c["dO"][:, 0]
+    G = np.cumsum((q[:, :, None] * do[:, None, :])[::-1], axis=0)[::-1] + c["dS"][0, 0]
+    assert np.allclose(g["dbeta"][:, 0], np.einsum("ti,tij,tj->t", k, G, v - k @ S0), rtol=1e-12)
+    assert np.allclose(g["dlog_alpha"][:, 0], np.einsum("tij,ij->ti", G, S0), rtol=1e-12)
 
 
 @pytest.mark.parametrize("T,chunk", [(37, 8), (64, 16), (5, 8), (130, 64)])
