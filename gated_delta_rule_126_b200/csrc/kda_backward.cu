@@ -22,10 +22,12 @@
 //
 // Three launches:
 //   1. states: the forward sweep, storing w_t for every token and the state before
-//      every 32nd token of each sequence (checkpoints);
+//      every 32nd token of each sequence (checkpoints); each 32-token block's alpha
+//      and k rows are staged in shared memory first;
 //   2. grads:  the backward sweep, 32-token blocks from the last: the 4-token
-//      sub-blocks (last first) are replayed from the block's checkpoint with the
-//      stored w (no reduction needed), their input states kept in shared memory;
+//      sub-blocks (last first) are replayed with the stored w (no reduction needed)
+//      from the block's checkpoint or, past the middle, from the state before the
+//      block's 16th token, their input states kept in shared memory;
 //   3. reduce: sums the slices' partial dq, dk, dlog_alpha and dbeta.
 // CUDA cores in fp32 throughout; no tensor cores and no waits on other blocks.
 #include <algorithm>
@@ -39,6 +41,7 @@ constexpr int kCols = 16;  // value columns per slice
 constexpr int kRows = 128; // threads per block = key rows
 constexpr int kBlk = 32;   // tokens between checkpoints
 constexpr int kSub = 4;    // tokens per replayed sub-block
+constexpr int kMid = kBlk / 2;
 
 struct BwdArgs {
     const void *q, *k, *v, *dO;
@@ -145,6 +148,7 @@ __global__ void __launch_bounds__(kRows) bwd_states_kernel(const BwdArgs a) {
     __shared__ float4 red[2][4][4];
     __shared__ float vs[kBlk][kCols];
     __shared__ float bs[kBlk];
+    __shared__ float al_s[kBlk][kRows], k_s[kBlk][kRows];
     const Unit u = unit_of(a);
     const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
     const int H = a.H, dk = a.dk, dv = a.dv, dvp = a.nsl * kCols;
@@ -169,11 +173,23 @@ __global__ void __launch_bounds__(kRows) bwd_states_kernel(const BwdArgs a) {
             vs[tt][j] = (tt < n && u.c0 + j < dv) ? ldf(vp + ((tb + tt) * H + u.h) * dv + u.c0 + j) : 0.f;
         }
         if (i < kBlk) bs[i] = i < n ? a.beta[(tb + i) * H + u.h] : 0.f;
+        for (int t8 = 0; t8 < kBlk; t8 += 8) {  // this row's alpha and k, eight tokens' loads at a time
+            float la[8], kx[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const bool in = row && t8 + j < n;
+                const int64_t r = ((tb + t8 + j) * H + u.h) * dk + i;
+                la[j] = in ? a.log_alpha[r] : 0.f;
+                kx[j] = in ? ldf(kp + r) : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) al_s[t8 + j][i] = expf(la[j]), k_s[t8 + j][i] = kx[j];
+        }
         __syncthreads();
         for (int tt = 0; tt < n; ++tt) {
-            const int64_t t = tb + tt, r = (t * H + u.h) * dk + i;
-            const float al = row ? expf(a.log_alpha[r]) : 1.f;
-            const float kk = row ? ldf(kp + r) : 0.f;
+            const int64_t t = tb + tt;
+            const float al = al_s[tt][i];
+            const float kk = k_s[tt][i];
             float c[kCols], ps[kCols];
 #pragma unroll
             for (int j = 0; j < kCols; ++j) {
@@ -197,6 +213,7 @@ __global__ void __launch_bounds__(kRows) bwd_states_kernel(const BwdArgs a) {
 template <typename T>
 __global__ void __launch_bounds__(kRows, 4) bwd_grads_kernel(const BwdArgs a) {
     __shared__ float4 hist[kSub][4][kRows];  // input states of the sub-block's tokens (own rows)
+    __shared__ float4 midst[4][kRows];       // state before the block's middle token (own rows)
     __shared__ float4 red[2][4][4];
     __shared__ float ws[kBlk][kCols], dos[kBlk][kCols];
     __shared__ float bs[kBlk];
@@ -229,18 +246,42 @@ __global__ void __launch_bounds__(kRows, 4) bwd_grads_kernel(const BwdArgs a) {
         if (i < kBlk) bs[i] = i < n ? a.beta[(t0 + i) * H + u.h] : 0.f;
         __syncthreads();
         const float4 *ckp = ck_slice(a, u, bi);
-        const int nsb = (n + kSub - 1) / kSub;
-        for (int sb = nsb - 1; sb >= 0; --sb) {
-            // replay from the checkpoint to the sub-block's first token, then record the
-            // input state of each of its tokens (each thread touches only its own row)
+        // S <- Diag(alpha_tt) S + beta_tt k_tt w_tt^T, from the stored w
+        auto replay = [&](float(&S)[kCols], int tt) {
+            const int64_t r = ((t0 + tt) * H + u.h) * dk + i;
+            const float al = row ? expf(a.log_alpha[r]) : 1.f;
+            const float kb = row ? ldf(kp + r) * bs[tt] : 0.f;
+#pragma unroll
+            for (int j = 0; j < kCols; ++j) S[j] = fmaf(kb, ws[tt][j], al * S[j]);
+        };
+        if (n > kMid) {  // the state before the block's middle token, for the later sub-blocks
             float S[kCols];
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) {
                 const float4 x = ckp[q4 * kRows + i];
                 S[4 * q4] = x.x, S[4 * q4 + 1] = x.y, S[4 * q4 + 2] = x.z, S[4 * q4 + 3] = x.w;
             }
+            for (int tt = 0; tt < kMid; ++tt) replay(S, tt);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) midst[q4][i] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
+        }
+        const int nsb = (n + kSub - 1) / kSub;
+        for (int sb = nsb - 1; sb >= 0; --sb) {
+            // replay from the nearest checkpoint to the sub-block's first token, then record
+            // the input state of each of its tokens (each thread touches only its own row)
             const int first = sb * kSub, m_n = min(kSub, n - first);
-            for (int tt = 0; tt < first + m_n - 1; ++tt) {
+            const int from = first >= kMid ? kMid : 0;
+            float qpre[kSub];
+#pragma unroll
+            for (int m = 0; m < kSub; ++m)
+                qpre[m] = (row && m < m_n) ? ldf(qp + ((t0 + first + m) * H + u.h) * dk + i) : 0.f;
+            float S[kCols];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+                const float4 x = from ? midst[q4][i] : ckp[q4 * kRows + i];
+                S[4 * q4] = x.x, S[4 * q4 + 1] = x.y, S[4 * q4 + 2] = x.z, S[4 * q4 + 3] = x.w;
+            }
+            for (int tt = from; tt < first + m_n - 1; ++tt) {
                 if (tt >= first) {
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4)
@@ -256,12 +297,14 @@ __global__ void __launch_bounds__(kRows, 4) bwd_grads_kernel(const BwdArgs a) {
             for (int q4 = 0; q4 < 4; ++q4)
                 hist[m_n - 1][q4][i] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
 
-            for (int m = m_n - 1; m >= 0; --m) {
+#pragma unroll
+            for (int m = kSub - 1; m >= 0; --m) {
+                if (m >= m_n) continue;
                 const int tt = first + m;
                 const int64_t t = t0 + tt, r = (t * H + u.h) * dk + i;
                 const float al = row ? expf(a.log_alpha[r]) : 1.f;
                 const float kk = row ? ldf(kp + r) : 0.f;
-                const float qq = row ? ldf(qp + r) : 0.f;
+                const float qq = qpre[m];
                 const float b = bs[tt];
                 float P[kCols], c[kCols];
                 float pq = 0.f, dka = 0.f;

@@ -84,6 +84,11 @@ WORKLOADS = {
     "batched_prefill_2x8192": Workload("batched_prefill_2x8192", "prefill", H=32, dk=128, dv=128,
                                        dtype="bf16", s0_std=0.0, seed=SEED_BASE + 2, chunk=64,
                                        seqlens=(8192,) * 2),
+    # the backward pass's profiler case: 4 x 2048 tokens, 32 heads (inputs above L2,
+    # about 4 GB of backward workspace)
+    "batched_prefill_4x2048": Workload("batched_prefill_4x2048", "prefill", H=32, dk=128, dv=128,
+                                       dtype="bf16", s0_std=0.0, seed=SEED_BASE + 2, chunk=64,
+                                       seqlens=(2048,) * 4),
     "decode": Workload("decode", "decode", H=32, dk=128, dv=128, dtype="bf16",
                        s0_std=S0_STD, seed=SEED_BASE + 3, batch=256, steps=64),
     "longctx_varlen_prefill": Workload("longctx_varlen_prefill", "prefill", H=32, dk=128,
