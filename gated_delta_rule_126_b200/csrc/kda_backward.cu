@@ -261,6 +261,7 @@ __global__ void __launch_bounds__(kRows, 4) bwd_grads_kernel(const BwdArgs a) {
                 const float4 x = ckp[q4 * kRows + i];
                 S[4 * q4] = x.x, S[4 * q4 + 1] = x.y, S[4 * q4 + 2] = x.z, S[4 * q4 + 3] = x.w;
             }
+#pragma unroll 4
             for (int tt = 0; tt < kMid; ++tt) replay(S, tt);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4) midst[q4][i] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
@@ -281,6 +282,7 @@ __global__ void __launch_bounds__(kRows, 4) bwd_grads_kernel(const BwdArgs a) {
                 const float4 x = from ? midst[q4][i] : ckp[q4 * kRows + i];
                 S[4 * q4] = x.x, S[4 * q4 + 1] = x.y, S[4 * q4 + 2] = x.z, S[4 * q4 + 3] = x.w;
             }
+#pragma unroll 4
             for (int tt = from; tt < first + m_n - 1; ++tt) {
                 if (tt >= first) {
 #pragma unroll
