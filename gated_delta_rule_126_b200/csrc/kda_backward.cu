@@ -406,6 +406,7 @@ kda_status_t kda_backward(const void *q, const void *k, const void *v, kda_dtype
     if (num_seqs < 0 || H < 1 || d_k < 1 || d_v < 1) return KDA_ERR_INVALID_ARG;
     if (qkv_dtype != KDA_DTYPE_F32 && qkv_dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARG;
     if (d_k > 128 || d_v > 128) return KDA_ERR_UNSUPPORTED;
+    if (int64_t(num_seqs) * H * ((d_v + kCols - 1) / kCols) > INT32_MAX) return KDA_ERR_UNSUPPORTED;  // grid size
     if (!cu_seqlens_host || !cu_seqlens_dev) return KDA_ERR_INVALID_ARG;
     if (cu_seqlens_host[0] != 0) return KDA_ERR_INVALID_ARG;
     for (int n = 0; n < num_seqs; ++n)

@@ -298,8 +298,9 @@ KDA_API size_t kda_backward_workspace_size(int num_seqs, int64_t total_tokens, i
  * written (gradients of empty sequences' tokens do not exist; dS0 of an empty
  * sequence is dS_final).
  *
- * Supported: 1 <= d_k, d_v <= 128, float32 or bfloat16 q/k/v/dO; no alignment
- * beyond each type's own.  Workspace: kda_backward_workspace_size bytes,
+ * Supported: 1 <= d_k, d_v <= 128, float32 or bfloat16 q/k/v/dO, num_seqs * H *
+ * ceil(d_v / 16) < 2^31 (KDA_ERR_UNSUPPORTED otherwise); no alignment beyond each
+ * type's own.  Workspace: kda_backward_workspace_size bytes,
  * 256-byte aligned (KDA_ERR_WORKSPACE otherwise).  Launches three kernels on
  * `stream`, asynchronously; the workspace and outputs must not be touched until
  * they finish.  Argument errors are reported before anything is queued.

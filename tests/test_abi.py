@@ -201,6 +201,7 @@ def test_backward_rejects_bad_arguments(lib):
     assert _backward(lib, [0, 4], 1, ws_bytes=256) == WORKSPACE
     assert _backward(lib, [0, 4], 1, ws=ctypes.c_void_p((1 << 20) + 16)) == WORKSPACE
     assert _backward(lib, [0], 0) == 0                          # no sequences: nothing to do
+    assert _backward(lib, [0] * 65537, 65536, H=4096) == UNSUPPORTED  # grid of 2^31 blocks
 
 
 def test_wait_timeout_selftest_rejects_bad_arguments(lib):

@@ -121,3 +121,21 @@ def test_bench_size_sampled_units():
         part = {key: got[key][s:e, h:h + 1] for key in NAMES[:-1]}
         part["dS0"] = got["dS0"][n:n + 1, h:h + 1]
         check_all(part, ref)
+
+
+def test_empty_sequences_pass_the_final_gradient_through():
+    """Empty sequences among non-empty ones: their dS0 is dS_final unchanged, and the
+    non-empty ones match the oracle."""
+    inp, dO, dS = case([0, 5, 0, 40, 0], 2, 32, 24, "f32", seed=11)
+    got = run_gpu(inp, dO, dS)
+    for n in (0, 2, 4):
+        assert torch.equal(got["dS0"][n], dS[n])
+    check_all(got, run_oracle(inp, dO, dS))
+
+
+def test_all_sequences_empty():
+    """T = 0: no token gradients exist; dS0 = dS_final."""
+    inp, dO, dS = case([0, 0], 1, 16, 16, "f32", seed=12)
+    got = run_gpu(inp, dO, dS)
+    assert got["dq"].numel() == 0 and got["dbeta"].numel() == 0
+    assert torch.equal(got["dS0"], dS)
