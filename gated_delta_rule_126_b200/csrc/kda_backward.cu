@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kRows) bwd_states_kernel(const BwdArgs a) {
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4)
             ckp[q4 * kRows + i] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
-        __syncthreads();  // the previous block's reads of vs and bs are done
+        __syncthreads();  // the previous block's reads of the staged rows are done
         for (int e = i; e < kBlk * kCols; e += kRows) {
             const int tt = e / kCols, j = e % kCols;
             vs[tt][j] = (tt < n && u.c0 + j < dv) ? ldf(vp + ((tb + tt) * H + u.h) * dv + u.c0 + j) : 0.f;
