@@ -6,7 +6,8 @@
 //   q = l2norm(swish(conv_q(q_pre))), k likewise, v = swish(conv_v(v_pre))
 //   log_alpha = -rate[h] softplus(a),  beta = sigmoid(b)
 // Each warp walks 32 consecutive tokens of one head, four channels a lane, keeping
-// the convolution's three previous rows in registers; HBM-bound.
+// the convolution's three previous rows in registers and loading rows four tokens
+// ahead (bf16 rows stay packed until used, so this fits in 64 registers); HBM-bound.
 #include <cmath>
 
 #include "kda_internal.h"
@@ -36,6 +37,24 @@ template <> struct Vec4<__nv_bfloat16> {
     }
 };
 
+// Four consecutive elements as loaded (bf16 stays packed until used).
+template <typename T> struct Raw4;
+template <> struct Raw4<float> {
+    using type = float4;
+    static __device__ __forceinline__ float4 load(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+    static __device__ __forceinline__ float4 zero() { return make_float4(0.f, 0.f, 0.f, 0.f); }
+    static __device__ __forceinline__ float4 widen(float4 v) { return v; }
+};
+template <> struct Raw4<__nv_bfloat16> {
+    using type = uint2;
+    static __device__ __forceinline__ uint2 load(const __nv_bfloat16 *p) { return *reinterpret_cast<const uint2 *>(p); }
+    static __device__ __forceinline__ uint2 zero() { return make_uint2(0u, 0u); }
+    static __device__ __forceinline__ float4 widen(uint2 u) {
+        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                           __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+    }
+};
+
 // The CUDA fast intrinsics (a few ulp): the outputs are bf16, or float32 held to 1e-5.
 __device__ __forceinline__ float sigmoid_f(float x) { return __fdividef(1.f, 1.f + __expf(-x)); }
 // max(x, 0) + log(1 + e^{-|x|}): where e^{-|x|} is below fp32's resolution of 1 the
@@ -53,10 +72,13 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 // One projection's sliding window for this lane's four channels: the taps' weights and
-// the three previous rows (x[t - 1], x[t - 2], x[t - 3]; zero before the sequence start).
+// the three previous rows as loaded (x[t - 1], x[t - 2], x[t - 3]; zero before the
+// sequence start).
+template <typename T>
 struct Window {
-    float4 w[4];     // w[tap] = weights of channels c0 .. c0 + 3 at that tap (zero past W)
-    float4 hist[3];
+    using Raw = typename Raw4<T>::type;
+    float4 w[4];  // w[tap] = weights of channels c0 .. c0 + 3 at that tap (zero past W)
+    Raw hist[3];
     __device__ __forceinline__ void load_weights(const float *weight, int W, int h, int d, int c0) {
 #pragma unroll
         for (int tap = 0; tap < 4; ++tap) {
@@ -68,55 +90,65 @@ struct Window {
     }
     __device__ __forceinline__ void clear() {
 #pragma unroll
-        for (int i = 0; i < 3; ++i) hist[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < 3; ++i) hist[i] = Raw4<T>::zero();
     }
     // conv(x)[t] from the current row, then the window moves on by one token
-    __device__ __forceinline__ float4 step(float4 x) {
+    __device__ __forceinline__ float4 step(Raw xr) {
+        const float4 x = Raw4<T>::widen(xr), h0 = Raw4<T>::widen(hist[0]), h1 = Raw4<T>::widen(hist[1]),
+                     h2 = Raw4<T>::widen(hist[2]);
         float4 z;
-        z.x = w[0].x * x.x + w[1].x * hist[0].x + w[2].x * hist[1].x + w[3].x * hist[2].x;
-        z.y = w[0].y * x.y + w[1].y * hist[0].y + w[2].y * hist[1].y + w[3].y * hist[2].y;
-        z.z = w[0].z * x.z + w[1].z * hist[0].z + w[2].z * hist[1].z + w[3].z * hist[2].z;
-        z.w = w[0].w * x.w + w[1].w * hist[0].w + w[2].w * hist[1].w + w[3].w * hist[2].w;
+        z.x = w[0].x * x.x + w[1].x * h0.x + w[2].x * h1.x + w[3].x * h2.x;
+        z.y = w[0].y * x.y + w[1].y * h0.y + w[2].y * h1.y + w[3].y * h2.y;
+        z.z = w[0].z * x.z + w[1].z * h0.z + w[2].z * h1.z + w[3].z * h2.z;
+        z.w = w[0].w * x.w + w[1].w * h0.w + w[2].w * h1.w + w[3].w * h2.w;
         hist[2] = hist[1];
         hist[1] = hist[0];
-        hist[0] = x;
+        hist[0] = xr;
         return z;
     }
 };
 
-constexpr int kRun = 32;  // consecutive tokens of one head per warp
+constexpr int kRun = 32;    // consecutive tokens of one head per warp
+constexpr int kAhead = 4;   // rows loaded ahead of the one in use
 
 // Walks tokens [t0, t_end) of head h for one projection: swish(conv(x)), L2-normalised
-// over the head's d channels when kNorm, stored in out.  seq/next: the sequence of t0.
+// over the head's d channels when kNorm, stored in out.  seq: the sequence of t0.
+// Rows are loaded kAhead tokens ahead into a rotating set of registers.
 template <typename T, bool kNorm>
 __device__ __forceinline__ void run_projection(const PrologueArgs &a, const T *x, const float *weight, int d, T *out,
                                                int h, int64_t t0, int64_t t_end, int seq, int lane) {
+    using Raw = typename Raw4<T>::type;
     const int H = a.H, c0 = 4 * lane;
     const bool on = c0 < d;
     int64_t seq_start = a.cu_seqlens[seq], next = a.cu_seqlens[seq + 1];
-    auto ld = [&](int64_t t) {
-        return on ? Vec4<T>::load(x + (size_t(t) * H + h) * d + c0) : make_float4(0.f, 0.f, 0.f, 0.f);
-    };
-    Window win;
+    auto ld = [&](int64_t t) { return on ? Raw4<T>::load(x + (size_t(t) * H + h) * d + c0) : Raw4<T>::zero(); };
+    Raw ahead[kAhead];
+#pragma unroll
+    for (int k = 0; k < kAhead; ++k) ahead[k] = t0 + k < t_end ? ld(t0 + k) : Raw4<T>::zero();
+    Window<T> win;
     win.load_weights(weight, a.W, h, d, c0);
     win.clear();
     for (int back = 3; back >= 1; --back)  // rows t0 - 3 .. t0 - 1 of the same sequence
         if (t0 - back >= seq_start) win.step(ld(t0 - back));
-    float4 xn = ld(t0);  // this token's row, loaded one token ahead
-    for (int64_t t = t0; t < t_end; ++t) {
-        while (t >= next) {  // a new sequence starts at t (empty sequences are skipped)
-            ++seq;
-            next = a.cu_seqlens[seq + 1];
-            win.clear();
+    for (int64_t tb = t0; tb < t_end; tb += kAhead) {
+#pragma unroll
+        for (int k = 0; k < kAhead; ++k) {
+            const int64_t t = tb + k;
+            if (t >= t_end) break;
+            const Raw cur = ahead[k];
+            if (t + kAhead < t_end) ahead[k] = ld(t + kAhead);
+            while (t >= next) {  // a new sequence starts at t (empty sequences are skipped)
+                ++seq;
+                next = a.cu_seqlens[seq + 1];
+                win.clear();
+            }
+            float4 z = swish4(win.step(cur));
+            if (kNorm) {
+                const float rn = rsqrtf(warp_sum(z.x * z.x + z.y * z.y + z.z * z.z + z.w * z.w) + a.l2_eps);
+                z = make_float4(z.x * rn, z.y * rn, z.z * rn, z.w * rn);
+            }
+            if (on) Vec4<T>::store(out + (size_t(t) * H + h) * d + c0, z);
         }
-        const float4 xc = xn;
-        if (t + 1 < t_end) xn = ld(t + 1);
-        float4 z = swish4(win.step(xc));
-        if (kNorm) {
-            const float rn = rsqrtf(warp_sum(z.x * z.x + z.y * z.y + z.z * z.z + z.w * z.w) + a.l2_eps);
-            z = make_float4(z.x * rn, z.y * rn, z.z * rn, z.w * rn);
-        }
-        if (on) Vec4<T>::store(out + (size_t(t) * H + h) * d + c0, z);
     }
 }
 
@@ -141,11 +173,17 @@ __global__ void __launch_bounds__(32 * kRows, 4) prologue_kernel(const PrologueA
     const float r = -a.rate[h];
     const int c0 = 4 * lane;
     if (c0 < a.dk) {
-        for (int64_t t = t0; t < t_end; ++t) {
-            const size_t off = (size_t(t) * H + h) * a.dk + c0;
-            const float4 g = *reinterpret_cast<const float4 *>(a.a + off);
-            *reinterpret_cast<float4 *>(a.log_alpha + off) =
-                make_float4(r * softplus_f(g.x), r * softplus_f(g.y), r * softplus_f(g.z), r * softplus_f(g.w));
+        for (int64_t tb = t0; tb < t_end; tb += kAhead) {
+            float4 g[kAhead];
+#pragma unroll
+            for (int k = 0; k < kAhead; ++k)
+                if (tb + k < t_end) g[k] = *reinterpret_cast<const float4 *>(a.a + (size_t(tb + k) * H + h) * a.dk + c0);
+#pragma unroll
+            for (int k = 0; k < kAhead; ++k)
+                if (tb + k < t_end)
+                    *reinterpret_cast<float4 *>(a.log_alpha + (size_t(tb + k) * H + h) * a.dk + c0) =
+                        make_float4(r * softplus_f(g[k].x), r * softplus_f(g[k].y), r * softplus_f(g[k].z),
+                                    r * softplus_f(g[k].w));
         }
     }
     if (lane < t_end - t0) {
