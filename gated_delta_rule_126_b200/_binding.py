@@ -109,6 +109,42 @@ def _need(t, name, dtype=None, device=None):
         raise ValueError(f"{name} is on {t.device}, expected {device}")
 
 
+def _dims(t, name, ndim):
+    """Shape of t, which must be a tensor with ndim dimensions."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+    return tuple(t.shape)
+
+
+def _shapes(**named):
+    """Checks name=(tensor or None, expected shape) before any pointer reaches the library:
+    the kernels trust the sizes they are given."""
+    for name, (t, shape) in named.items():
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _offsets(cu_seqlens, cu_seqlens_host, T):
+    """(N, host copy of the offsets); the offsets must end within the T rows given."""
+    if not isinstance(cu_seqlens, torch.Tensor) or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be a 1-D tensor")
+    if cu_seqlens_host is None:
+        cu_seqlens_host = cu_seqlens.cpu()
+    cu_h = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
+    N = cu_h.numel() - 1
+    if N < 0 or cu_seqlens.numel() != N + 1:
+        raise ValueError("cu_seqlens and cu_seqlens_host differ in length")
+    if int(cu_h[-1]) > T:
+        raise ValueError(f"cu_seqlens ends at token {int(cu_h[-1])} but the inputs hold {T} tokens")
+    return N, cu_h
+
+
 def prefill_workspace_size(num_seqs, total_tokens, H, d_k, d_v, chunk=64, dtype=torch.bfloat16):
     return int(load().kda_prefill_workspace_size(int(num_seqs), int(total_tokens), int(H),
                                                  int(d_k), int(d_v), int(chunk),
@@ -125,26 +161,23 @@ def kda_prefill(q, k, v, log_alpha, beta, cu_seqlens, cu_seqlens_host=None, S0=N
     synchronises), S0 [N,H,d_k,d_v] f32 or None.  Returns ``(o, S_final)``.
     """
     lib = load()
+    T, H, dk = _dims(q, "q", 3)
+    dv = _dims(v, "v", 3)[2]
+    N, cu_h = _offsets(cu_seqlens, cu_seqlens_host, T)
+    _shapes(k=(k, (T, H, dk)), v=(v, (T, H, dv)), log_alpha=(log_alpha, (T, H, dk)), beta=(beta, (T, H)),
+            S0=(S0, (N, H, dk, dv)), o=(o, (T, H, dv)), S_final=(S_final, (N, H, dk, dv)))
     dev = q.device
     dt = q.dtype
     if dt not in DTYPE_CODE:
         raise ValueError("q/k/v dtype must be float32 or bfloat16")
     _need(q, "q", dt)
-    T, H, dk = q.shape
     _need(k, "k", dt, dev)
     _need(v, "v", dt, dev)
-    dv = v.shape[2]
     _need(log_alpha, "log_alpha", torch.float32, dev)
     _need(beta, "beta", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
     if S0 is not None:
         _need(S0, "S0", torch.float32, dev)
-    if cu_seqlens_host is None:
-        cu_seqlens_host = cu_seqlens.cpu()
-    cu_h = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
-    N = cu_h.numel() - 1
-    if cu_seqlens.numel() != N + 1:
-        raise ValueError("cu_seqlens and cu_seqlens_host differ in length")
     if o is None:
         o = torch.empty(T, H, dv, dtype=dt, device=dev)
     if S_final is None:
@@ -174,15 +207,19 @@ def kda_prefill_gated(q, k, v, log_alpha, beta, cu_seqlens, gate, norm_weight, e
     eps > 0; returns ``(y, S_final)`` with y = o / sqrt(mean(o^2) + eps) * w * sigmoid(gate).
     """
     lib = load()
+    T, H, dk = _dims(q, "q", 3)
+    dv = _dims(v, "v", 3)[2]
+    N, cu_h = _offsets(cu_seqlens, cu_seqlens_host, T)
+    _shapes(k=(k, (T, H, dk)), v=(v, (T, H, dv)), log_alpha=(log_alpha, (T, H, dk)), beta=(beta, (T, H)),
+            gate=(gate, (T, H, dv)), norm_weight=(norm_weight, (dv,)), S0=(S0, (N, H, dk, dv)),
+            y=(y, (T, H, dv)), S_final=(S_final, (N, H, dk, dv)))
     dev = q.device
     dt = q.dtype
     if dt not in DTYPE_CODE:
         raise ValueError("q/k/v dtype must be float32 or bfloat16")
     _need(q, "q", dt)
-    T, H, dk = q.shape
     _need(k, "k", dt, dev)
     _need(v, "v", dt, dev)
-    dv = v.shape[2]
     _need(log_alpha, "log_alpha", torch.float32, dev)
     _need(beta, "beta", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
@@ -190,12 +227,6 @@ def kda_prefill_gated(q, k, v, log_alpha, beta, cu_seqlens, gate, norm_weight, e
     _need(norm_weight, "norm_weight", torch.float32, dev)
     if S0 is not None:
         _need(S0, "S0", torch.float32, dev)
-    if cu_seqlens_host is None:
-        cu_seqlens_host = cu_seqlens.cpu()
-    cu_h = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
-    N = cu_h.numel() - 1
-    if cu_seqlens.numel() != N + 1:
-        raise ValueError("cu_seqlens and cu_seqlens_host differ in length")
     if y is None:
         y = torch.empty(T, H, dv, dtype=dt, device=dev)
     if S_final is None:
@@ -226,27 +257,28 @@ def kda_prologue(q_pre, k_pre, v_pre, conv_q, conv_k, conv_v, a_gate, rate, b_ga
     log_alpha, beta in kda_prefill's layouts (``out`` may supply them).
     """
     lib = load()
+    T, H, dk = _dims(q_pre, "q_pre", 3)
+    dv = _dims(v_pre, "v_pre", 3)[2]
+    W = _dims(conv_q, "conv_q", 3)[2]
+    N, cu_h = _offsets(cu_seqlens, cu_seqlens_host, T)
+    given = dict(out or {})
+    _shapes(k_pre=(k_pre, (T, H, dk)), v_pre=(v_pre, (T, H, dv)), conv_q=(conv_q, (H, dk, W)),
+            conv_k=(conv_k, (H, dk, W)), conv_v=(conv_v, (H, dv, W)), a_gate=(a_gate, (T, H, dk)),
+            rate=(rate, (H,)), b_gate=(b_gate, (T, H)), q=(given.get("q"), (T, H, dk)),
+            k=(given.get("k"), (T, H, dk)), v=(given.get("v"), (T, H, dv)),
+            log_alpha=(given.get("log_alpha"), (T, H, dk)), beta=(given.get("beta"), (T, H)))
     dev = q_pre.device
     dt = q_pre.dtype
     if dt not in DTYPE_CODE:
         raise ValueError("projection dtype must be float32 or bfloat16")
     _need(q_pre, "q_pre", dt)
-    T, H, dk = q_pre.shape
     _need(k_pre, "k_pre", dt, dev)
     _need(v_pre, "v_pre", dt, dev)
-    dv = v_pre.shape[2]
     for name, t in (("conv_q", conv_q), ("conv_k", conv_k), ("conv_v", conv_v), ("a_gate", a_gate),
                     ("rate", rate), ("b_gate", b_gate)):
         _need(t, name, torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
-    W = conv_q.shape[-1]
-    if conv_k.shape[-1] != W or conv_v.shape[-1] != W:
-        raise ValueError("the three convolutions must have the same width")
-    if cu_seqlens_host is None:
-        cu_seqlens_host = cu_seqlens.cpu()
-    cu_h = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
-    N = cu_h.numel() - 1
-    out = dict(out or {})
+    out = given
     out.setdefault("q", torch.empty(T, H, dk, dtype=dt, device=dev))
     out.setdefault("k", torch.empty(T, H, dk, dtype=dt, device=dev))
     out.setdefault("v", torch.empty(T, H, dv, dtype=dt, device=dev))
@@ -274,15 +306,17 @@ def kda_decode_step(q, k, v, log_alpha, beta, S, o=None, stream=None):
     S [B,H,d_k,d_v] f32 (updated in place).  Returns o [B,H,d_v].
     """
     lib = load()
+    B, H, dk = _dims(q, "q", 3)
+    dv = _dims(v, "v", 3)[2]
+    _shapes(k=(k, (B, H, dk)), v=(v, (B, H, dv)), log_alpha=(log_alpha, (B, H, dk)), beta=(beta, (B, H)),
+            S=(S, (B, H, dk, dv)), o=(o, (B, H, dv)))
     dev = q.device
     dt = q.dtype
     if dt not in DTYPE_CODE:
         raise ValueError("q/k/v dtype must be float32 or bfloat16")
     _need(q, "q", dt)
-    B, H, dk = q.shape
     _need(k, "k", dt, dev)
     _need(v, "v", dt, dev)
-    dv = v.shape[2]
     _need(log_alpha, "log_alpha", torch.float32, dev)
     _need(beta, "beta", torch.float32, dev)
     _need(S, "S", torch.float32, dev)
@@ -305,15 +339,19 @@ def kda_decode_tokens(q, k, v, log_alpha, beta, S_pool, slot_idx=None, o=None, s
     device or None (slot b).  Returns o [B,n,H,d_v].
     """
     lib = load()
+    B, n, H, dk = _dims(q, "q", 4)
+    dv = _dims(v, "v", 4)[3]
+    ns = _dims(S_pool, "S_pool", 4)[0]
+    _shapes(k=(k, (B, n, H, dk)), v=(v, (B, n, H, dv)), log_alpha=(log_alpha, (B, n, H, dk)),
+            beta=(beta, (B, n, H)), S_pool=(S_pool, (ns, H, dk, dv)), slot_idx=(slot_idx, (B,)),
+            o=(o, (B, n, H, dv)))
     dev = q.device
     dt = q.dtype
     if dt not in DTYPE_CODE:
         raise ValueError("q/k/v dtype must be float32 or bfloat16")
     _need(q, "q", dt)
-    B, n, H, dk = q.shape
     _need(k, "k", dt, dev)
     _need(v, "v", dt, dev)
-    dv = v.shape[3]
     _need(log_alpha, "log_alpha", torch.float32, dev)
     _need(beta, "beta", torch.float32, dev)
     _need(S_pool, "S_pool", torch.float32, dev)
@@ -344,28 +382,25 @@ def kda_backward(q, k, v, log_alpha, beta, cu_seqlens, dO, cu_seqlens_host=None,
     dlog_alpha, dbeta and dS0 (None unless ``want_dS0``).
     """
     lib = load()
+    T, H, dk = _dims(q, "q", 3)
+    dv = _dims(v, "v", 3)[2]
+    N, cu_h = _offsets(cu_seqlens, cu_seqlens_host, T)
+    _shapes(k=(k, (T, H, dk)), v=(v, (T, H, dv)), dO=(dO, (T, H, dv)), log_alpha=(log_alpha, (T, H, dk)),
+            beta=(beta, (T, H)), S0=(S0, (N, H, dk, dv)), dS_final=(dS_final, (N, H, dk, dv)))
     dev = q.device
     dt = q.dtype
     if dt not in DTYPE_CODE:
         raise ValueError("q/k/v dtype must be float32 or bfloat16")
     _need(q, "q", dt)
-    T, H, dk = q.shape
     _need(k, "k", dt, dev)
     _need(v, "v", dt, dev)
     _need(dO, "dO", dt, dev)
-    dv = v.shape[2]
     _need(log_alpha, "log_alpha", torch.float32, dev)
     _need(beta, "beta", torch.float32, dev)
     _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
     for t, name in ((S0, "S0"), (dS_final, "dS_final")):
         if t is not None:
             _need(t, name, torch.float32, dev)
-    if cu_seqlens_host is None:
-        cu_seqlens_host = cu_seqlens.cpu()
-    cu_h = torch.as_tensor(cu_seqlens_host, dtype=torch.int32).contiguous()
-    N = cu_h.numel() - 1
-    if cu_seqlens.numel() != N + 1:
-        raise ValueError("cu_seqlens and cu_seqlens_host differ in length")
     f32 = dict(dtype=torch.float32, device=dev)
     out = dict(dq=torch.empty(T, H, dk, **f32), dk=torch.empty(T, H, dk, **f32),
                dv=torch.empty(T, H, dv, **f32), dlog_alpha=torch.empty(T, H, dk, **f32),
