@@ -83,13 +83,26 @@ def measured_traffic(kernel, units):
     return rec["dram_bytes"] * units / rec["units"]
 
 
-def prefill_launches(seqlens, H, tc_path):
+def prefill_launches(seqlens, H, tc_path, sms=148):
     """Kernel launches of one kda_prefill call: the ordering kernel and the prefill; on the
     tensor-core path a long sequence is split (a sequence of at least 16,384 tokens with
-    2 L 148 > 3 T H), which adds the chain of start states and a second prefill pass."""
+    2 L sms > 3 T H on a device with ``sms`` SMs), which adds the chain of start states
+    and a second prefill pass, plus the plain sequences' own launch when the split's
+    chain runs on its side stream."""
     T = sum(seqlens)
-    split = tc_path and any(L >= 16384 and 2 * L * 148 > 3 * T * H for L in seqlens)
-    return 4 if split else 2
+    split = tc_path and any(L >= 16384 and 2 * L * sms > 3 * T * H for L in seqlens)
+    return 5 if split else 2
+
+
+def workload_config(w, world):
+    """The ``config`` object of the JSON line: the same for both arms."""
+    N = len(w.seqlens)
+    return {"workload": w.name, "num_seqs": N,
+            "seq_lens": "x".join(str(x) for x in sorted(set(w.seqlens))) if N < 10 else f"{N} varlen",
+            "total_tokens_per_gpu": w.total_tokens, "H": w.H, "d_k": w.dk, "d_v": w.dv,
+            "chunk": w.chunk, "qkv": w.dtype, "state": "fp32", "gates": "fp32",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "inputs larger than L2 (no flush)"}
 
 
 def load_peaks():
@@ -102,64 +115,125 @@ def load_peaks():
 
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples the SM clock and the clock-event (throttle) reasons while the timed
+    region runs, through read-only NVML queries in a background thread
+    (``nvmlDeviceGetClockInfo``, ``nvmlDeviceGetMaxClockInfo``,
+    ``nvmlDeviceGetCurrentClocksEventReasons``); ``nvidia-smi --query-gpu`` is the
+    fallback when NVML cannot be loaded.  Only samples taken between ``mark_start()``
+    and ``mark_end()`` (the timed region) enter the summary.  Nothing here changes a
+    setting of the GPU."""
 
-    FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
-              "clocks_event_reasons.hw_thermal_slowdown",
-              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
     NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    # NVML clock-event reason bits (nvml.h): SwPowerCap 0x4, HwSlowdown 0x8,
+    # SwThermalSlowdown 0x20, HwThermalSlowdown 0x40
+    BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+            "hw_thermal_slowdown": 0x40}
+    SMI_FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
+                  "clocks_event_reasons.hw_thermal_slowdown",
+                  "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
 
-    def __init__(self, index):
+    def __init__(self, index, period_s=0.002):
         self.index = index
-        self.proc = None
-        self.lines = []
-        self.thread = None
+        self.period = period_s
+        self.samples = []  # (perf_counter, sm_mhz, max_mhz, set of reasons)
+        self.source = None
+        self.t0 = self.t1 = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nvml = None
+        self._handle = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        handle = None
+        try:  # the CUDA device's PCI bus id names the same GPU in NVML
+            props = torch.cuda.get_device_properties(self.index)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            handle = None
+        if handle is None:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            ids = [x for x in vis.split(",") if x.strip()]
+            idx = int(ids[self.index]) if self.index < len(ids) and ids[self.index].strip().isdigit() else self.index
+            handle = pynvml.nvmlDeviceGetHandleByIndex(idx)
+        return pynvml, handle
+
+    def _reasons_nvml(self):
+        nv = self._nvml
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        bits = int(fn(self._handle))
+        return {n for n, b in self.BITS.items() if bits & b}
+
+    def _poll_nvml(self):
+        nv, h = self._nvml, self._handle
+        mx = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+        while not self._stop.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                self.samples.append((time.perf_counter(), sm, mx, self._reasons_nvml()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def _poll_smi(self):
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index),
+                                      f"--query-gpu={','.join(self.SMI_FIELDS)}",
+                                      "--format=csv,noheader,nounits"],
+                                     capture_output=True, text=True, timeout=5).stdout
+                parts = [p.strip() for p in out.strip().split(",")]
+                if len(parts) == len(self.SMI_FIELDS):
+                    reasons = {n for n, v in zip(self.NAMES, parts[2:]) if v.lower() == "active"}
+                    self.samples.append((time.perf_counter(), float(parts[0]), float(parts[1]), reasons))
+            except Exception:
+                pass
+            time.sleep(0.02)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={','.join(self.FIELDS)}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except OSError:
-            self.proc = None
-        time.sleep(0.3)
+            self._nvml, self._handle = self._nvml_handle()
+            self.source = "nvml"
+            target = self._poll_nvml
+        except Exception:
+            self.source = "nvidia-smi"
+            target = self._poll_smi
+        self._thread = threading.Thread(target=target, daemon=True)
+        self._thread.start()
         return self
 
-    def _read(self):
-        for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
 
     def __exit__(self, *exc):
-        time.sleep(0.2)
-        if self.proc is not None:
-            self.proc.terminate()
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=10)
+        if self.source == "nvml":
             try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
         return False
 
     def summary(self):
-        sm, smax, reasons = [], [], set()
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) != len(self.FIELDS):
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for name, val in zip(self.NAMES, parts[2:]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        lo = self.t0 if self.t0 is not None else float("-inf")
+        hi = self.t1 if self.t1 is not None else float("inf")
+        win = [x for x in self.samples if lo <= x[0] <= hi]
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": self.source}
+        reasons = set()
+        for x in win:
+            reasons |= x[3]
+        return {"sm_mhz": statistics.median(x[1] for x in win), "sm_max_mhz": max(x[2] for x in win),
+                "reasons": sorted(reasons), "samples": len(win), "source": self.source}
 
 
 def dist_setup(backend="nccl"):
@@ -175,16 +249,21 @@ def dist_setup(backend="nccl"):
     return world, rank, local
 
 
-def time_region(fn, steps, stream):
-    """Device time of ``steps`` calls of fn, CUDA events on the launching stream."""
+def time_region(fn, steps, stream, clock=None):
+    """Device time of ``steps`` calls of fn, CUDA events on the launching stream.
+    ``clock`` (a running ClockSampler) is told where the region starts and ends."""
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
+    if clock is not None:
+        clock.mark_start()
     start.record(stream)
     for _ in range(steps):
         fn()
     end.record(stream)
     torch.cuda.synchronize()
+    if clock is not None:
+        clock.mark_end()
     return start.elapsed_time(end) / 1e3
 
 
@@ -261,8 +340,7 @@ def run_reference(args):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "total_tokens": w.total_tokens, "H": w.H,
-                       "d_k": w.dk, "d_v": w.dv, "chunk": w.chunk},
+            "config": workload_config(w, world), "sample": sample,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -279,6 +357,7 @@ def run_ours(args):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
     peaks, peak_kind = load_peaks()
     w = inputs.WORKLOADS[args.workload]
     assert w.kind == "prefill"
@@ -301,7 +380,7 @@ def run_ours(args):
         step()
     barrier(world)
     with ClockSampler(local) as clk:
-        elapsed = time_region(step, args.steps, stream)
+        elapsed = time_region(step, args.steps, stream, clock=clk)
     barrier(world)
     elapsed = max_over_ranks(elapsed, world)
     ms = elapsed / args.steps * 1e3
@@ -447,13 +526,14 @@ def run_ours(args):
         # adjoint 18 (P, S_t, G += q do^T, S_t do, G e, G^T k, dP, P du, dP.P, alpha dP)
         b_flops = head_tokens * w.dk * w.dv * 23
         b_tf = b_flops / b_t / 1e12
-        alu_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+        sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
+        alu_peak = sms * 128 * 2 * sm_mhz * 1e6 / 1e12
         backward = {"value": weak_scaling_value(T, b_steps, b_el, world), "unit": UNIT,
                     "ms_per_step": b_t * 1e3, "steps": b_steps, "gpu_launches_per_step": 3,
                     "grads": "dq, dk, dv, dlog_alpha, dbeta, dS0 (float32)",
                     "roofline": {"bound": "alu", "achieved": b_tf, "peak": alu_peak, "unit": "TFLOP/s",
                                  "frac": b_tf / alu_peak, "alg_flops_per_launch": b_flops,
-                                 "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 flops x 1965 MHz"}}
+                                 "peak_source": f"derived: {sms} SMs x 128 fp32 lanes x 2 flops x {sm_mhz:.0f} MHz"}}
         del dO, dSf, bws
 
     # decode: 256 sequences x 32 heads, 64 consecutive one-token steps
@@ -517,6 +597,41 @@ def run_ours(args):
                   "gpu_launches_per_step": 1, "multi_token": decode_tokens}
         del dinp, S
 
+    # the 1,048,576-token long-context packing (one 524,288-token sequence + 64 shorter
+    # ones, H = 32), timed like the headline workload; the tensor-core path splits the
+    # long sequence into segments that run in parallel
+    longctx = None
+    if not args.no_longctx and args.workload != "longctx_varlen_prefill":
+        lw = inputs.WORKLOADS["longctx_varlen_prefill"]
+        linp = inputs.prefill_inputs(lw.seqlens, lw.H, lw.dk, lw.dv, lw.dtype, lw.s0_std,
+                                     lw.seed + 1000 * rank, device=dev)
+        LT, LN = lw.total_tokens, len(lw.seqlens)
+        lo = torch.empty(LT, lw.H, lw.dv, dtype=linp["q"].dtype, device=dev)
+        lS = torch.empty(LN, lw.H, lw.dk, lw.dv, dtype=torch.float32, device=dev)
+        lws = torch.empty(max(256, prefill_workspace_size(LN, LT, lw.H, lw.dk, lw.dv, lw.chunk,
+                                                          linp["q"].dtype)), dtype=torch.uint8, device=dev)
+
+        def lstep():
+            kda_prefill(linp["q"], linp["k"], linp["v"], linp["log_alpha"], linp["beta"],
+                        linp["cu_seqlens"], linp["cu_seqlens_host"], S0=linp["S0"], chunk=lw.chunk,
+                        o=lo, S_final=lS, workspace=lws, stream=stream)
+
+        for _ in range(args.warmup):
+            lstep()
+        barrier(world)
+        l_steps = max(1, min(args.steps, 5))
+        l_el = max_over_ranks(time_region(lstep, l_steps, stream), world)
+        l_t = l_el / l_steps
+        l_bytes = LT * lw.H * prefill_bytes_per_head_token(lw.dk, lw.dv, 2) + LN * lw.H * lw.dk * lw.dv * 4
+        l_gbs = l_bytes / l_t / 1e9
+        longctx = {"workload": lw.name, "total_tokens": LT, "num_seqs": LN, "longest": max(lw.seqlens),
+                   "ms_per_step": l_t * 1e3, "steps": l_steps,
+                   "value": weak_scaling_value(LT, l_steps, l_el, world), "unit": UNIT,
+                   "gpu_launches_per_step": prefill_launches(lw.seqlens, lw.H, True, sms),
+                   "roofline": {"bound": "hbm", "achieved": l_gbs, "peak": hbm_peak, "unit": "GB/s",
+                                "frac": l_gbs / hbm_peak, "alg_bytes_per_launch": l_bytes}}
+        del linp, lo, lS, lws
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, sample, _ = oracle_sample(inputs.WORKLOADS[args.workload], args.ref_head_tokens)
@@ -527,17 +642,12 @@ def run_ours(args):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": w.name, "num_seqs": N, "seq_lens": "x".join(
-                    str(x) for x in sorted(set(w.seqlens))) if N < 10 else f"{N} varlen",
-                    "total_tokens_per_gpu": T, "H": w.H, "d_k": w.dk, "d_v": w.dv,
-                    "chunk": w.chunk, "state": "fp32", "gates": "fp32",
-                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                    "l2": "inputs larger than L2 (no flush)"},
+                "config": workload_config(w, world),
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": prefill_launches(w.seqlens, w.H, w.dtype == "bf16" and w.dk == 128 and w.dv == 128
-                                                 and w.chunk == 64) * args.steps,
+                                                 and w.chunk == 64, sms) * args.steps,
                 "clocks": clk.summary(), "decode": decode,
-                "gated_epilogue": gated, "prologue": prologue, "backward": backward}
+                "longctx": longctx, "gated_epilogue": gated, "prologue": prologue, "backward": backward}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -559,6 +669,7 @@ def main():
     ap.add_argument("--no-gated", action="store_true")
     ap.add_argument("--no-prologue", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-longctx", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps

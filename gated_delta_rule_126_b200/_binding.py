@@ -131,7 +131,14 @@ def _shapes(**named):
 
 
 def _offsets(cu_seqlens, cu_seqlens_host, T):
-    """(N, host copy of the offsets); the offsets must end within the T rows given."""
+    """(N, host copy of the offsets); the offsets must end within the T rows given.
+
+    ``cu_seqlens_host`` must hold the same values as the device tensor ``cu_seqlens``:
+    the host copy sizes the launches and is the one checked here, while the kernels
+    read the device copy.  Offsets on the device that differ from the host copy (or
+    end past the T rows) make the kernels read and write outside the tensors.  When
+    in doubt, pass ``cu_seqlens_host=None``: the offsets are then copied from the
+    device (which synchronises)."""
     if not isinstance(cu_seqlens, torch.Tensor) or cu_seqlens.dim() != 1:
         raise ValueError("cu_seqlens must be a 1-D tensor")
     if cu_seqlens_host is None:

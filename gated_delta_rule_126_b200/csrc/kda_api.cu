@@ -77,12 +77,13 @@ kda_status_t launch_prefill_prologue(const kda::PrefillArgs &a, cudaStream_t st)
 
 // Plans the sequence split of the tensor-core prefill (see kda_internal.h) when the
 // workspace has room: sequences with L >= kSplitMinLen whose critical path exceeds 1.5x
-// the even spread of the whole call over the SMs (2 L 148 > 3 T H), longest first.
+// the even spread of the whole call over the device's SMs (2 L SMs > 3 T H), longest first.
 // Returns false (no split) otherwise.
 bool plan_split(kda::PrefillArgs &a, const int32_t *cu_host, void *workspace, size_t workspace_bytes) {
     const kda::WorkspaceLayout wl = kda::workspace_layout(a.num_seqs, a.total_tokens, a.H, true);
     if (wl.split_offset == 0 || workspace_bytes < wl.total) return false;
-    const int m_max = kda::split_max_seqs(a.total_tokens, a.H);
+    const int sms = kda::device_sm_count();
+    const int m_max = kda::split_max_seqs(a.total_tokens, a.H, sms);
     int picked[kda::kMaxSplitSeqs];
     int m = 0;
     for (; m < m_max; ++m) {  // the longest qualifying sequences not yet picked
@@ -92,7 +93,7 @@ bool plan_split(kda::PrefillArgs &a, const int32_t *cu_host, void *workspace, si
             const int64_t len = int64_t(cu_host[n + 1]) - cu_host[n];
             bool taken = false;
             for (int i = 0; i < m; ++i) taken |= picked[i] == n;
-            if (taken || len < kda::kSplitMinLen || 2 * len * 148 <= 3 * a.total_tokens * a.H) continue;
+            if (taken || len < kda::kSplitMinLen || 2 * len * sms <= 3 * a.total_tokens * a.H) continue;
             if (len > best_len) best = n, best_len = len;
         }
         if (best < 0) break;
@@ -206,6 +207,23 @@ cudaError_t launch_prefill_tc_split(kda::PrefillArgs a, const int32_t *cu_host, 
 }
 
 }  // namespace
+
+namespace kda {
+
+int device_sm_count() {
+    constexpr int kMaxDevices = 64;
+    static int per_device[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (per_device[dev] <= 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        per_device[dev] = n;
+    }
+    return per_device[dev];
+}
+
+}  // namespace kda
 
 extern "C" {
 

@@ -381,7 +381,7 @@ cudaError_t launch_backward_t(const BwdArgs &a, cudaStream_t st) {
     bwd_grads_kernel<T><<<grid, kRows, 0, st>>>(a);
     if (a.T > 0) {
         const int64_t n = a.T * a.H * a.dk;
-        const unsigned rg = unsigned(std::min<int64_t>((n + 255) / 256, 148 * 16));
+        const unsigned rg = unsigned(std::min<int64_t>((n + 255) / 256, int64_t(kda::device_sm_count()) * 16));
         bwd_reduce_kernel<<<rg, 256, 0, st>>>(a);
     }
     return cudaGetLastError();

@@ -422,14 +422,7 @@ cudaError_t launch_decode_tokens(const DecodeTokensArgs &a, cudaStream_t stream)
     const uintptr_t rows = reinterpret_cast<uintptr_t>(a.q) | reinterpret_cast<uintptr_t>(a.k) |
                            reinterpret_cast<uintptr_t>(a.v) | reinterpret_cast<uintptr_t>(a.log_alpha);
     if (full && (rows & 15u) == 0) {  // persistent, state-streaming form (its cp.async copies need 16-byte rows)
-        static int sm_count = 0;
-        if (sm_count == 0) {
-            int dev = 0;
-            if (cudaGetDevice(&dev) != cudaSuccess ||
-                cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sm_count <= 0)
-                sm_count = 148;
-        }
-        const unsigned pgrid = min(grid, unsigned(sm_count * kStreamCtasPerSm));
+        const unsigned pgrid = min(grid, unsigned(device_sm_count() * kStreamCtasPerSm));
         cudaError_t err;
         if (a.dtype == KDA_DTYPE_BF16) {
             constexpr uint32_t smem = kStateBytes + stream_raw_bytes<__nv_bfloat16>();

@@ -38,12 +38,17 @@ struct SplitPlan {
     float *sstart = nullptr, *lmat = nullptr, *mmat = nullptr;  // [slot][H][128][128] float32 each
 };
 
-// Most sequences a split can take for these sizes (the criterion in kda_api.cu:
-// L >= kSplitMinLen and 2 L 148 > 3 T H, so fewer than 296 / (3 H) sequences qualify).
-inline int split_max_seqs(int64_t total_tokens, int H) {
+// Streaming multiprocessors of the current device (cudaDevAttrMultiProcessorCount,
+// read once per device; 148, the B200's count, if the query fails).
+int device_sm_count();
+
+// Most sequences a split can take for these sizes on a device with `sms` SMs (the
+// criterion in kda_api.cu: L >= kSplitMinLen and 2 L sms > 3 T H, so fewer than
+// 2 sms / (3 H) sequences qualify).
+inline int split_max_seqs(int64_t total_tokens, int H, int sms) {
     int64_t m = total_tokens / kSplitMinLen;
     m = m < kMaxSplitSeqs ? m : kMaxSplitSeqs;
-    const int64_t by_h = 296 / (3 * int64_t(H > 0 ? H : 1));
+    const int64_t by_h = 2 * int64_t(sms) / (3 * int64_t(H > 0 ? H : 1));
     return int(m < by_h ? m : by_h);
 }
 
@@ -57,12 +62,12 @@ struct WorkspaceLayout {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// split_states: room for a sequence split (tensor-core path only).
+// split_states: room for a sequence split (tensor-core path only) on the current device.
 inline WorkspaceLayout workspace_layout(int num_seqs, int64_t total_tokens = 0, int H = 0, bool split_states = false) {
     WorkspaceLayout L;
     L.order_offset = WorkspaceLayout::kStatusBytes;
     L.total = align256(L.order_offset + sizeof(int32_t) * size_t(num_seqs > 0 ? num_seqs : 1));
-    const int m = split_states ? split_max_seqs(total_tokens, H) : 0;
+    const int m = split_states ? split_max_seqs(total_tokens, H, device_sm_count()) : 0;
     if (m > 0) {
         L.split_offset = L.total;
         L.split_array_bytes = size_t(m) * kSplitP * size_t(H) * 128 * 128 * sizeof(float);

@@ -7,7 +7,9 @@
 // the scratch that kda_prefill keeps in the caller's workspace (a device status
 // word and the longest-first sequence order) lives in one file-scope device array
 // instead.  Every GPU that loads this library holds that array until the process
-// exits.  The launches are the same as kda_prefill's.
+// exits.  It never splits a long sequence into segments (the split keeps segment
+// start states in the workspace), so each (sequence, head) is one unit; for inputs
+// that kda_prefill runs unsplit, the launches and results are the same as its.
 #include <mutex>
 
 #include "kda_internal.h"

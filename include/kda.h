@@ -219,7 +219,12 @@ KDA_API kda_status_t kda_decode_step(const void *q, const void *k, const void *v
  * until the process exits.
  *
  * - num_seqs > KDA_NOALLOC_MAX_SEQS returns KDA_ERR_WORKSPACE before anything is
- *   queued; every other check and result is kda_prefill's.
+ *   queued; the other argument checks are kda_prefill's.
+ * - It never uses kda_prefill's sequence split (which needs workspace for the
+ *   segments' start states): every (sequence, head) runs as one unit.  Where
+ *   kda_prefill would split a very long sequence, this call takes longer (the
+ *   long sequence's chunks run one after another on one SM per head); elsewhere
+ *   it runs the same kernels on the same inputs and gives bit-identical results.
  * - The first call on a device looks up the array's device address for that
  *   device (once per device, with that device current); make that first call
  *   before any stream capture.
