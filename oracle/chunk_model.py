@@ -21,8 +21,14 @@ Within one chunk of L <= C tokens that starts from state S (rows r, i = tokens):
   O       = (Q * exp(g)) S + P U                          (rows o_r = S_r^T q_r)
   S_next  = Diag(exp(g_L)) S + (K * exp(g_L - g))^T U
 
-Every exponent is formed as a difference before exp, so nothing overflows; the
-chunk model is slow on purpose and only runs on small inputs.
+The decay between token i and a later token r, exp(g_r - g_i), is the product of the
+alphas of tokens i+1 .. r.  The page's decay range alpha in [0, 1]^{d_k} (its
+"Channel-wise 衰减" bullet) includes alpha = 0 (log alpha = -inf), where the running
+sums g are -inf from that token on and g_r - g_i would be -inf - (-inf).  So every
+exponent here is formed as a sum of log alpha over exactly the tokens it spans
+(g_r - g_i over i+1 .. r, g_L - g_r over r+1 .. L), never as a difference of running
+sums; nothing overflows and alpha = 0 gives exact zeros.  The chunk model is slow on
+purpose and only runs on small inputs.
 """
 from __future__ import annotations
 
@@ -43,8 +49,13 @@ def chunk_stages(q, k, v, log_alpha, beta):
     b = np.asarray(beta, np.float64)
     L = q.shape[0]
     g = np.cumsum(la, axis=0)
-    # decay between token i and a later token r, per channel: exp(g_r - g_i)
-    diff = np.exp(g[:, None, :] - g[None, :, :])            # [L, L, d_k]
+    # decay between token i and a later token r, per channel: exp(sum of log alpha over
+    # tokens i+1 .. r); zero for r < i (those pairs are masked out below)
+    diff = np.zeros((L, L, la.shape[1]))                     # [r, i, d_k]
+    for i in range(L):
+        diff[i, i] = 1.0
+        if i + 1 < L:
+            diff[i + 1:, i] = np.exp(np.cumsum(la[i + 1:], axis=0))
     kk = np.einsum("rc,ic,ric->ri", k, k, diff)
     qk = np.einsum("rc,ic,ric->ri", q, k, diff)
     strict = np.tril(np.ones((L, L)), -1)
@@ -54,7 +65,10 @@ def chunk_stages(q, k, v, log_alpha, beta):
     P = qk * incl
     Kg = k * np.exp(g)
     Qg = q * np.exp(g)
-    Khat = k * np.exp(g[-1][None, :] - g)
+    # g_L - g_r = sum of log alpha over tokens r+1 .. L (zero for the last token)
+    after = np.zeros_like(la)
+    after[:-1] = np.cumsum(la[::-1], axis=0)[::-1][1:]
+    Khat = k * np.exp(after)
     return dict(g=g, A=A, T=T, P=P, Kg=Kg, Qg=Qg, Khat=Khat, Gamma=np.exp(g[-1]),
                 Ut=T @ v, W=T @ Kg)
 

@@ -251,8 +251,60 @@ def pin_varlen_independence(run, seed=10):
         assert rel_err(S[n], Sn[0]) < RTOL
 
 
+def pin_zero_decay_erases_state(run, seed=11):
+    """alpha in [0,1] (the KDA section's channel-wise decay bullet) includes 0.  A token
+    whose decay is 0 in every key channel (log alpha = -inf) zeroes Diag(alpha_t) S_{t-1},
+    so S_t = beta_t k_t v_t^T and o_t = beta_t (q_t . k_t) v_t whatever came before, and
+    every later output and the final state are independent of S0 and of the earlier
+    tokens.  No value may be NaN or infinite."""
+    rng = np.random.default_rng(seed)
+    T, H, dk, dv, t0 = 9, 2, 4, 3, 4
+    q, k, v, la, b = _rand_case(rng, T, H, dk, dv)
+    la[t0] = -np.inf
+    cu = _single(T)
+    o, S = run(q, k, v, la, b, cu, rng.standard_normal((1, H, dk, dv)))
+    assert np.isfinite(o).all() and np.isfinite(S).all()
+    for h in range(H):
+        want = b[t0, h] * np.dot(q[t0, h], k[t0, h]) * v[t0, h]
+        assert rel_err(o[t0, h], want) < RTOL
+    _, St0 = run(q[:t0 + 1], k[:t0 + 1], v[:t0 + 1], la[:t0 + 1], b[:t0 + 1], _single(t0 + 1),
+                 rng.standard_normal((1, H, dk, dv)))
+    for h in range(H):
+        assert rel_err(St0[0, h], b[t0, h] * np.outer(k[t0, h], v[t0, h])) < RTOL
+    # other earlier tokens and another initial state: the same outputs from t0 on
+    q2, k2, v2, la2, b2 = _rand_case(rng, T, H, dk, dv)
+    for x, x2 in ((q, q2), (k, k2), (v, v2), (la, la2), (b, b2)):
+        x2[t0:] = x[t0:]
+    o2, S2 = run(q2, k2, v2, la2, b2, cu, rng.standard_normal((1, H, dk, dv)))
+    assert rel_err(o2[t0:], o[t0:]) < RTOL
+    assert rel_err(S2, S) < RTOL
+
+
+def pin_bruteforce_strong_decay(run, seed=12):
+    """The explicit products M_t = (I - beta_t k_t k_t^T) Diag(alpha_t) with decays over the
+    whole range [0, 1]: single channels with alpha = 0 (log alpha = -inf), decays far below
+    the fp32 range (log alpha = -200) and near-one decays mixed in one head."""
+    rng = np.random.default_rng(seed)
+    T, H, dk, dv = 7, 1, 4, 3
+    q, k, v, la, b = _rand_case(rng, T, H, dk, dv, unit_k=False)
+    la[:, 0, 0] = -200.0          # channel 0 forgets within one token
+    la[2, 0, 1] = -np.inf         # channel 1 is erased at token 2
+    la[5, 0, 2] = -np.inf         # channel 2 at token 5
+    la[:, 0, 3] = -1e-3           # channel 3 nearly keeps everything
+    S0 = rng.standard_normal((1, H, dk, dv))
+    o, S = run(q, k, v, la, b, _single(T), S0)
+    assert np.isfinite(o).all() and np.isfinite(S).all()
+    M = [(np.eye(dk) - b[t, 0] * np.outer(k[t, 0], k[t, 0])) @ np.diag(np.exp(la[t, 0])) for t in range(T)]
+    St = S0[0, 0]
+    for t in range(T):
+        St = M[t] @ St + b[t, 0] * np.outer(k[t, 0], v[t, 0])
+        assert rel_err(o[t, 0], St.T @ q[t, 0]) < RTOL
+    assert rel_err(S[0, 0], St) < RTOL
+
+
 ALL_PINS = [pin_hand_worked, pin_beta_zero_closed_form, pin_exact_reconstruction,
             pin_orthonormal_linear_attention, pin_scalar_gate_gdn,
             lambda run: pin_scalar_gate_gdn(run, ungated=True),
             pin_bruteforce_products, pin_scalar_d1, pin_linearity,
-            pin_householder_norms, pin_split_invariance, pin_varlen_independence]
+            pin_householder_norms, pin_split_invariance, pin_varlen_independence,
+            pin_zero_decay_erases_state, pin_bruteforce_strong_decay]
