@@ -148,6 +148,25 @@ def prefill_inputs(seqlens, H, dk, dv, dtype="bf16", s0_std=0.0, seed=0,
                 cu_seqlens_host=cu_host)
 
 
+def decay_log_alpha(T, H, dk, scale=1.0, zero_frac=0.0, seed=0, device="cpu"):
+    """log alpha [T,H,dk] fp32 for decays across the whole range alpha in [0, 1].
+
+    log alpha = -scale * softplus(N(0, 1)); ``scale`` is a float or a per-channel
+    tensor [dk] (fast- and slow-forgetting channels side by side).  A fraction
+    ``zero_frac`` of the entries, drawn at random, is -inf (alpha = 0: the channel is
+    erased at that token).  The workloads use scale 0.1 and no zeros; these stronger
+    decays test the chunked paths over the rest of the range.
+    """
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    f32 = dict(dtype=torch.float32, device=device, generator=gen)
+    sc = torch.as_tensor(scale, dtype=torch.float32, device=device)
+    la = -sc * F.softplus(torch.randn(T, H, dk, **f32))
+    if zero_frac > 0:
+        la = torch.where(torch.rand(T, H, dk, **f32) < zero_frac, torch.full_like(la, float("-inf")), la)
+    return la.contiguous()
+
+
 def gate_inputs(T, H, dv, dtype="bf16", seed=0, device="cpu"):
     """Synthetic inputs of the output epilogue: the gate pre-activation [T,H,dv]
     (dtype, ~ N(0, 1)) and the RMSNorm weight [dv] (float32, ~ 1 + 0.1 N(0, 1)).
