@@ -75,6 +75,7 @@ constexpr int NP = 256;  // prep group: warps 4-11
 constexpr int NT = NS + NP;
 constexpr uint32_t BAR_S = 1, BAR_P = 2;  // named barriers of the two groups
 constexpr float kShiftBound = 16.f;       // |H_R| (base 2) up to which a block's own pairs use the tensor cores
+constexpr float kFastBound = 5.f;         // |H_R| (base 2) of every block up to which a chunk takes the mid-chunk factoring
 
 // Shared memory map (bytes from a 1024-aligned base).
 constexpr uint32_t OFF_QK = 0;        // raw k|q boxes [k0 q0 k1 q1] -> [Km; Qm] in place (128 x 128 fp16, K-major)
@@ -87,31 +88,44 @@ constexpr int LDF = 68;
 constexpr uint32_t OFF_EB = OFF_AX + 64 * LDF * 4;  // solve scratch; the block totals while the rows are built
 constexpr int LDE = 20;
 constexpr int LDG = 33;
-constexpr uint32_t OFF_P = 178176;    // P (64 x 64 fp16), two buffers
+constexpr uint32_t OFF_P = 178176;    // P (64 x 64 fp16), two buffers (after the control structures below)
 static_assert(OFF_EB + 32 * LDG * 4 <= OFF_P && OFF_EB + 8 * D * 4 <= OFF_P, "solve scratch overflows");
 constexpr uint32_t OFF_T = OFF_P + 16384;    // T (64 x 64 fp16); the exact diagonal blocks' partial sums
 constexpr uint32_t OFF_Y = OFF_T + 8192;     // the bf16 output tile (two 64 x 64 boxes); the gate tile (gated)
 constexpr uint32_t OFF_ID = OFF_Y + 16384;   // -I (64 x 64 bf16): loads -V^T into Z with an MMA
 constexpr uint32_t OFF_VEC = OFF_ID + 8192;  // per-chunk vectors, two buffers (chunk parity)
 constexpr uint32_t VEC_BETA = 0;      // beta                 64 f32
-constexpr uint32_t VEC_GAM = 256;     // e^{g_L}             128 f32
-constexpr uint32_t VEC_BYTES = 768;
-constexpr uint32_t OFF_BAR = OFF_VEC + 2 * VEC_BYTES;   // mbarriers
+constexpr uint32_t VEC_FS = 256;      // the pass over R: Sop = fp16(R f_s)      128 f32
+constexpr uint32_t VEC_FR = 768;      //                  R <- R f_r             128 f32
+constexpr uint32_t VEC_BYTES = 1280;
+// Small control structures, in the gap before the 1024-aligned P tiles.
+constexpr uint32_t OFF_BAR = OFF_EB + 32 * LDG * 4;     // mbarriers of the TMA loads and MMAs
 constexpr int NBAR = 8;
 constexpr int B_QK = 0, B_V = 1, B_M1 = 2, B_M2 = 3, B_M3 = 4, B_M45 = 5, B_G = 6;
-constexpr uint32_t OFF_CNT = OFF_BAR + 8 * NBAR;        // progress counters
-constexpr int CNT_P2 = 0, CNT_KQF = 1, CNT_TP = 2, CNT_TW = 3, CNT_M45 = 4;
-constexpr uint32_t OFF_ISS = OFF_CNT + 32;              // phases issued / waited per mbarrier
+// Hand-overs between the groups: one thread-arrive mbarrier per signal and chunk parity; the
+// signal of chunk c completes phase c >> 1 of barrier 2 * signal + (c & 1).  No producer can
+// complete chunk c + 2's phase before the consumer has waited for chunk c's.
+constexpr uint32_t OFF_SIG = OFF_BAR + 8 * NBAR;
+constexpr int S_P2 = 0, S_KQF = 1, S_TP = 2, S_TW = 3, S_M45 = 4, NSIG = 5;
+//   S_P2:  prep -> state: the operand rows, f_s, f_r and beta of chunk c (and M1 issued)
+//   S_KQF: state -> prep: M2 of chunk c has read [Kg; Qg]
+//   S_TP:  prep -> state: X of chunk c
+//   S_TW:  state -> prep: T of chunk c formed (X read)
+//   S_M45: state -> prep: M4/M5 of chunk c done (Kl, P of its parity and the T tile read)
+constexpr uint32_t OFF_ISS = OFF_SIG + 8 * 2 * NSIG;    // phases issued / waited per mbarrier
 constexpr uint32_t OFF_WT = OFF_ISS + 4 * NBAR;
-constexpr uint32_t OFF_FLAG = OFF_WT + 4 * NBAR;        // per (block, channel box): a channel past the bound
-constexpr uint32_t OFF_MISC = OFF_FLAG + 32;            // tmem base, abort flag, S_final pointer
-constexpr uint32_t SMEM_USED = OFF_MISC + 16;
+constexpr uint32_t OFF_FLAG = OFF_WT + 4 * NBAR;        // per (block, channel box): bit 0 past the exact bound,
+                                                        // bit 1 past the fast bound; then the chunk kind by parity
+constexpr uint32_t OFF_MISC = OFF_FLAG + 48;            // tmem base, abort flag, S_final pointer
+constexpr uint32_t OFF_CTRL_END = OFF_MISC + 16;
+constexpr uint32_t SMEM_USED = OFF_VEC + 2 * VEC_BYTES;
 // The gated output epilogue's per-token reduction of o^2 (4 x 64 partial sums, then 64
 // reciprocal RMS values); its gate tile shares the output tile.
 constexpr uint32_t OFF_RED = SMEM_USED;
 constexpr uint32_t SMEM_USED_G = OFF_RED + 320 * 4;
 constexpr uint32_t smem_alloc(bool gated) { return (gated ? SMEM_USED_G : SMEM_USED) + 1024; }  // + alignment slack
 static_assert(smem_alloc(true) <= 232448, "shared memory");
+static_assert(OFF_CTRL_END <= OFF_P, "control structures overflow into the P tiles");
 static_assert(OFF_KL % 1024 == 0 && OFF_V % 1024 == 0 && OFF_P % 1024 == 0 && OFF_Y % 1024 == 0 &&
               OFF_ID % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 
@@ -277,7 +291,7 @@ __global__ void __launch_bounds__(NT, 1)
 
     auto vec = [&](int par, uint32_t field) { return reinterpret_cast<float *>(sm + OFF_VEC + par * VEC_BYTES + field); };
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-    uint32_t *cnt = reinterpret_cast<uint32_t *>(sm + OFF_CNT);
+    uint64_t *sigs = reinterpret_cast<uint64_t *>(sm + OFF_SIG);
     uint32_t *iss = reinterpret_cast<uint32_t *>(sm + OFF_ISS);
     uint32_t *wt = reinterpret_cast<uint32_t *>(sm + OFF_WT);
     int *flags = reinterpret_cast<int *>(sm + OFF_FLAG);
@@ -294,7 +308,7 @@ __global__ void __launch_bounds__(NT, 1)
             iss[b] = 0;
             wt[b] = 0;
         }
-        for (int i = 0; i < 8; ++i) cnt[i] = 0;
+        for (int i = 0; i < 2 * NSIG; ++i) ptx::mbar_init(sigs + i, 1);
         ptx::fence_mbar_init();
         *s_abort = 0;
         *reinterpret_cast<float **>(sm + OFF_MISC + 8) = sfin;  // read back at the end (frees registers)
@@ -351,25 +365,29 @@ __global__ void __launch_bounds__(NT, 1)
         if (leader) wt[b] = phase + 1;
         return true;
     };
-    // Wait until progress counter i reaches `target` (bounded, gives up on an abort).
-    auto cwait = [&](int i, uint32_t target) {
-        if (ptx::ld_acquire(cnt + i) >= target) return true;
+    // Wait for signal g of chunk c (bounded, gives up on an abort); chunk c < 0 needs no wait.
+    auto swait = [&](int g, int c) {
+        if (c < 0) return true;
+        uint64_t *bar = sigs + 2 * g + (c & 1);
+        const uint32_t parity = uint32_t(c >> 1) & 1u;
+        if (ptx::mbar_try_wait(bar, parity)) return true;
         const long long t0 = clock64();
-        while (ptx::ld_acquire(cnt + i) < target) {
+        while (!ptx::mbar_try_wait(bar, parity)) {
             if (*reinterpret_cast<volatile int *>(s_abort) || clock64() - t0 > kWaitCycles) {
                 fail();
                 return false;
             }
-            __nanosleep(20);
         }
         return true;
     };
+    // Signal g of chunk c (one thread, after its group's barrier): release at CTA scope.
+    auto sarrive = [&](int g, int c) { ptx::mbar_arrive(sigs + 2 * g + (c & 1)); };
 
-    // Launched with 384 x 168 registers: the prep group (8 warps) drops to 128, the
-    // state group (4 warps) rises to 240; 4 x 32 x 240 + 8 x 32 x 128 <= 384 x 168.
+    // Launched with 384 x 168 registers: the prep group (8 warps) drops to 160, the
+    // state group (4 warps) rises to 184; 4 x 32 x 184 + 8 x 32 x 160 = 384 x 168.
     if (warp < 4) {
         // =================================================================== state group
-        ptx::regs_inc<240>();
+        ptx::regs_inc<184>();
         const int row = tid;  // TMEM lane = value column j
         const uint32_t tl = tbase + (uint32_t(warp * 32) << 16);
         const bool leader = tid == 0;
@@ -403,38 +421,54 @@ __global__ void __launch_bounds__(NT, 1)
             const bool has_next = ci + 1 < nchunks;
             const int par = ci & 1;
 
-            // ---- E0: Sop = fp16(R) (the chunk-start state), then R *= e^{g_L} per key channel.
-            cwait(CNT_P2, ci + 1);  // e^{g_L}, beta and [Kg; Qg] of this chunk
+            // ---- E0: Sop = fp16(R f_s), R <- R f_r per key channel.  R holds S^T Diag(e^{g_m - g_L})
+            // after a fast chunk and S^T after the other kind; this chunk's kind wants Sop =
+            // S^T Diag(e^{g_m}) and R = S^T Diag(e^{g_m}) (fast), or Sop = S^T and R = S^T Diag(e^{g_L}).
+            swait(S_P2, ci);  // the operand rows, f_s, f_r and beta of this chunk
+            const bool fast = flags[8 + par] != 0;
             {
-                const float4 *gam = reinterpret_cast<const float4 *>(vec(par, VEC_GAM));
+                const float4 *fsv = reinterpret_cast<const float4 *>(vec(par, VEC_FS));
+                const float4 *frv = reinterpret_cast<const float4 *>(vec(par, VEC_FR));
                 uint32_t r4[4][32], pk[16];
 #pragma unroll
                 for (int p = 0; p < 4; ++p) ptx::tmem_ld32(tl + TS + 32 * p, r4[p]);
                 ptx::tmem_wait_ld();
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {  // 64 columns at a time
-                    uint32_t(&v)[32] = r4[2 * p];
-                    uint32_t(&w)[32] = r4[2 * p + 1];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_h2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-                    ptx::tmem_st16(tl + TSOP + 32 * p, pk);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_h2(__uint_as_float(w[2 * e]), __uint_as_float(w[2 * e + 1]));
-                    ptx::tmem_st16(tl + TSOP + 32 * p + 16, pk);
+                // x *= f (32 columns starting at column c0, factors as float4 from f4)
+                auto scale32 = [](uint32_t(&x)[32], const float4 *f4) {
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 f0 = gam[16 * p + e4], f1 = gam[16 * p + 8 + e4];
-                        v[4 * e4 + 0] = __float_as_uint(__uint_as_float(v[4 * e4 + 0]) * f0.x);
-                        v[4 * e4 + 1] = __float_as_uint(__uint_as_float(v[4 * e4 + 1]) * f0.y);
-                        v[4 * e4 + 2] = __float_as_uint(__uint_as_float(v[4 * e4 + 2]) * f0.z);
-                        v[4 * e4 + 3] = __float_as_uint(__uint_as_float(v[4 * e4 + 3]) * f0.w);
-                        w[4 * e4 + 0] = __float_as_uint(__uint_as_float(w[4 * e4 + 0]) * f1.x);
-                        w[4 * e4 + 1] = __float_as_uint(__uint_as_float(w[4 * e4 + 1]) * f1.y);
-                        w[4 * e4 + 2] = __float_as_uint(__uint_as_float(w[4 * e4 + 2]) * f1.z);
-                        w[4 * e4 + 3] = __float_as_uint(__uint_as_float(w[4 * e4 + 3]) * f1.w);
+                        const float4 f = f4[e4];
+                        x[4 * e4 + 0] = __float_as_uint(__uint_as_float(x[4 * e4 + 0]) * f.x);
+                        x[4 * e4 + 1] = __float_as_uint(__uint_as_float(x[4 * e4 + 1]) * f.y);
+                        x[4 * e4 + 2] = __float_as_uint(__uint_as_float(x[4 * e4 + 2]) * f.z);
+                        x[4 * e4 + 3] = __float_as_uint(__uint_as_float(x[4 * e4 + 3]) * f.w);
                     }
-                    ptx::tmem_st32(tl + TS + 64 * p, v);
-                    ptx::tmem_st32(tl + TS + 64 * p + 32, w);
+                };
+                // fp16 pairs of x (times f, when given) -> 16 words
+                auto pack32 = [&](const uint32_t(&x)[32], const float4 *f4) {
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 f = f4 ? f4[e4] : make_float4(1.f, 1.f, 1.f, 1.f);
+                        pk[2 * e4] = pack_h2(__uint_as_float(x[4 * e4 + 0]) * f.x, __uint_as_float(x[4 * e4 + 1]) * f.y);
+                        pk[2 * e4 + 1] = pack_h2(__uint_as_float(x[4 * e4 + 2]) * f.z, __uint_as_float(x[4 * e4 + 3]) * f.w);
+                    }
+                };
+                if (fast) {  // f_s = f_r: one product per element, packed and stored back
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        scale32(r4[p], fsv + 8 * p);
+                        pack32(r4[p], nullptr);
+                        ptx::tmem_st16(tl + TSOP + 16 * p, pk);
+                        ptx::tmem_st32(tl + TS + 32 * p, r4[p]);
+                    }
+                } else {
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        pack32(r4[p], fsv + 8 * p);
+                        ptx::tmem_st16(tl + TSOP + 16 * p, pk);
+                        scale32(r4[p], frv + 8 * p);
+                        ptx::tmem_st32(tl + TS + 32 * p, r4[p]);
+                    }
                 }
                 ptx::tmem_wait_st();
             }
@@ -455,9 +489,10 @@ __global__ void __launch_bounds__(NT, 1)
                 // Z = Sop [Kg; Qg]^T (the k and q boxes of a channel block are rows 0-63 and
                 // 64-127 of one 128-row operand), then Z[:, :64] += V^T (-I), V read MN-major
                 // from its TMA tile
+                const uint32_t kq_base = OFF_KQ;  // [Kt; Qt] or [Kg; Qg]
                 for (int ks = 0; ks < 8; ++ks) {
                     const uint32_t kq = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
-                    ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + OFF_KQ + kq), IDESC_N128,
+                    ptx::mma_ts(tbase + TZ, tbase + TSOP + 8 * ks, ptx::sdesc_sw128(sb + kq_base + kq), IDESC_N128,
                                 ks > 0);
                 }
                 if (!v_zero) {
@@ -472,7 +507,7 @@ __global__ void __launch_bounds__(NT, 1)
             mwait(B_M2, ci, leader);
             ptx::tc_fence_after();
             if (leader) {
-                ptx::st_release(cnt + CNT_KQF, ci + 1);  // [Kg; Qg] has been read
+                sarrive(S_KQF, ci);  // [Kg; Qg] has been read
                 if (has_next && !v_zero) load_v(s + C);  // the V tile has been read by the MMA
             }
 
@@ -496,7 +531,56 @@ __global__ void __launch_bounds__(NT, 1)
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
 
             // ---- M3: U^T = Y^T T^T into Z[:, :64] (T of this chunk from the prep group's X).
-            cwait(CNT_TP, ci + 1);
+            swait(S_TP, ci);
+            {  // X_21 = -(X_H1 A_21) X_H0 over 32x32 halves (X_H1 = X[32:64, 32:64] and X_H0 =
+               // X[0:32, 0:32] are zero above their diagonals); F = X_H1 A_21 in fp32 over the T tile
+                const float *Af = reinterpret_cast<const float *>(sm + OFF_AX);
+                float *X = reinterpret_cast<float *>(sm + OFF_AX);
+                float *F = reinterpret_cast<float *>(sm + OFF_T);
+                {  // F[r][c], eight columns a thread: r = tid >> 2, c8 = 8 (tid & 3)
+                    const int r = tid >> 2, c8 = 8 * (tid & 3);
+                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    const float *xr = X + (32 + r) * LDF + 32;
+                    const int mend = r < 16 ? 16 : 32;
+                    for (int m = 0; m < mend; ++m) {
+                        const float xv = xr[m];
+                        const float4 a0 = *reinterpret_cast<const float4 *>(Af + (32 + m) * LDF + c8);
+                        const float4 a1 = *reinterpret_cast<const float4 *>(Af + (32 + m) * LDF + c8 + 4);
+                        acc[0] = fmaf(xv, a0.x, acc[0]);
+                        acc[1] = fmaf(xv, a0.y, acc[1]);
+                        acc[2] = fmaf(xv, a0.z, acc[2]);
+                        acc[3] = fmaf(xv, a0.w, acc[3]);
+                        acc[4] = fmaf(xv, a1.x, acc[4]);
+                        acc[5] = fmaf(xv, a1.y, acc[5]);
+                        acc[6] = fmaf(xv, a1.z, acc[6]);
+                        acc[7] = fmaf(xv, a1.w, acc[7]);
+                    }
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) F[r * LDG + c8 + q] = acc[q];
+                }
+                ptx::named_barrier(BAR_S, NS);
+                {  // X_21[r][c] = -sum_m F[r][m] X_H0[m][c], eight columns a thread: r = tid & 31, c8 = 8 (tid >> 5)
+                    const int r = tid & 31, c8 = 8 * (tid >> 5);
+                    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    const float *fr = F + r * LDG;
+                    for (int m = c8 < 16 ? 0 : 16; m < 32; ++m) {
+                        const float fv = fr[m];
+                        const float4 x0 = *reinterpret_cast<const float4 *>(X + m * LDF + c8);
+                        const float4 x1 = *reinterpret_cast<const float4 *>(X + m * LDF + c8 + 4);
+                        acc[0] = fmaf(fv, x0.x, acc[0]);
+                        acc[1] = fmaf(fv, x0.y, acc[1]);
+                        acc[2] = fmaf(fv, x0.z, acc[2]);
+                        acc[3] = fmaf(fv, x0.w, acc[3]);
+                        acc[4] = fmaf(fv, x1.x, acc[4]);
+                        acc[5] = fmaf(fv, x1.y, acc[5]);
+                        acc[6] = fmaf(fv, x1.z, acc[6]);
+                        acc[7] = fmaf(fv, x1.w, acc[7]);
+                    }
+                    *reinterpret_cast<float4 *>(X + (32 + r) * LDF + c8) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+                    *reinterpret_cast<float4 *>(X + (32 + r) * LDF + c8 + 4) = make_float4(-acc[4], -acc[5], -acc[6], -acc[7]);
+                }
+                ptx::named_barrier(BAR_S, NS);
+            }
             {  // T[r][i] = X[r][i] beta_i for i <= r as an fp16 operand (rows r, K = i)
                 const float *X = reinterpret_cast<const float *>(sm + OFF_AX);
                 const float *beta = vec(par, VEC_BETA);
@@ -522,7 +606,7 @@ __global__ void __launch_bounds__(NT, 1)
             ptx::fence_proxy_async_smem();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
             if (leader) {
-                ptx::st_release(cnt + CNT_TW, ci + 1);
+                sarrive(S_TW, ci);
                 ptx::tc_fence_after();
                 for (int ks = 0; ks < 4; ++ks)
                     ptx::mma_ts(tbase + TZ, tbase + TY16 + 8 * ks, ptx::sdesc_sw128(sb + OFF_T + 32 * ks), IDESC_N64,
@@ -562,7 +646,7 @@ __global__ void __launch_bounds__(NT, 1)
             }
             mwait(B_M45, ci, leader);
             ptx::tc_fence_after();
-            if (leader) ptx::st_release(cnt + CNT_M45, ci + 1);
+            if (leader) sarrive(S_M45, ci);
             if (!o_skip) {  // E4: outputs of this chunk, staged over the Y^T tile as two 128-byte
                             // swizzled boxes (columns 0-63, 64-127)
                 uint32_t vo[2][32];
@@ -658,20 +742,22 @@ __global__ void __launch_bounds__(NT, 1)
             // the staged tile is rewritten (by the gate load or the next E4) only after the next
             // E0 barrier, before which the leader waits for the tile stores' reads
         }
-        // Final state S_final[c][j] = R[j][c].
-        if (!*reinterpret_cast<volatile int *>(s_abort)) {
+        // Final state S_final[c][j] = R[j][c] f[c], f = e^{g_L - g_m} after a fast last chunk, else 1.
+        if (!*reinterpret_cast<volatile int *>(s_abort) && swait(S_P2, nchunks)) {
             ptx::tc_fence_after();
             float *const sf = *reinterpret_cast<float *const *>(sm + OFF_MISC + 8);
+            const float *fin = vec(nchunks & 1, VEC_FR);
             uint32_t v[32];
             for (int p = 0; p < 4; ++p) {
                 ptx::tmem_ld32(tl + TS + 32 * p, v);
                 ptx::tmem_wait_ld();
                 for (int e = 0; e < 32; ++e) {
                     const int c = 32 * p + e;
+                    const float x = __uint_as_float(v[e]) * fin[c];
                     if constexpr (kSplit) {
-                        if (sf) sf[c * D + row] = __uint_as_float(v[e]);
+                        if (sf) sf[c * D + row] = x;
                     } else {
-                        a.S_final[((size_t(seq) * H + h) * D + c) * D + row] = __uint_as_float(v[e]);
+                        a.S_final[((size_t(seq) * H + h) * D + c) * D + row] = x;
                     }
                 }
             }
@@ -679,7 +765,7 @@ __global__ void __launch_bounds__(NT, 1)
         if (leader) ptx::bulk_wait0();
     } else {
         // =================================================================== prep group
-        ptx::regs_dec<128>();
+        ptx::regs_dec<160>();
         const int pt = tid - NS;  // 0..255
         const int pw = pt >> 5;   // prep warp 0..7
         const bool leader = pt == 0;
@@ -690,6 +776,7 @@ __global__ void __launch_bounds__(NT, 1)
         const uint32_t ob = uint32_t(g4 & 1) * 8u;
         float4 lap[8];          // log alpha of rows 16 Rb + 8 hh + j, loaded a chunk ahead
         float beta_reg = 0.f;   // beta of token pt (pt < 64), loaded a chunk ahead
+        float ecm_prev[4] = {1.f, 1.f, 1.f, 1.f};  // restores S^T from TMEM after the previous chunk
         auto load_la = [&](int cj) {
             if (cj >= nchunks) return;
             const int sj = bos + cj * C;
@@ -718,7 +805,6 @@ __global__ void __launch_bounds__(NT, 1)
         for (int ci = 0; ci < nchunks; ++ci) {
             const int s = bos + ci * C;
             const int L = min(C, eos - s);
-            const bool has_next = ci + 1 < nchunks;
             const int par = ci & 1;
 
             // ---- P2a: block sums of log alpha (base 2) for this thread's 4 channels: over its
@@ -733,7 +819,7 @@ __global__ void __launch_bounds__(NT, 1)
                 la2[j][3] = lap[j].w * kLog2e;
             }
             float pq[4], sq[4], Hb[4], shift[4];
-            bool good_all = true;
+            bool good_all = true, fast_all = true;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 float t = 0.f;
@@ -747,26 +833,55 @@ __global__ void __launch_bounds__(NT, 1)
                 const bool good = Hb[e] >= -kShiftBound;
                 shift[e] = good ? 0.5f * Hb[e] : 0.f;
                 good_all = good_all && good;
+                fast_all = fast_all && Hb[e] >= -kFastBound;
             }
             const bool wbad = __any_sync(0xffffffffu, !good_all);
+            const bool wslow = __any_sync(0xffffffffu, !fast_all);
             float *xtot = reinterpret_cast<float *>(sm + OFF_EB);  // [block][channel] totals, then shifts
             if (hh == 0) {
                 *reinterpret_cast<float4 *>(xtot + Rb * D + c0) = make_float4(Hb[0], Hb[1], Hb[2], Hb[3]);
                 *reinterpret_cast<float4 *>(xtot + 4 * D + Rb * D + c0) = make_float4(shift[0], shift[1], shift[2], shift[3]);
             }
-            if (lane == 0) flags[2 * Rb + bx] = wbad ? 1 : 0;
+            if (lane == 0) flags[2 * Rb + bx] = (wbad ? 1 : 0) | (wslow ? 2 : 0);
             mwait(B_QK, ci, leader);  // the raw k|q tile of this chunk
             if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
 
-            // ---- P2b: the per-channel factors from the four blocks' totals, then the operand
-            // rows from the raw k|q tile (rows >= L belong to the next sequence: zero): Kl and
-            // Kc^(R) for R >= Rb (backward over the rows), then Km, Qm over the raw rows, Kg and
-            // Qg (forward).
-            bool any_bad = false;
+            // ---- P2b: the chunk's kind, the per-channel factors from the four blocks' totals,
+            // then the operand rows from the raw k|q tile (rows >= L belong to the next
+            // sequence: zero).
+            //   fast (every block's decay within 2^-kFastBound in every channel): the mid-chunk
+            //     factoring, g_m = g at the end of block 1: Kt = K e^{g - g_m} and Qt = Q e^{g - g_m}
+            //     over the raw rows, Kb = K e^{g_m - g} (factors within 2^{+-2 kFastBound}); TMEM
+            //     then holds S^T e^{g_m - g_L} after the chunk.
+            //   otherwise: Kl and Kc^(R) for R >= Rb (backward over the rows), then Km, Qm over the
+            //     raw rows, Kg and Qg (forward); TMEM holds S^T.
+            bool any_bad = false, fast = true;
 #pragma unroll
-            for (int b = 0; b < 8; ++b) any_bad = any_bad || flags[b] != 0;
-            cwait(CNT_KQF, ci);                 // M2 of chunk ci - 1 has read [Kg; Qg]
-            if (ci >= 2) cwait(CNT_M45, ci - 1);  // M4/M5 of chunk ci - 2 have read Kl and P (buffer par)
+            for (int b = 0; b < 8; ++b) {
+                any_bad = any_bad || (flags[b] & 1) != 0;
+                fast = fast && (flags[b] & 2) == 0;
+            }
+            swait(S_KQF, ci - 1);  // M2 of chunk ci - 1 has read the K/Q operand tile
+            swait(S_M45, ci - 2);             // M4/M5 of chunk ci - 2 have read Kl and P (buffer par)
+            if (Rb == 0 && hh == 0) {  // the pass over R: f_s, f_r; the factor that restores S^T after this chunk
+                float fs[4], fr[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float h0 = xtot[0 * D + c0 + e], h1 = xtot[1 * D + c0 + e];
+                    const float h2 = xtot[2 * D + c0 + e], h3 = xtot[3 * D + c0 + e];
+                    if (fast) {
+                        fs[e] = fr[e] = ecm_prev[e] * ptx::ex2_approx(h0 + h1);
+                        ecm_prev[e] = ptx::ex2_approx(h2 + h3);
+                    } else {
+                        fs[e] = ecm_prev[e];
+                        fr[e] = ecm_prev[e] * ptx::ex2_approx(h0 + h1 + h2 + h3);
+                        ecm_prev[e] = 1.f;
+                    }
+                }
+                *reinterpret_cast<float4 *>(vec(par, VEC_FS) + c0) = make_float4(fs[0], fs[1], fs[2], fs[3]);
+                *reinterpret_cast<float4 *>(vec(par, VEC_FR) + c0) = make_float4(fr[0], fr[1], fr[2], fr[3]);
+            }
+            if (pt == 0) flags[8 + par] = fast ? 1 : 0;
             auto st4 = [&](uint32_t off, float x0, float x1, float x2, float x3) {
                 *reinterpret_cast<uint2 *>(sm + off) = make_uint2(pack_h2(x0, x1), pack_h2(x2, x3));
             };
@@ -777,66 +892,16 @@ __global__ void __launch_bounds__(NT, 1)
                 f[2] = bf16_lo(w.y);
                 f[3] = bf16_hi(w.y);
             };
-            {
-                float fKl[4], fKd[4], fKc[3][4];
+            if (fast) {
+                float off[4];  // g_r - g_m = (h_r within the block) + (totals before the block) - g_m
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    float after = 0.f;
+                    float before = 0.f;
 #pragma unroll
                     for (int R = 0; R < 4; ++R)
-                        if (R > Rb) after += xtot[R * D + c0 + e];
-                    fKl[e] = ptx::ex2_approx(after);
-                    // block Rb's own columns, e^{shift - h_i} = e^{s_i} e^{-shift}; zero past the bound
-                    // (the exact path recomputes that block)
-                    fKd[e] = Hb[e] >= -kShiftBound ? ptx::ex2_approx(-shift[e]) : 0.f;
-                    float between = 0.f;  // totals of the blocks strictly between Rb and Rb + 1 + k2
-#pragma unroll
-                    for (int k2 = 0; k2 < 3; ++k2) {
-                        const int R2 = Rb + 1 + k2;
-                        fKc[k2][e] = R2 < 4 ? ptx::ex2_approx(between + xtot[4 * D + (R2 & 3) * D + c0 + e]) : 0.f;
-                        if (R2 < 4) between += xtot[(R2 & 3) * D + c0 + e];
-                    }
+                        if (R < Rb) before += xtot[R * D + c0 + e];
+                    off[e] = pq[e] + before - (xtot[0 * D + c0 + e] + xtot[1 * D + c0 + e]);
                 }
-                float su[4] = {sq[0], sq[1], sq[2], sq[3]};  // sum after row j, within the block
-#pragma unroll
-                for (int j = 7; j >= 0; --j) {
-                    const int r = 16 * Rb + 8 * hh + j;
-                    const uint32_t o = sw(r, g4 >> 1) + ob;
-                    float kf[4];
-                    raw4(OFF_QK + bx * 16384 + o, r, kf);
-                    float base[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        base[e] = kf[e] * ptx::ex2_approx(su[e]);
-                        su[e] += la2[j][e];
-                    }
-                    st4(OFF_KL + par * 16384 + bx * 8192 + o, base[0] * fKl[0], base[1] * fKl[1], base[2] * fKl[2],
-                        base[3] * fKl[3]);
-                    st4(kc_off(Rb, bx) + o, base[0] * fKd[0], base[1] * fKd[1], base[2] * fKd[2], base[3] * fKd[3]);
-#pragma unroll
-                    for (int k2 = 0; k2 < 3; ++k2)
-                        if (Rb + 1 + k2 < 4)
-                            st4(kc_off(Rb + 1 + k2, bx) + o, base[0] * fKc[k2][0], base[1] * fKc[k2][1],
-                                base[2] * fKc[k2][2], base[3] * fKc[k2][3]);
-                }
-            }
-            {
-                float eMu[4], gam[4];  // Kg = Km e^{mu} with mu = (totals before the block) + shift
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float before = 0.f, all = 0.f;
-#pragma unroll
-                    for (int R = 0; R < 4; ++R) {
-                        const float t = xtot[R * D + c0 + e];
-                        if (R < Rb) before += t;
-                        all += t;
-                    }
-                    eMu[e] = ptx::ex2_approx(before + shift[e]);
-                    gam[e] = ptx::ex2_approx(all);
-                }
-                if (Rb == 0 && hh == 0)
-                    *reinterpret_cast<float4 *>(vec(par, VEC_GAM) + c0) = make_float4(gam[0], gam[1], gam[2], gam[3]);
-                float hr[4] = {pq[0], pq[1], pq[2], pq[3]};  // sum from the block's first token to row j
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int r = 16 * Rb + 8 * hh + j;
@@ -844,29 +909,112 @@ __global__ void __launch_bounds__(NT, 1)
                     float kf[4], qf[4];
                     raw4(OFF_QK + bx * 16384 + o, r, kf);
                     raw4(OFF_QK + bx * 16384 + 8192 + o, r, qf);
-                    float km[4], qm[4];
+                    float up[4], dn[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        hr[e] += la2[j][e];
-                        const float u = ptx::ex2_approx(hr[e] - shift[e]);
-                        km[e] = kf[e] * u;
-                        qm[e] = qf[e] * u;
+                        off[e] += la2[j][e];
+                        up[e] = ptx::ex2_approx(off[e]);
+                        dn[e] = ptx::ex2_approx(-off[e]);
                     }
-                    st4(OFF_QK + bx * 16384 + o, km[0], km[1], km[2], km[3]);
-                    st4(OFF_QK + bx * 16384 + 8192 + o, qm[0], qm[1], qm[2], qm[3]);
-                    st4(OFF_KQ + bx * 16384 + o, km[0] * eMu[0], km[1] * eMu[1], km[2] * eMu[2], km[3] * eMu[3]);
-                    st4(OFF_KQ + bx * 16384 + 8192 + o, qm[0] * eMu[0], qm[1] * eMu[1], qm[2] * eMu[2],
-                        qm[3] * eMu[3]);
+                    st4(OFF_KQ + bx * 16384 + o, kf[0] * up[0], kf[1] * up[1], kf[2] * up[2], kf[3] * up[3]);
+                    st4(OFF_KQ + bx * 16384 + 8192 + o, qf[0] * up[0], qf[1] * up[1], qf[2] * up[2], qf[3] * up[3]);
+                    st4(OFF_KL + par * 16384 + bx * 8192 + o, kf[0] * dn[0], kf[1] * dn[1], kf[2] * dn[2], kf[3] * dn[3]);
+                }
+            } else {
+                {
+                    float fKl[4], fKd[4], fKc[3][4];
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float after = 0.f;
+    #pragma unroll
+                        for (int R = 0; R < 4; ++R)
+                            if (R > Rb) after += xtot[R * D + c0 + e];
+                        fKl[e] = ptx::ex2_approx(after);
+                        // block Rb's own columns, e^{shift - h_i} = e^{s_i} e^{-shift}; zero past the bound
+                        // (the exact path recomputes that block)
+                        fKd[e] = Hb[e] >= -kShiftBound ? ptx::ex2_approx(-shift[e]) : 0.f;
+                        float between = 0.f;  // totals of the blocks strictly between Rb and Rb + 1 + k2
+    #pragma unroll
+                        for (int k2 = 0; k2 < 3; ++k2) {
+                            const int R2 = Rb + 1 + k2;
+                            fKc[k2][e] = R2 < 4 ? ptx::ex2_approx(between + xtot[4 * D + (R2 & 3) * D + c0 + e]) : 0.f;
+                            if (R2 < 4) between += xtot[(R2 & 3) * D + c0 + e];
+                        }
+                    }
+                    float su[4] = {sq[0], sq[1], sq[2], sq[3]};  // sum after row j, within the block
+    #pragma unroll
+                    for (int j = 7; j >= 0; --j) {
+                        const int r = 16 * Rb + 8 * hh + j;
+                        const uint32_t o = sw(r, g4 >> 1) + ob;
+                        float kf[4];
+                        raw4(OFF_QK + bx * 16384 + o, r, kf);
+                        float base[4];
+    #pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            base[e] = kf[e] * ptx::ex2_approx(su[e]);
+                            su[e] += la2[j][e];
+                        }
+                        st4(OFF_KL + par * 16384 + bx * 8192 + o, base[0] * fKl[0], base[1] * fKl[1], base[2] * fKl[2],
+                            base[3] * fKl[3]);
+                        st4(kc_off(Rb, bx) + o, base[0] * fKd[0], base[1] * fKd[1], base[2] * fKd[2], base[3] * fKd[3]);
+    #pragma unroll
+                        for (int k2 = 0; k2 < 3; ++k2)
+                            if (Rb + 1 + k2 < 4)
+                                st4(kc_off(Rb + 1 + k2, bx) + o, base[0] * fKc[k2][0], base[1] * fKc[k2][1],
+                                    base[2] * fKc[k2][2], base[3] * fKc[k2][3]);
+                    }
+                }
+                {
+                    float eMu[4];  // Kg = Km e^{mu} with mu = (totals before the block) + shift
+    #pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float before = 0.f;
+    #pragma unroll
+                        for (int R = 0; R < 4; ++R)
+                            if (R < Rb) before += xtot[R * D + c0 + e];
+                        eMu[e] = ptx::ex2_approx(before + shift[e]);
+                    }
+                    float hr[4] = {pq[0], pq[1], pq[2], pq[3]};  // sum from the block's first token to row j
+    #pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int r = 16 * Rb + 8 * hh + j;
+                        const uint32_t o = sw(r, g4 >> 1) + ob;
+                        float kf[4], qf[4];
+                        raw4(OFF_QK + bx * 16384 + o, r, kf);
+                        raw4(OFF_QK + bx * 16384 + 8192 + o, r, qf);
+                        float km[4], qm[4];
+    #pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            hr[e] += la2[j][e];
+                            const float u = ptx::ex2_approx(hr[e] - shift[e]);
+                            km[e] = kf[e] * u;
+                            qm[e] = qf[e] * u;
+                        }
+                        st4(OFF_QK + bx * 16384 + o, km[0], km[1], km[2], km[3]);
+                        st4(OFF_QK + bx * 16384 + 8192 + o, qm[0], qm[1], qm[2], qm[3]);
+                        st4(OFF_KQ + bx * 16384 + o, km[0] * eMu[0], km[1] * eMu[1], km[2] * eMu[2], km[3] * eMu[3]);
+                        st4(OFF_KQ + bx * 16384 + 8192 + o, qm[0] * eMu[0], qm[1] * eMu[1], qm[2] * eMu[2],
+                            qm[3] * eMu[3]);
+                    }
                 }
             }
             if (pt < C) vec(par, VEC_BETA)[pt] = beta_reg;
             ptx::fence_proxy_async_smem();
             if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
 
-            // ---- M1: [A; P]^raw of block R = [Km; Qm] Kc^(R)T, R = 0..3
+            // ---- M1: fast, [A; P]^raw = [Kt; Qt] Kb^T (N = 64); otherwise, block R's rows of
+            // [Km; Qm] Kc^(R)T for R = 0..3 (N = 16 (R + 1))
             if (leader) {
-                ptx::st_release(cnt + CNT_P2, ci + 1);  // [Kg; Qg], e^{g_L}, beta of chunk ci
+                if (fast && ci + 1 < nchunks) load_qk(s + C);  // the raw k|q tile has been read
                 ptx::tc_fence_after();
+                if (fast) {
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t ka = uint32_t(ks >> 2) * 16384u + uint32_t(ks & 3) * 32u;
+                        const uint32_t kb = OFF_KL + par * 16384 + uint32_t(ks >> 2) * 8192u + uint32_t(ks & 3) * 32u;
+                        ptx::mma_ss(tbase + TAP, ptx::sdesc_sw128(sb + OFF_KQ + ka), ptx::sdesc_sw128(sb + kb), IDESC_N64,
+                                    ks > 0);
+                    }
+                } else {
                 for (int R = 0; R < 4; ++R) {
                     const uint32_t idesc = ptx::idesc_f16_f32(128, 16 * (R + 1));
                     for (int ks = 0; ks < 8; ++ks) {
@@ -876,17 +1024,81 @@ __global__ void __launch_bounds__(NT, 1)
                                     ptx::sdesc_sw128(sb + kb), idesc, ks > 0);
                     }
                 }
+                }
                 commit(B_M1);
+                // then the state group's M2 may follow on the tensor pipe
+                sarrive(S_P2, ci);  // the operand rows, f_s, f_r, beta of chunk ci
                 if (ci + 2 < nchunks) prefetch_l2(ci + 2);
             }
             mwait(B_M1, ci, leader);
             ptx::tc_fence_after();
-            if (leader && has_next) load_qk(s + C);  // [Km; Qm] has been read
+            if (leader && !fast && ci + 1 < nchunks) load_qk(s + C);  // M1 has read [Km; Qm] (over the raw tile)
 
             // ---- E1: A rows -> fp32 (beta_r, i < r) over the previous chunk's X, P rows -> fp16
             // operand (i <= r, zeros above; buffer par, last read by M5 of chunk ci - 2).
-            if (ci >= 1) cwait(CNT_TW, ci);  // the state group has formed T from X of chunk ci - 1
-            {
+            swait(S_TW, ci - 1);  // the state group has formed T from X of chunk ci - 1
+            if (fast) {  // every row's 64 columns: lane quarter qd, columns 32 half .. 32 half + 31
+                const int qd = warp & 3, half = pw >> 2;
+                const int trow = qd * 32 + lane;
+                uint32_t v[32];
+                ptx::tmem_ld32(tbase + (uint32_t(qd * 32) << 16) + TAP + 32 * half, v);
+                ptx::tmem_wait_ld();
+                if (qd < 2) {
+                    const int r = trow;
+                    const float br = vec(par, VEC_BETA)[r];
+                    float *af = reinterpret_cast<float *>(sm + OFF_AX) + r * LDF + 32 * half;
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        float4 x;
+                        const int i = 32 * half + e;
+                        x.x = (i + 0 < r) ? br * __uint_as_float(v[e + 0]) : 0.f;
+                        x.y = (i + 1 < r) ? br * __uint_as_float(v[e + 1]) : 0.f;
+                        x.z = (i + 2 < r) ? br * __uint_as_float(v[e + 2]) : 0.f;
+                        x.w = (i + 3 < r) ? br * __uint_as_float(v[e + 3]) : 0.f;
+                        *reinterpret_cast<float4 *>(af + e) = x;
+                    }
+                } else {
+                    const int r = trow - 64;
+                    uint8_t *pt_tile = sm + OFF_P + par * 8192;
+#pragma unroll
+                    for (int qq = 0; qq < 4; ++qq) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            const int e = 8 * qq + 2 * e2, i = 32 * half + e;
+                            pk[e2] = pack_h2(i <= r ? __uint_as_float(v[e]) : 0.f,
+                                             i + 1 <= r ? __uint_as_float(v[e + 1]) : 0.f);
+                        }
+                        *reinterpret_cast<uint4 *>(pt_tile + sw(r, 4 * half + qq)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+                // the warps that wrote the diagonal 16x16 blocks of A (rows and columns 0-31:
+                // prep warp 0; 32-63: prep warp 5) invert them at once
+                const float *Af = reinterpret_cast<const float *>(sm + OFF_AX);
+                float *X = reinterpret_cast<float *>(sm + OFF_AX);
+                if (pw == 0 || pw == 5) {  // the warps whose E1 wrote the diagonal blocks: 0, 1 and 2, 3
+                    const int b = (pw == 0 ? 0 : 2) + (lane >> 4), jj = lane & 15;
+                    const float *ab = Af + (16 * b) * LDF + 16 * b;
+                    float x[16];
+                    __syncwarp();  // this warp's A rows are written
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) {  // x_rr = [rr == jj] - sum_{ss < rr} A_bb[rr][ss] x_ss
+                        float acc = (rr == jj) ? 1.f : 0.f;
+#pragma unroll
+                        for (int s4 = 0; s4 < rr; s4 += 4) {
+                            const float4 a4 = *reinterpret_cast<const float4 *>(ab + rr * LDF + s4);
+                            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                if (s4 + u < rr) acc = fmaf(-av[u], x[s4 + u], acc);
+                        }
+                        x[rr] = acc;
+                    }
+                    __syncwarp();  // every lane has read its A_bb
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) X[(16 * b + rr) * LDF + 16 * b + jj] = x[rr];
+                }
+            } else {
                 float *Af = reinterpret_cast<float *>(sm + OFF_AX);
                 uint8_t *pt_tile = sm + OFF_P + par * 8192;
                 const int qdt = warp & 3;                 // TMEM lane quarter of this warp
@@ -949,10 +1161,10 @@ __global__ void __launch_bounds__(NT, 1)
             // pairs, P_ri = <q_r, k_i prod_{i<t<=r} alpha_t> and A_ri = beta_r <k_r, ...>, from the
             // rows in L2 (fp32, running products), over the values E1 wrote.  Partial sums per
             // (block, channel box) go to the T tile, free once M3 of chunk ci - 1 has read it.
-            if (any_bad) {
+            if (!fast && any_bad) {
                 float *part = reinterpret_cast<float *>(sm + OFF_T);  // [block][box][256]
-                cwait(CNT_M45, ci);
-                if (flags[2 * Rb] | flags[2 * Rb + 1])  // uniform over the warp
+                swait(S_M45, ci - 1);
+                if ((flags[2 * Rb] | flags[2 * Rb + 1]) & 1)  // uniform over the warp
                     exact_block_partials(part + (Rb * 2 + bx) * 256, static_cast<const __nv_bfloat16 *>(a.k),
                                          static_cast<const __nv_bfloat16 *>(a.q), a.log_alpha, H, s, L, h, Rb, bx, lane);
                 ptx::named_barrier(BAR_P, NP);
@@ -960,7 +1172,7 @@ __global__ void __launch_bounds__(NT, 1)
                 uint8_t *pt_tile = sm + OFF_P + par * 8192;
                 const int rl = pt >> 4, il = pt & 15;
                 for (int R = 0; R < 4; ++R) {
-                    if (!(flags[2 * R] | flags[2 * R + 1]) || il > rl) continue;
+                    if (!((flags[2 * R] | flags[2 * R + 1]) & 1) || il > rl) continue;
                     const int r = 16 * R + rl, i = 16 * R + il;
                     const float *p0 = part + (R * 2) * 256, *p1 = p0 + 256;
                     const int vp = diag_run_start(il) + 2 * (rl - il);
@@ -982,30 +1194,31 @@ __global__ void __launch_bounds__(NT, 1)
                 const float *Af = reinterpret_cast<const float *>(sm + OFF_AX);
                 float *X = reinterpret_cast<float *>(sm + OFF_AX);
                 float *E = reinterpret_cast<float *>(sm + OFF_EB);
-                if (pw < 4) {
-                    const int b = pw, jj = lane & 15;
-                    const float *ab = Af + (16 * b) * LDF + 16 * b;
-                    float x[16];
+                if (!fast) {  // after the exact path; fast chunks inverted the blocks right after E1
+                    if (pw == 0 || pw == 5) {  // the warps whose E1 wrote the diagonal blocks: 0, 1 and 2, 3
+                        const int b = (pw == 0 ? 0 : 2) + (lane >> 4), jj = lane & 15;
+                        const float *ab = Af + (16 * b) * LDF + 16 * b;
+                        float x[16];
+                        __syncwarp();  // this warp's A rows are written
 #pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) {  // x_rr = [rr == jj] - sum_{ss < rr} A_bb[rr][ss] x_ss
-                        float acc = (rr == jj) ? 1.f : 0.f;
+                        for (int rr = 0; rr < 16; ++rr) {  // x_rr = [rr == jj] - sum_{ss < rr} A_bb[rr][ss] x_ss
+                            float acc = (rr == jj) ? 1.f : 0.f;
 #pragma unroll
-                        for (int s4 = 0; s4 < rr; s4 += 4) {
-                            const float4 a4 = *reinterpret_cast<const float4 *>(ab + rr * LDF + s4);
-                            const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+                            for (int s4 = 0; s4 < rr; s4 += 4) {
+                                const float4 a4 = *reinterpret_cast<const float4 *>(ab + rr * LDF + s4);
+                                const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                if (s4 + u < rr) acc = fmaf(-av[u], x[s4 + u], acc);
+                                for (int u = 0; u < 4; ++u)
+                                    if (s4 + u < rr) acc = fmaf(-av[u], x[s4 + u], acc);
+                            }
+                            x[rr] = acc;
                         }
-                        x[rr] = acc;
-                    }
-                    __syncwarp();  // every lane has read A_bb
-                    if (lane < 16) {
+                        __syncwarp();  // every lane has read its A_bb
 #pragma unroll
                         for (int rr = 0; rr < 16; ++rr) X[(16 * b + rr) * LDF + 16 * b + jj] = x[rr];
                     }
+                    ptx::named_barrier(BAR_P, NP);
                 }
-                ptx::named_barrier(BAR_P, NP);
                 {  // E_h = X_{b1 b1} A_{b1 b0} (16x16, h = 0: b = 1, 0; h = 1: b = 3, 2); two columns a thread.
                    // Diagonal blocks of X hold zeros above their diagonal.
                     const int hh = pt >> 7, r = (pt >> 3) & 15, c2 = 2 * (pt & 7);
@@ -1035,66 +1248,20 @@ __global__ void __launch_bounds__(NT, 1)
                     *reinterpret_cast<float2 *>(X + (16 * b1 + r) * LDF + 16 * b0 + c2) = make_float2(-a0, -a1);
                 }
                 ptx::named_barrier(BAR_P, NP);
-                {  // F = X_H1 A_21 (32x32; X_H1 = X[32:64, 32:64] is zero above its diagonal, and
-                   // its upper-right 16x16 block is never read); F[r][c] at E[r * LDG + c]
-                    const int r = pt >> 3, c4 = 4 * (pt & 7);
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                    const float *xr = X + (32 + r) * LDF + 32;
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        const float xv = xr[m];
-                        const float4 av = *reinterpret_cast<const float4 *>(Af + (32 + m) * LDF + c4);
-                        acc[0] = fmaf(xv, av.x, acc[0]);
-                        acc[1] = fmaf(xv, av.y, acc[1]);
-                        acc[2] = fmaf(xv, av.z, acc[2]);
-                        acc[3] = fmaf(xv, av.w, acc[3]);
-                    }
-                    if (r >= 16) {  // uniform over a warp
-#pragma unroll
-                        for (int m = 16; m < 32; ++m) {
-                            const float xv = xr[m];
-                            const float4 av = *reinterpret_cast<const float4 *>(Af + (32 + m) * LDF + c4);
-                            acc[0] = fmaf(xv, av.x, acc[0]);
-                            acc[1] = fmaf(xv, av.y, acc[1]);
-                            acc[2] = fmaf(xv, av.z, acc[2]);
-                            acc[3] = fmaf(xv, av.w, acc[3]);
-                        }
-                    }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) E[r * LDG + c4 + q] = acc[q];
-                }
-                ptx::named_barrier(BAR_P, NP);
-                {  // X_21 = -F X_H0 (X_H0 = X[0:32, 0:32]; its upper-right block is never read)
-                    const int r = pt & 31, c4 = 4 * (pt >> 5);
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                    const float *fr = E + r * LDG;
-                    if (c4 < 16) {  // uniform over a warp
-#pragma unroll
-                        for (int m = 0; m < 16; ++m) {
-                            const float fv = fr[m];
-                            const float4 xv = *reinterpret_cast<const float4 *>(X + m * LDF + c4);
-                            acc[0] = fmaf(fv, xv.x, acc[0]);
-                            acc[1] = fmaf(fv, xv.y, acc[1]);
-                            acc[2] = fmaf(fv, xv.z, acc[2]);
-                            acc[3] = fmaf(fv, xv.w, acc[3]);
-                        }
-                    }
-#pragma unroll
-                    for (int m = 16; m < 32; ++m) {
-                        const float fv = fr[m];
-                        const float4 xv = *reinterpret_cast<const float4 *>(X + m * LDF + c4);
-                        acc[0] = fmaf(fv, xv.x, acc[0]);
-                        acc[1] = fmaf(fv, xv.y, acc[1]);
-                        acc[2] = fmaf(fv, xv.z, acc[2]);
-                        acc[3] = fmaf(fv, xv.w, acc[3]);
-                    }
-                    *reinterpret_cast<float4 *>(X + (32 + r) * LDF + c4) = make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
-                }
-                ptx::named_barrier(BAR_P, NP);
             }
-            // X (fp32) is handed to the state group, which forms T = X Diag(beta)
+            // X but its lower-left 32x32 block (fp32) is handed to the state group, which completes
+            // it (X_21) and forms T = X Diag(beta)
             if (ptx::named_barrier_or(BAR_P, NP, *s_abort != 0)) break;
-            if (leader) ptx::st_release(cnt + CNT_TP, ci + 1);
+            if (leader) sarrive(S_TP, ci);
+        }
+        // the factor that restores S^T from TMEM after the last chunk, in the vector buffer the
+        // state group read two chunks ago
+        if (!*reinterpret_cast<volatile int *>(s_abort)) {
+            if (Rb == 0 && hh == 0)
+                *reinterpret_cast<float4 *>(vec(nchunks & 1, VEC_FR) + c0) =
+                    make_float4(ecm_prev[0], ecm_prev[1], ecm_prev[2], ecm_prev[3]);
+            ptx::named_barrier(BAR_P, NP);
+            if (leader) sarrive(S_P2, nchunks);
         }
     }
 

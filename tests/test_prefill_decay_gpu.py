@@ -142,3 +142,21 @@ def test_backward_strong_decay():
     for name, r in ref.items():
         assert torch.isfinite(g[name]).all(), name
         assert rel_l2(host64(g[name]), r) <= 1e-5, name
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_mild_and_strong_chunks_alternate(dtype):
+    """Decay strength changes along the sequence (mild 64-token stretches between strong
+    ones, erased channels only in the strong ones): the tensor-core path switches its
+    factoring from chunk to chunk and must carry the state across every switch."""
+    lens = [64 * 7 - 9, 150]
+    T = sum(lens)
+    per_tok = torch.tensor(([0.1] * 64 + [4.0] * 64 + [0.1] * 128 + [16.0] * 64 + [0.1] * 64 + [1.0] * 64)[:lens[0]]
+                           + [0.1] * 70 + [4.0] * 80, dtype=torch.float32)
+    inp = _inp(lens, 2, 128, 128, dtype, 1.0)
+    la = inputs.decay_log_alpha(T, 2, 128, per_tok.view(T, 1, 1).to(DEV), 0.0, seed=66, device=DEV)
+    zeros = inputs.decay_log_alpha(T, 2, 128, 1.0, 0.02, seed=67, device=DEV)
+    strong = (per_tok > 0.5).view(T, 1, 1).to(DEV)
+    inp["log_alpha"] = torch.where(strong & torch.isinf(zeros), zeros, la).contiguous()
+    o, S = _prefill(inp)
+    compare_full(inp, o, S, dtype)
