@@ -64,8 +64,8 @@ def decode_bytes_per_head_step(dk, dv, qkv_bytes):
 # Prefill: one launch on 2 x 8192 tokens x 32 heads (524,288 head-tokens).
 MEASURED_TRAFFIC = {
     "prefill_tc": {"source": "gated_delta_rule_126_b200/csrc/kda_prefill_tc.cu",
-                   "sha256": "6bf2ede04c3e0659e3fcd1a4713a7362b0d853e12680aff369f01cd785c3365d",
-                   "units": 2 * 8192 * 32, "dram_bytes": 673465088 + 120951808},
+                   "sha256": "f9a4ef97c07e11e7f636d2b37a71992c14d7d5cda80bb7f21abc32f1907b343a",
+                   "units": 2 * 8192 * 32, "dram_bytes": 673443840 + 120949760},
 }
 
 
