@@ -64,7 +64,7 @@ def decode_bytes_per_head_step(dk, dv, qkv_bytes):
 # Prefill: one launch on 2 x 8192 tokens x 32 heads (524,288 head-tokens).
 MEASURED_TRAFFIC = {
     "prefill_tc": {"source": "gated_delta_rule_126_b200/csrc/kda_prefill_tc.cu",
-                   "sha256": "f9a4ef97c07e11e7f636d2b37a71992c14d7d5cda80bb7f21abc32f1907b343a",
+                   "sha256": "7a13a8e29c214c4bb30f78e92bfa9759e6c71ca222c8e86455d67855232c77c7",
                    "units": 2 * 8192 * 32, "dram_bytes": 673443840 + 120949760},
 }
 

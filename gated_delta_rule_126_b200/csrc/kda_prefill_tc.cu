@@ -13,41 +13,50 @@
 // Decay range.  The section's channel-wise decay bullet allows any alpha in [0, 1],
 // alpha = 0 (log alpha = -inf) included, so every exponent here is a sum of log alpha
 // over the tokens it spans (never -inf - -inf) and every tensor-core operand stays in
-// fp16 range:
-// * The chunk is cut into four 16-token blocks.  In block R, h_r sums log alpha from
-//   the block's first token to r, s_r over the tokens after r to the block's end, H_R
-//   is the block total.  Each block takes a reference point mu_R = (end of block R-1)
-//   + shift_R with shift_R = H_R / 2 for channels whose block decay stays within
-//   2^{-16} (|H_R| <= 16 in base 2), else 0.
-// * Rows:     Km = K e^{h - shift}, Qm = Q e^{h - shift}            (<= 2^8 |k|)
-//   Columns:  Kc^(R)_i = K_i e^{mu_R - g_i}, i < 16 (R + 1): <= 1 for i in earlier
-//   blocks, within 2^{+-8} in block R (zero for channels past the bound).
-//   M1 issues one MMA per row block R (N = 16, 32, 48, 64); block R's rows of its
-//   output are A and P.
-// * A block whose decay leaves that bound in any channel has its own 16 x 16 pairs
-//   recomputed exactly on CUDA cores (products of the alphas between the two tokens,
-//   reloaded from L2), over the tensor-core values.
-// * State products from the chunk start: Kg = K e^{g}, Qg = Q e^{g}, Kl = K e^{g_L - g},
-//   all <= |k|; TMEM holds S^T itself.
+// fp16 range.  The chunk is cut into four 16-token blocks; H_R is block R's total (base
+// 2) per channel.  Each chunk takes one of two forms, chosen by the prep group from the
+// block totals (a vote over all channels):
+// * Fast form, when every block total is >= -kFastBound (2^-5) in every channel: the
+//   decays are factored at g_m, the running sum at the end of block 1 (mid-chunk):
+//     Kt = K e^{g - g_m}, Qt = Q e^{g - g_m}, Kb = K e^{g_m - g}   (factors within 2^{+-10})
+//     M1  [A; P]^raw = [Kt; Qt] Kb^T   (N = 64),
+//   the state's products use Kt, Qt and Kb (M2 = Sop [Kt; Qt]^T, M4 += U^T Kb), and TMEM
+//   carries S^T Diag(e^{g_m - g_L}) out of the chunk; the pass over R at the start of the
+//   next chunk folds the factor back.
+// * Block-reference form otherwise.  In block R, h_r sums log alpha from the block's
+//   first token to r, s_r over the tokens after r to the block's end.  Each block takes a
+//   reference point mu_R = (end of block R-1) + shift_R with shift_R = H_R / 2 for
+//   channels whose block decay stays within 2^{-16} (|H_R| <= kShiftBound), else 0.
+//     Rows:     Km = K e^{h - shift}, Qm = Q e^{h - shift}            (<= 2^8 |k|)
+//     Columns:  Kc^(R)_i = K_i e^{mu_R - g_i}, i < 16 (R + 1): <= 1 for i in earlier
+//               blocks, within 2^{+-8} in block R (zero for channels past the bound).
+//   M1 issues one MMA per row block R (N = 16, 32, 48, 64); block R's rows of its output
+//   are A and P.  A block whose decay leaves that bound in any channel has its own
+//   16 x 16 pairs recomputed exactly on CUDA cores (products of the alphas between the
+//   two tokens, with k, q and log alpha reloaded from L2), over the tensor-core values.
+//   The state products run from the chunk start: Kg = K e^{g}, Qg = Q e^{g},
+//   Kl = K e^{g_L - g}, all <= |k|, and TMEM holds S^T itself.
 //
 // Design (one CTA of 384 threads per (sequence, head), walking its chunks):
 // * The fp32 state is kept TRANSPOSED in tensor memory (lane = value column j) for
 //   the whole sequence, so every state product is a 128-row UMMA with d_v on M:
-//     M1  [A; P]^raw = [Km; Qm] Kc^(R)T        M=128 N=16(R+1) K=128, R = 0..3
-//     M2  Z          = Sop [Kg; Qg]^T          M=128 N=128 K=128 (Sop = fp16 S^T)
-//           Z[:, :64] = (Kg S)^T,  Z[:, 64:] = (Qg S)^T
+//     M1  [A; P]^raw   (fast: N=64 K=128; block-reference: N=16(R+1) K=128, R = 0..3)
+//     M2  Z          = Sop [Kg; Qg]^T          M=128 N=128 K=128 (Sop = fp16 of R scaled)
+//           Z[:, :64] = (Kg S)^T,  Z[:, 64:] = (Qg S)^T     (Kt, Qt in the fast form)
 //     Mv  Z[:, :64] += V^T (-I)     (V read MN-major from its TMA tile)   N=64 K=64
 //     M3  U^T        = Y^T T^T  -> Z[:, :64],  Y^T = -Z[:, :64]    N=64 K=64
-//     M4  R         += U^T Kl      (Kl read as an MN-major operand)  N=128 K=64
+//     M4  R         += U^T Kl      (Kl, or Kb, read as an MN-major operand)  N=128 K=64
 //     M5  Z[:, 64:] += U^T P^T  ( = O^T )                   N=64  K=64
-//   The pass over R at the start of a chunk packs Sop and multiplies R by e^{g_L}.
+//   The pass over R at the start of a chunk packs Sop = fp16(R f_s) and sets R <- R f_r,
+//   with per-channel factors the prep group derives from the block totals for the pair
+//   of chunk forms (previous, current).
 // * Two warp groups work on different chunks at once.  The prep group (warps 4-11)
-//   builds chunk c + 1 -- the block sums and the fp16 operand rows (Km, Qm over the
-//   raw k|q tile, Kg, Qg, Kl, Kc), M1, A and P, and X = (I + A)^{-1} in place -- while
-//   the state group (warps 0-3) runs chunk c -- the pass over R, M2, Y, T = X
-//   Diag(beta), M3, U, M4/M5 and the outputs.  They hand buffers over through
-//   release/acquire progress counters in shared memory; Kl and P are double-buffered
-//   by chunk parity.
+//   builds chunk c + 1 -- the block sums, the form vote, the fp16 operand rows over the
+//   raw k|q tile, M1, A and P, the exact blocks, and X = (I + A)^{-1} in place but its
+//   lower-left 32 x 32 block -- while the state group (warps 0-3) runs chunk c -- the
+//   pass over R, M2, Y, X_21 = -(X_H1 A_21) X_H0 and T = X Diag(beta), M3, U, M4/M5 and
+//   the outputs.  They hand buffers over through thread-arrive mbarriers, one per signal
+//   and chunk parity; Kl/Kb and P are double-buffered by chunk parity.
 // * Operands are fp16 (fp32 accumulation): the S-dependent chain keeps the relative
 //   error near fp16's 2^-11, which the parity bounds need (bf16 operands do not meet
 //   them).
