@@ -24,10 +24,11 @@
 //   1. states: the forward sweep, storing w_t for every token and the state before
 //      every 32nd token of each sequence (checkpoints); each 32-token block's alpha
 //      and k rows are staged in shared memory first;
-//   2. grads:  the backward sweep, 32-token blocks from the last: the 4-token
-//      sub-blocks (last first) are replayed with the stored w (no reduction needed)
-//      from the block's checkpoint or, past the middle, from the state before the
-//      block's 16th token, their input states kept in shared memory;
+//   2. grads:  the backward sweep, 32-token blocks from the last: each block's alpha
+//      and k rows are staged in shared memory first (off the per-token critical path);
+//      the 4-token sub-blocks (last first) are replayed with the stored w (no reduction
+//      needed) from the block's checkpoint or, past the middle, from the state before
+//      the block's 16th token, their input states kept in shared memory;
 //   3. reduce: sums the slices' partial dq, dk, dlog_alpha and dbeta.
 // CUDA cores in fp32 throughout; no tensor cores and no waits on other blocks.
 #include <algorithm>
@@ -211,8 +212,12 @@ __global__ void __launch_bounds__(kRows) bwd_states_kernel(const BwdArgs a) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kRows, 4) bwd_grads_kernel(const BwdArgs a) {
+__global__ void __launch_bounds__(kRows, 3) bwd_grads_kernel(const BwdArgs a) {
     __shared__ float4 hist[kSub][4][kRows];  // input states of the sub-block's tokens (own rows)
+    // alpha and k of the block's tokens (each thread its own row), in dynamic shared memory
+    extern __shared__ __align__(16) uint8_t bwd_dyn[];
+    float(*als)[kRows] = reinterpret_cast<float(*)[kRows]>(bwd_dyn);
+    T(*ks)[kRows] = reinterpret_cast<T(*)[kRows]>(bwd_dyn + kBlk * kRows * sizeof(float));
     __shared__ float4 midst[4][kRows];       // state before the block's middle token (own rows)
     __shared__ float4 red[2][4][4];
     __shared__ float ws[kBlk][kCols], dos[kBlk][kCols];
@@ -244,13 +249,17 @@ __global__ void __launch_bounds__(kRows, 4) bwd_grads_kernel(const BwdArgs a) {
             dos[tt][j] = (in && u.c0 + j < dv) ? ldf(dop + ((t0 + tt) * H + u.h) * dv + u.c0 + j) : 0.f;
         }
         if (i < kBlk) bs[i] = i < n ? a.beta[(t0 + i) * H + u.h] : 0.f;
+        for (int tt = 0; tt < n; ++tt) {  // each thread its own row: no barrier needed for these
+            const int64_t r = ((t0 + tt) * H + u.h) * dk + i;
+            als[tt][i] = row ? expf(a.log_alpha[r]) : 1.f;
+            ks[tt][i] = row ? kp[r] : T(0.f);
+        }
         __syncthreads();
         const float4 *ckp = ck_slice(a, u, bi);
         // S <- Diag(alpha_tt) S + beta_tt k_tt w_tt^T, from the stored w
         auto replay = [&](float(&S)[kCols], int tt) {
-            const int64_t r = ((t0 + tt) * H + u.h) * dk + i;
-            const float al = row ? expf(a.log_alpha[r]) : 1.f;
-            const float kb = row ? ldf(kp + r) * bs[tt] : 0.f;
+            const float al = als[tt][i];
+            const float kb = ldf(&ks[tt][i]) * bs[tt];
 #pragma unroll
             for (int j = 0; j < kCols; ++j) S[j] = fmaf(kb, ws[tt][j], al * S[j]);
         };
@@ -289,9 +298,8 @@ __global__ void __launch_bounds__(kRows, 4) bwd_grads_kernel(const BwdArgs a) {
                     for (int q4 = 0; q4 < 4; ++q4)
                         hist[tt - first][q4][i] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
                 }
-                const int64_t r = ((t0 + tt) * H + u.h) * dk + i;
-                const float al = row ? expf(a.log_alpha[r]) : 1.f;
-                const float kb = row ? ldf(kp + r) * bs[tt] : 0.f;
+                const float al = als[tt][i];
+                const float kb = ldf(&ks[tt][i]) * bs[tt];
 #pragma unroll
                 for (int j = 0; j < kCols; ++j) S[j] = fmaf(kb, ws[tt][j], al * S[j]);
             }
@@ -303,9 +311,9 @@ __global__ void __launch_bounds__(kRows, 4) bwd_grads_kernel(const BwdArgs a) {
             for (int m = kSub - 1; m >= 0; --m) {
                 if (m >= m_n) continue;
                 const int tt = first + m;
-                const int64_t t = t0 + tt, r = (t * H + u.h) * dk + i;
-                const float al = row ? expf(a.log_alpha[r]) : 1.f;
-                const float kk = row ? ldf(kp + r) : 0.f;
+                const int64_t t = t0 + tt;
+                const float al = als[tt][i];
+                const float kk = ldf(&ks[tt][i]);
                 const float qq = qpre[m];
                 const float b = bs[tt];
                 float P[kCols], c[kCols];
@@ -378,7 +386,10 @@ template <typename T>
 cudaError_t launch_backward_t(const BwdArgs &a, cudaStream_t st) {
     const unsigned grid = unsigned(int64_t(a.num_seqs) * a.H * a.nsl);
     bwd_states_kernel<T><<<grid, kRows, 0, st>>>(a);
-    bwd_grads_kernel<T><<<grid, kRows, 0, st>>>(a);
+    constexpr int dyn = kBlk * kRows * int(sizeof(float) + sizeof(T));
+    cudaError_t err = cudaFuncSetAttribute(bwd_grads_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+    if (err != cudaSuccess) return err;
+    bwd_grads_kernel<T><<<grid, kRows, dyn, st>>>(a);
     if (a.T > 0) {
         const int64_t n = a.T * a.H * a.dk;
         const unsigned rg = unsigned(std::min<int64_t>((n + 255) / 256, int64_t(kda::device_sm_count()) * 16));
