@@ -336,9 +336,12 @@ def run_reference(args):
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
+    total_tokens = sum(w.seqlens)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": total_tokens / value * 1e3,
+            "ms_per_step_basis": "the workload's tokens at the sample's rate (each step times a bounded sample)",
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, world), "sample": sample,
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
