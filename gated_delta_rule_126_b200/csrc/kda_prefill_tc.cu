@@ -55,8 +55,9 @@
 //   raw k|q tile, M1, A and P, the exact blocks, and X = (I + A)^{-1} in place but its
 //   lower-left 32 x 32 block -- while the state group (warps 0-3) runs chunk c -- the
 //   pass over R, M2, Y, X_21 = -(X_H1 A_21) X_H0 and T = X Diag(beta), M3, U, M4/M5 and
-//   the outputs.  They hand buffers over through thread-arrive mbarriers, one per signal
-//   and chunk parity; Kl/Kb and P are double-buffered by chunk parity.
+//   the outputs.  X_21 and T are formed while M2 runs.  The groups hand buffers over
+//   through thread-arrive mbarriers, one per signal and chunk parity, and the MMAs'
+//   completion barriers; Kl/Kb and P are double-buffered by chunk parity.
 // * Operands are fp16 (fp32 accumulation): the S-dependent chain keeps the relative
 //   error near fp16's 2^-11, which the parity bounds need (bf16 operands do not meet
 //   them).
@@ -115,12 +116,13 @@ constexpr int B_QK = 0, B_V = 1, B_M1 = 2, B_M2 = 3, B_M3 = 4, B_M45 = 5, B_G = 
 // signal of chunk c completes phase c >> 1 of barrier 2 * signal + (c & 1).  No producer can
 // complete chunk c + 2's phase before the consumer has waited for chunk c's.
 constexpr uint32_t OFF_SIG = OFF_BAR + 8 * NBAR;
-constexpr int S_P2 = 0, S_KQF = 1, S_TP = 2, S_TW = 3, S_M45 = 4, NSIG = 5;
+constexpr int S_P2 = 0, S_TP = 1, S_TW = 2, S_M45 = 3, NSIG = 4;
 //   S_P2:  prep -> state: the operand rows, f_s, f_r and beta of chunk c (and M1 issued)
-//   S_KQF: state -> prep: M2 of chunk c has read [Kg; Qg]
 //   S_TP:  prep -> state: X of chunk c
 //   S_TW:  state -> prep: T of chunk c formed (X read)
 //   S_M45: state -> prep: M4/M5 of chunk c done (Kl, P of its parity and the T tile read)
+// The prep group learns that M2 of chunk c has read the K/Q operand tile from M2's own
+// completion barrier (B_M2), which the tensor core arrives on.
 constexpr uint32_t OFF_ISS = OFF_SIG + 8 * 2 * NSIG;    // phases issued / waited per mbarrier
 constexpr uint32_t OFF_WT = OFF_ISS + 4 * NBAR;
 constexpr uint32_t OFF_FLAG = OFF_WT + 4 * NBAR;        // per (block, channel box): bit 0 past the exact bound,
@@ -513,33 +515,8 @@ __global__ void __launch_bounds__(NT, 1)
                 }
                 commit(B_M2);
             }
-            mwait(B_M2, ci, leader);
-            ptx::tc_fence_after();
-            if (leader) {
-                sarrive(S_KQF, ci);  // [Kg; Qg] has been read
-                if (has_next && !v_zero) load_v(s + C);  // the V tile has been read by the MMA
-            }
-
-            // ---- E2: Y^T = -Z[:, :64] = V^T - (K e^{g} S)^T -> fp16 pairs in TMEM, the A
-            // operand of M3 (rows i >= L of V are never used: T's columns i >= L are zero).
-            {
-                uint32_t vz[2][32], pk[16];
-                ptx::tmem_ld32(tl + TZ, vz[0]);
-                ptx::tmem_ld32(tl + TZ + 32, vz[1]);
-                ptx::tmem_wait_ld();
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = pack_h2(-__uint_as_float(vz[p][2 * e]), -__uint_as_float(vz[p][2 * e + 1]));
-                    ptx::tmem_st16(tl + TY16 + 16 * p, pk);
-                }
-                ptx::tmem_wait_st();
-            }
-            ptx::tc_fence_before();
-            if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
-
-            // ---- M3: U^T = Y^T T^T into Z[:, :64] (T of this chunk from the prep group's X).
+            // ---- X_21 and T of this chunk (from the prep group's X) while M2 runs; then E2 and
+            // M3: U^T = Y^T T^T into Z[:, :64].
             swait(S_TP, ci);
             {  // X_21 = -(X_H1 A_21) X_H0 over 32x32 halves (X_H1 = X[32:64, 32:64] and X_H0 =
                // X[0:32, 0:32] are zero above their diagonals); F = X_H1 A_21 in fp32 over the T tile
@@ -614,8 +591,33 @@ __global__ void __launch_bounds__(NT, 1)
             }
             ptx::fence_proxy_async_smem();
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
+            if (leader) sarrive(S_TW, ci);  // T is formed: the prep group may overwrite X
+            mwait(B_M2, ci, leader);
+            ptx::tc_fence_after();
             if (leader) {
-                sarrive(S_TW, ci);
+                if (has_next && !v_zero) load_v(s + C);  // the V tile has been read by the MMA
+            }
+
+            // ---- E2: Y^T = -Z[:, :64] = V^T - (K e^{g} S)^T -> fp16 pairs in TMEM, the A
+            // operand of M3 (rows i >= L of V are never used: T's columns i >= L are zero).
+            {
+                uint32_t vz[2][32], pk[16];
+                ptx::tmem_ld32(tl + TZ, vz[0]);
+                ptx::tmem_ld32(tl + TZ + 32, vz[1]);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_h2(-__uint_as_float(vz[p][2 * e]), -__uint_as_float(vz[p][2 * e + 1]));
+                    ptx::tmem_st16(tl + TY16 + 16 * p, pk);
+                }
+                ptx::tmem_wait_st();
+            }
+            ptx::tc_fence_before();
+            if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
+
+            if (leader) {
                 ptx::tc_fence_after();
                 for (int ks = 0; ks < 4; ++ks)
                     ptx::mma_ts(tbase + TZ, tbase + TY16 + 8 * ks, ptx::sdesc_sw128(sb + OFF_T + 32 * ks), IDESC_N64,
@@ -870,7 +872,7 @@ __global__ void __launch_bounds__(NT, 1)
                 any_bad = any_bad || (flags[b] & 1) != 0;
                 fast = fast && (flags[b] & 2) == 0;
             }
-            swait(S_KQF, ci - 1);  // M2 of chunk ci - 1 has read the K/Q operand tile
+            if (ci > 0) mwait(B_M2, ci - 1, false);  // M2 of chunk ci - 1 has read the K/Q operand tile
             swait(S_M45, ci - 2);             // M4/M5 of chunk ci - 2 have read Kl and P (buffer par)
             if (Rb == 0 && hh == 0) {  // the pass over R: f_s, f_r; the factor that restores S^T after this chunk
                 float fs[4], fr[4];
