@@ -106,7 +106,7 @@ def test_decode_tokens_full_shape_sampled():
 
 def test_decode_tokens_unaligned_rows_take_the_other_kernel():
     """q/k/v/log alpha whose rows start 2 bytes past a 16-byte boundary (a contiguous view
-    one element into a buffer) cannot use the streaming kernel's 16-byte copies; the
+    one element into a buffer) cannot use the column-slice kernel's 16-byte copies; the
     call must take the per-unit kernel and still match the oracle."""
     B, n, H, num_slots = 5, 3, 2, 5
     inp = _tokens_inputs(B, n, H, 128, 128, "bf16", num_slots, seed=25)
