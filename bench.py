@@ -64,7 +64,7 @@ def decode_bytes_per_head_step(dk, dv, qkv_bytes):
 # Prefill: one launch on 2 x 8192 tokens x 32 heads (524,288 head-tokens).
 MEASURED_TRAFFIC = {
     "prefill_tc": {"source": "gated_delta_rule_126_b200/csrc/kda_prefill_tc.cu",
-                   "sha256": "3996fb87b0fb3d0042ded8eea954861425d151c04a823b707384073b9ea6cd67",
+                   "sha256": "2cefdd81b3f23a40798ee9431f8c194622fadb610fd0ecc148454e5ec3f58842",
                    "units": 2 * 8192 * 32, "dram_bytes": 673340416 + 120702976},
 }
 

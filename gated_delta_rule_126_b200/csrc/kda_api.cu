@@ -294,7 +294,11 @@ kda_status_t kda_prefill_gated(const void *q, const void *k, const void *v, kda_
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const kda_status_t pro = launch_prefill_prologue(a, st);
     if (pro != KDA_OK) return pro;
-    if (fused) return from_cuda(kda::launch_prefill_tc(a, st));
+    if (fused) {  // long sequences are split as in kda_prefill; the epilogue is per token
+        if (plan_split(a, cu_seqlens_host, workspace, workspace_bytes))
+            return from_cuda(launch_prefill_tc_split(a, cu_seqlens_host, st));
+        return from_cuda(kda::launch_prefill_tc(a, st));
+    }
     const cudaError_t err = kda::launch_prefill_simt(a, st);  // o into y, then the epilogue in place
     if (err != cudaSuccess) return KDA_ERR_CUDA;
     return from_cuda(kda::launch_gated_rmsnorm(a, st));

@@ -487,7 +487,7 @@ __global__ void __launch_bounds__(NT, 1)
             if (leader) ptx::bulk_wait_read0();  // the output tile's last store has read it
             if (ptx::named_barrier_or(BAR_S, NS, *s_abort != 0)) break;
             if (leader) {
-                if (kGated) load_g(s);  // over the output tile, read by this chunk's E4
+                if (kGated && !o_skip) load_g(s);  // over the output tile, read (and waited) by this chunk's E4
                 if (ci + 2 < nchunks && !v_zero) {
                     ptx::tma_prefetch_l2_3d(&maps.v, 0, h, s + 2 * C);
                     ptx::tma_prefetch_l2_3d(&maps.v, 64, h, s + 2 * C);
@@ -1353,6 +1353,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
     }
     if (!make_map(&maps.g, a.gate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.H, a.total_tokens))
         return cudaErrorInvalidValue;
+    if (a.split.num_units > 0 || a.split.num_seqs > 0) return launch_tc<true, true>(maps, a, stream);
     return launch_tc<true, false>(maps, a, stream);
 }
 

@@ -95,3 +95,19 @@ def test_batched_workload_sampled():
         worst_y = max(worst_y, rel_l2(host64(y[s:e, h]), y_ref))
         worst_S = max(worst_S, rel_l2(host64(S[n, h]), S_ref))
     assert worst_y <= TOL["bf16"]["o"] and worst_S <= TOL["bf16"]["S"], (worst_y, worst_S)
+
+
+def test_long_sequence_is_split():
+    """A 24,000-token sequence next to a 500-token one, 2 heads: the gated call cuts the long
+    sequence into segments as kda_prefill does (the segment passes that produce no outputs
+    load no gate tiles).  y and S_final against the oracles; S_final bit for bit against
+    kda_prefill, which takes the same state path."""
+    inp, gate, w = _inputs([24000, 500], 2, 128, 128, "bf16", seed=37)
+    y, S = _run(inp, gate, w)
+    o_p, S_p = kda_prefill(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["cu_seqlens"],
+                           inp["cu_seqlens_host"], S0=inp["S0"])
+    torch.cuda.synchronize()
+    assert torch.equal(S, S_p)
+    y_ref, S_ref = _oracle_all(inp, gate, w)
+    ey, eS = rel_l2(host64(y), y_ref), rel_l2(host64(S), S_ref)
+    assert ey <= TOL["bf16"]["o"] and eS <= TOL["bf16"]["S"], (ey, eS)
