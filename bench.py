@@ -84,14 +84,22 @@ def measured_traffic(kernel, units):
 
 
 def prefill_launches(seqlens, H, tc_path, sms=148):
-    """Kernel launches of one kda_prefill call: the ordering kernel and the prefill; on the
-    tensor-core path a long sequence is split (a sequence of at least 16,384 tokens with
-    2 L sms > 3 T H on a device with ``sms`` SMs), which adds the chain of start states
-    and a second prefill pass, plus the plain sequences' own launch when the split's
-    chain runs on its side stream."""
+    """Kernel launches of one kda_prefill call: the ordering kernel and the prefill.  On the
+    tensor-core path long sequences are split: up to m = min(T / 16384, 8, 2 sms / (3 H))
+    sequences of at least 16,384 tokens with 2 L sms > 3 T H (longest first), each cut
+    into nseg segments (the most with m H (2 nseg - 3) <= sms, within [3, 8], segments of
+    at least 4096 tokens).  That adds nseg - 2 launches of the start-state chain, a second
+    prefill pass and the plain sequences' own launch (the chain runs on its side stream)."""
     T = sum(seqlens)
-    split = tc_path and any(L >= 16384 and 2 * L * sms > 3 * T * H for L in seqlens)
-    return 5 if split else 2
+    if not tc_path:
+        return 2
+    m_max = min(T // 16384, 8, 2 * sms // (3 * max(H, 1)))
+    picked = sorted((L for L in seqlens if L >= 16384 and 2 * L * sms > 3 * T * H), reverse=True)[:m_max]
+    if not picked:
+        return 2
+    m = len(picked)
+    nseg = max(3, min((sms // (m * H) + 3) // 2, min(picked) // 4096, 8))
+    return nseg + 2
 
 
 def workload_config(w, world):

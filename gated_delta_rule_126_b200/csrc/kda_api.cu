@@ -1,6 +1,7 @@
 // C-ABI entry points of the KDA library: argument checks on the host, then
 // kernel launches on the caller's stream.  See include/kda.h for the contract.
 #include <cmath>
+#include <cstdint>
 #include <cstring>
 #include <mutex>
 
@@ -100,6 +101,12 @@ bool plan_split(kda::PrefillArgs &a, const int32_t *cu_host, void *workspace, si
         picked[m] = best;
     }
     if (m == 0) return false;
+    int64_t shortest = INT64_MAX;
+    for (int j = 0; j < m; ++j) {
+        const int64_t len = int64_t(cu_host[picked[j] + 1]) - cu_host[picked[j]];
+        shortest = len < shortest ? len : shortest;
+    }
+    a.split.nseg = kda::split_segments(m, a.H, sms, shortest);
     char *base = static_cast<char *>(workspace) + wl.split_offset;
     a.split.sstart = reinterpret_cast<float *>(base);
     a.split.lmat = reinterpret_cast<float *>(base + wl.split_array_bytes);
@@ -109,13 +116,13 @@ bool plan_split(kda::PrefillArgs &a, const int32_t *cu_host, void *workspace, si
     return true;
 }
 
-// Segment p of split sequence j: chunk-aligned thirds (the last one takes the rest).
-void segment_bounds(const int32_t *cu_host, int seq, int p, int32_t *b, int32_t *e) {
+// Segment p of nseg of a split sequence: chunk-aligned, equal (the last one takes the rest).
+void segment_bounds(const int32_t *cu_host, int seq, int p, int nseg, int32_t *b, int32_t *e) {
     const int32_t bos = cu_host[seq], eos = cu_host[seq + 1];
     const int32_t chunks = (eos - bos + 63) / 64;
-    const int32_t seg = (chunks + kda::kSplitP - 1) / kda::kSplitP * 64;
+    const int32_t seg = (chunks + nseg - 1) / nseg * 64;
     *b = bos + p * seg < eos ? bos + p * seg : eos;
-    *e = p == kda::kSplitP - 1 ? eos : (bos + (p + 1) * seg < eos ? bos + (p + 1) * seg : eos);
+    *e = p == nseg - 1 ? eos : (bos + (p + 1) * seg < eos ? bos + (p + 1) * seg : eos);
 }
 
 // A second, high-priority stream and two events per device for the split: it runs the
@@ -166,31 +173,32 @@ cudaError_t launch_prefill_tc_split(kda::PrefillArgs a, const int32_t *cu_host, 
         if (err == cudaSuccess) err = cudaStreamWaitEvent(side.stream, side.fork, 0);
         if (err != cudaSuccess) return err;
     }
+    const int P = a.split.nseg;
     int n = 0;
     for (int j = 0; j < a.split.num_seqs; ++j) {
         const int seq = a.split.seqs[j];
         int32_t b, e;
-        segment_bounds(cu_host, seq, 0, &b, &e);
-        a.split.units[n++] = SplitUnit{b, e, seq, UNIT_FIRST, j * kSplitP};
-        for (int p = 1; p + 1 < kSplitP; ++p) {
-            segment_bounds(cu_host, seq, p, &b, &e);
-            a.split.units[n++] = SplitUnit{b, e, seq, UNIT_LOCAL, j * kSplitP + p};
-            a.split.units[n++] = SplitUnit{b, e, seq, UNIT_HOMOG, j * kSplitP + p};
+        segment_bounds(cu_host, seq, 0, P, &b, &e);
+        a.split.units[n++] = SplitUnit{b, e, seq, UNIT_FIRST, j * P};
+        for (int p = 1; p + 1 < P; ++p) {
+            segment_bounds(cu_host, seq, p, P, &b, &e);
+            a.split.units[n++] = SplitUnit{b, e, seq, UNIT_LOCAL, j * P + p};
+            a.split.units[n++] = SplitUnit{b, e, seq, UNIT_HOMOG, j * P + p};
         }
     }
     a.split.num_units = n;
     a.split.plain_units = !forked;
     err = launch_prefill_tc(a, chain);
-    for (int p = 2; p < kSplitP && err == cudaSuccess; ++p) err = launch_split_combine(a, p, chain);
+    for (int p = 2; p < P && err == cudaSuccess; ++p) err = launch_split_combine(a, p, chain);
     if (err != cudaSuccess) return err;
     PrefillArgs passB = a;
     n = 0;
     for (int j = 0; j < a.split.num_seqs; ++j) {
         const int seq = a.split.seqs[j];
-        for (int p = 1; p < kSplitP; ++p) {
+        for (int p = 1; p < P; ++p) {
             int32_t b, e;
-            segment_bounds(cu_host, seq, p, &b, &e);
-            passB.split.units[n++] = SplitUnit{b, e, seq, p + 1 < kSplitP ? UNIT_CONT : UNIT_LAST, j * kSplitP + p};
+            segment_bounds(cu_host, seq, p, P, &b, &e);
+            passB.split.units[n++] = SplitUnit{b, e, seq, p + 1 < P ? UNIT_CONT : UNIT_LAST, j * P + p};
         }
     }
     passB.split.num_units = n;

@@ -13,25 +13,29 @@ namespace kda {
 //   [0, 256)            device status words (error flag + detail)
 //   [256, 256 + 4*N)    sequence order, longest first (int32)
 // ---- sequence split (tensor-core prefill).  A sequence much longer than the rest
-// would keep H SMs busy long after the others finish; it is cut into kSplitP
-// segments.  The recurrence is affine in the state, S_end = M S_start + L with
-// M (d_k x d_k) the state's transition through a segment and L its end state from a
-// zero start, so: pass A runs segment 0 from S0 and, for each middle segment, L (from
-// zero) and M (from the identity, v = 0) in parallel; a small kernel chains
-// S_start(p) = M(p-1) S_start(p-1) + L(p-1); pass B runs the other segments from
-// their true start states.
-constexpr int kSplitP = 3;
+// would keep H SMs busy long after the others finish; it is cut into nseg segments.
+// The recurrence is affine in the state, S_end = M S_start + L with M (d_k x d_k) the
+// state's transition through a segment and L its end state from a zero start, so:
+// pass A runs segment 0 from S0 and, for each middle segment, L (from zero) and M
+// (from the identity, v = 0) in parallel; a small kernel chains
+// S_start(p) = M(p-1) S_start(p-1) + L(p-1), p = 2 .. nseg - 1; pass B runs the other
+// segments from their true start states.  nseg is as large as pass A's units
+// (m H (2 nseg - 3) CTAs for m split sequences) fit on the device's SMs, between 3 and
+// kMaxSplitP, with segments of at least kSplitMinSeg tokens.
+constexpr int kMaxSplitP = 8;
 constexpr int kMaxSplitSeqs = 8;
 constexpr int kSplitMinLen = 16384;
-constexpr int kMaxSplitUnits = kMaxSplitSeqs * (2 * kSplitP - 3);
+constexpr int kSplitMinSeg = 4096;
+constexpr int kMaxSplitUnits = kMaxSplitSeqs * (2 * kMaxSplitP - 3);
 enum UnitMode : int32_t { UNIT_FIRST = 1, UNIT_LOCAL = 2, UNIT_HOMOG = 3, UNIT_CONT = 4, UNIT_LAST = 5 };
 struct SplitUnit {
     int32_t bos, eos, seq, mode;
-    int32_t slot;  // (split sequence j) * kSplitP + segment: the scratch state it reads or writes
+    int32_t slot;  // (split sequence j) * nseg + segment: the scratch state it reads or writes
 };
 struct SplitPlan {
     int num_units = 0;  // split units at the front of a launch
     int num_seqs = 0;   // split sequences, skipped where the plain ordering meets them
+    int nseg = 3;       // segments per split sequence
     bool plain_units = true;  // the launch also runs every plain (sequence, head) after the split units
     int32_t seqs[kMaxSplitSeqs] = {};
     SplitUnit units[kMaxSplitUnits] = {};
@@ -52,6 +56,17 @@ inline int split_max_seqs(int64_t total_tokens, int H, int sms) {
     return int(m < by_h ? m : by_h);
 }
 
+// Segments per split sequence when m sequences of at least `shortest` tokens are split:
+// the most for which pass A's m H (2 nseg - 3) units fit on `sms` SMs, within
+// [3, kMaxSplitP], and no shorter than kSplitMinSeg tokens a segment.
+inline int split_segments(int m, int H, int sms, int64_t shortest) {
+    const int64_t fit = (int64_t(sms) / (int64_t(m > 0 ? m : 1) * (H > 0 ? H : 1)) + 3) / 2;
+    const int64_t by_len = shortest / kSplitMinSeg;
+    int64_t p = fit < by_len ? fit : by_len;
+    p = p < kMaxSplitP ? p : kMaxSplitP;
+    return int(p > 3 ? p : 3);
+}
+
 struct WorkspaceLayout {
     static constexpr size_t kStatusBytes = 256;
     size_t order_offset = kStatusBytes;
@@ -70,7 +85,9 @@ inline WorkspaceLayout workspace_layout(int num_seqs, int64_t total_tokens = 0, 
     const int m = split_states ? split_max_seqs(total_tokens, H, device_sm_count()) : 0;
     if (m > 0) {
         L.split_offset = L.total;
-        L.split_array_bytes = size_t(m) * kSplitP * size_t(H) * 128 * 128 * sizeof(float);
+        // room for the most segments one split sequence can take on this device
+        const int pmax = split_segments(1, H, device_sm_count(), int64_t(1) << 40);
+        L.split_array_bytes = size_t(m) * pmax * size_t(H) * 128 * 128 * sizeof(float);
         L.total = align256(L.split_offset + 3 * L.split_array_bytes);
     }
     return L;

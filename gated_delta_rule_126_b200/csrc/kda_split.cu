@@ -17,7 +17,7 @@ __global__ void __launch_bounds__(256) split_combine_kernel(const SplitPlan plan
     extern __shared__ float s_in[];  // [128][128]
     const int j = blockIdx.x / H, h = blockIdx.x % H;
     const size_t D2 = size_t(D) * D;
-    const size_t prev = (size_t(j) * kSplitP + (p - 1)) * H + h, cur = (size_t(j) * kSplitP + p) * H + h;
+    const size_t prev = (size_t(j) * plan.nseg + (p - 1)) * H + h, cur = (size_t(j) * plan.nseg + p) * H + h;
     const float *M = plan.mmat + prev * D2, *L = plan.lmat + prev * D2, *Sin = plan.sstart + prev * D2;
     float *Sout = plan.sstart + cur * D2;
     for (int i = threadIdx.x; i < D * D / 4; i += blockDim.x)

@@ -35,7 +35,10 @@ def test_launch_count_follows_the_split_rule():
     # order + pass A + start-state chain + pass B + the plain sequences' own launch
     assert bench.prefill_launches(long, 32, True) == 5
     assert bench.prefill_launches(long, 32, False) == 2      # the CUDA-core path does not split
-    assert bench.prefill_launches([16384], 1, True) == 5     # 2 L 148 > 3 T H with T = L, H = 1
+    # 2 L 148 > 3 T H with T = L, H = 1; four 4096-token segments: order, pass A, two chain
+    # steps, pass B and the plain launch
+    assert bench.prefill_launches([16384], 1, True) == 6
+    assert bench.prefill_launches([60000, 300], 2, True) == 10  # eight segments (the most)
     assert bench.prefill_launches([16384], 1, True, sms=1) == 2  # 2 L > 3 L fails on one SM
     assert bench.prefill_launches([16383], 1, True) == 2     # below the minimum length
 

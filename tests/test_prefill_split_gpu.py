@@ -47,3 +47,23 @@ def test_split_agrees_with_the_unsplit_run():
     assert rel_l2(host64(o1), host64(o2)) <= TOL["bf16"]["o"]
     assert rel_l2(host64(S1), host64(S2)) <= TOL["bf16"]["S"]
     assert torch.equal(o1[33000:], o2[33000:]) and torch.equal(S1[1], S2[1])
+
+
+def test_few_heads_take_more_segments():
+    """60,000 + 300 tokens on 2 heads: pass A's units leave room for the most segments
+    (eight, one start-state chain step each past the second); against the oracle, and the
+    short sequence bit for bit against the unsplit run."""
+    inp = inputs.prefill_inputs([60000, 300], 2, 128, 128, "bf16", s0_std=0.1, seed=54, device=DEV)
+    o, S = _run(inp)
+    o2, S2 = _run(inp, workspace=_minimal_workspace(2))
+    torch.cuda.synchronize()
+    compare_full(inp, o, S, "bf16")
+    assert torch.equal(o[60000:], o2[60000:]) and torch.equal(S[1], S2[1])
+
+
+def test_two_sequences_share_the_segments():
+    """Two long sequences on one head, eight segments each, and a short one."""
+    inp = inputs.prefill_inputs([40000, 100, 36000], 1, 128, 128, "bf16", s0_std=0.1, seed=55, device=DEV)
+    o, S = _run(inp)
+    torch.cuda.synchronize()
+    compare_full(inp, o, S, "bf16")
