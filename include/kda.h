@@ -77,9 +77,10 @@ KDA_API int kda_version(void);
  * its arguments; returns 0 for arguments kda_prefill would reject.  On the
  * tensor-core shapes (bf16, d_k = d_v = 128, chunk 64) with at least 16,384 tokens
  * the size includes room for the start states of a sequence split (up to
- * 3 * 3 * m * H * 64 KiB, m <= 8 split sequences): a sequence much longer than the
- * rest is cut into three segments run in parallel, with the states between them
- * chained from the segments' transitions.  A workspace of only 256 + 4 num_seqs
+ * 3 * P * m * H * 64 KiB, m <= 8 split sequences, P <= 8 segments): a sequence much
+ * longer than the rest is cut into as many segments (3 to 8, at least 4096 tokens
+ * each) as the device's SMs can run side by side for H heads, with the states between
+ * them chained from the segments' transitions.  A workspace of only 256 + 4 num_seqs
  * bytes (rounded up to 256) is still accepted; the call then runs unsplit.
  */
 KDA_API size_t kda_prefill_workspace_size(int num_seqs, int64_t total_tokens, int H, int d_k,

@@ -22,7 +22,7 @@ def _minimal_workspace(n):
 
 def test_one_long_sequence_is_split():
     """40,000 + 300 + 1,000 tokens, 2 heads, non-zero S0: the long sequence is cut into
-    three segments; every output and final state is compared with the oracle."""
+    segments (eight at 2 heads); every output and final state is compared with the oracle."""
     inp = inputs.prefill_inputs([40000, 300, 1000], 2, 128, 128, "bf16", s0_std=0.1, seed=51, device=DEV)
     assert prefill_workspace_size(3, 41300, 2, 128, 128) > _minimal_workspace(3).numel()
     o, S = _run(inp)
