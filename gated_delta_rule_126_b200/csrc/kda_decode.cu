@@ -322,8 +322,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kSliceBlocksPerSm) decode
     float *raw_beta = raw_la + kGroup * kMaxD;
     const int H = a.H, n = a.n;
     const int nt0 = min(kGroup, n);
-    const int bitems = a.B * H * (kSlices / kWarpsPerBlock);  // (sequence, head, half): one per block step
-    auto slot_of = [&](int bi) { const int b = bi / (H * 2); return a.slot_idx ? a.slot_idx[b] : b; };
+    constexpr int kParts = kSlices / kWarpsPerBlock;          // blocks per (sequence, head)
+    const int bitems = a.B * H * kParts;  // (sequence, head, part): one per block step
+    auto slot_of = [&](int bi) { const int b = bi / (H * kParts); return a.slot_idx ? a.slot_idx[b] : b; };
     auto next_valid = [&](int bi) {  // the first block item >= bi of this block's stride whose slot is in the pool
         for (; bi < bitems; bi += gridDim.x) {
             const int sl = slot_of(bi);
@@ -331,9 +332,9 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kSliceBlocksPerSm) decode
         }
         return bitems;
     };
-    auto token = [&](int bi, int t) { return (size_t(bi / (H * 2)) * n + t) * H + (bi >> 1) % H; };  // [B, n, H, .] row
+    auto token = [&](int bi, int t) { return (size_t(bi / (H * kParts)) * n + t) * H + (bi / kParts) % H; };  // [B, n, H, .] row
     auto fetch = [&](int bi) {  // this warp's slice (16 quads a lane) and a quarter of the first token group
-        const int h = (bi >> 1) % H, cs = (bi & 1) * kWarpsPerBlock + warp;
+        const int h = (bi / kParts) % H, cs = (bi % kParts) * kWarpsPerBlock + warp;
         const float *src = a.S_pool + (size_t(slot_of(bi)) * H + h) * kMaxD * kMaxD + cs * kSliceCols;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -386,8 +387,8 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kSliceBlocksPerSm) decode
     int bi = next_valid(blockIdx.x);
     if (bi < bitems) fetch(bi);
     while (bi < bitems) {
-        const int h = (bi >> 1) % H;
-        const int cbase = ((bi & 1) * kWarpsPerBlock + warp) * kSliceCols;  // this warp's first value column
+        const int h = (bi / kParts) % H;
+        const int cbase = ((bi % kParts) * kWarpsPerBlock + warp) * kSliceCols;  // this warp's first value column
         ptx::cp_async_wait_all();
         __syncthreads();  // this unit's slices and first token group have landed
         float s[16][4];
