@@ -102,11 +102,15 @@ def test_split_path_strong_decay(scale):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_decode_strong_decay(dtype):
-    """Single-step and multi-token decode with strong decays and erased channels."""
-    B, H, d, n = 6, 2, 128, 5
+@pytest.mark.parametrize("scale,zero_frac", [(4.0, 0.02), (2.0, 0.0), (1.0, 0.0)])
+def test_decode_strong_decay(dtype, scale, zero_frac):
+    """Single-step and multi-token decode with strong decays and erased channels, at three
+    decay rates.  Nine tokens make two full staged groups of four and a single token in
+    the multi-token kernel."""
+    B, H, d, n = 6, 2, 128, 9
     dinp = inputs.decode_inputs(B, H, d, d, n, dtype, seed=63, device=DEV)
-    dinp["log_alpha"] = inputs.decay_log_alpha(n * B, H, d, 4.0, 0.02, seed=64, device=DEV).reshape(n, B, H, d)
+    dinp["log_alpha"] = inputs.decay_log_alpha(n * B, H, d, scale, zero_frac, seed=64,
+                                               device=DEV).reshape(n, B, H, d)
     S = dinp["S0"].clone()
     outs = [kda_decode_step(dinp["q"][t], dinp["k"][t], dinp["v"][t], dinp["log_alpha"][t], dinp["beta"][t], S)
             for t in range(n)]
