@@ -63,6 +63,30 @@ def compare_units(inp, o_gpu, S_gpu, units, dtype):
     return worst_o, worst_S
 
 
+def compare_heads(inp, o_gpu, S_gpu, heads, dtype):
+    """Rel-L2 over every sequence of the heads in ``heads``, as one tensor each for o
+    and S_final, against the oracle; asserts the tolerances.  The oracle runs one head
+    at a time (all sequences of that head in one call, threaded over the sequences), so
+    the host holds one head's inputs in fp64 at once."""
+    cu = inp["cu_seqlens_host"]
+    err = {"o": 0.0, "S": 0.0}
+    ref2 = {"o": 0.0, "S": 0.0}
+    for h in heads:
+        sl = lambda t: host64(t[:, h:h + 1])
+        S0 = None if inp["S0"] is None else host64(inp["S0"][:, h:h + 1])
+        o_ref, S_ref = oracle.prefill(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["log_alpha"]),
+                                      host64(inp["beta"][:, h:h + 1]), cu, S0=S0)
+        for key, x, r in (("o", host64(o_gpu[:, h:h + 1]), o_ref), ("S", host64(S_gpu[:, h:h + 1]), S_ref)):
+            err[key] += float(np.sum((x - r) ** 2))
+            ref2[key] += float(np.sum(r ** 2))
+        del o_ref, S_ref
+    worst = {key: (err[key] / ref2[key]) ** 0.5 for key in err}
+    tol = TOL[dtype]
+    assert worst["o"] <= tol["o"], f"o rel-L2 {worst['o']:.3e} > {tol['o']} over heads {heads}"
+    assert worst["S"] <= tol["S"], f"S rel-L2 {worst['S']:.3e} > {tol['S']} over heads {heads}"
+    return worst["o"], worst["S"]
+
+
 def compare_full(inp, o_gpu, S_gpu, dtype):
     """Whole-tensor rel-L2 against the oracle over every (sequence, head)."""
     o_ref, S_ref = oracle.prefill(host64(inp["q"]), host64(inp["k"]), host64(inp["v"]),

@@ -5,7 +5,7 @@ import torch
 
 import oracle
 from gated_delta_rule_126_b200 import inputs, kda_decode_step, kda_prefill
-from tests.kda_check import TOL, compare_full, compare_units, host64, rel_l2
+from tests.kda_check import TOL, compare_full, compare_heads, compare_units, host64, rel_l2
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -128,18 +128,20 @@ def test_batched_prefill_workload_sampled():
     assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
     units = [(0, 0), (7, 31), (3, 17), (5, 2)]
     compare_units(inp, o, S, units, "bf16")
+    compare_heads(inp, o, S, [0, 13, 31], "bf16")
 
 
 def test_longctx_varlen_workload_sampled():
     """1,048,576 packed tokens (one 524,288-token sequence + 64 shorter ones), H = 32,
-    d = 128, bf16: the long sequence on one head and short sequences on others."""
+    d = 128, bf16, in the launch configuration the bench times (the long sequence split
+    into segments): every sequence on heads 0, 13 and 31 against the oracle, as one
+    tensor per head subset."""
     w = inputs.WORKLOADS["longctx_varlen_prefill"]
     inp = inputs.workload_inputs(w, device=DEV)
     o, S = run(inp, chunk=w.chunk)
     torch.cuda.synchronize()
     assert torch.isfinite(o.float()).all() and torch.isfinite(S).all()
-    units = [(0, 5), (1, 0), (64, 31), (30, 12)]
-    compare_units(inp, o, S, units, "bf16")
+    compare_heads(inp, o, S, [0, 13, 31], "bf16")
 
 
 def test_long_sequence_last_is_scheduled_the_same():
