@@ -14,18 +14,21 @@
 //
 // Every value column j of the state evolves on its own given (k, alpha, beta): the
 // key-side operators act on rows only.  So the work is cut into slices of 16 value
-// columns, one 128-thread block per (sequence, head, slice), thread i owning key row
-// i of the slice; the reductions over value columns (dq, dk, dlog_alpha, dbeta) are
-// per-slice partial sums that a third kernel adds up.  The one reduction over key
-// rows on the recurrence's critical path (w in the forward sweep, de in the backward
-// sweep) is a transposed warp butterfly plus a 4-warp exchange in shared memory.
+// columns.  The reductions over value columns (dq, dk, dlog_alpha, dbeta) are
+// per-slice partial sums that a third kernel adds up.
 //
 // Three launches:
-//   1. states: the forward sweep, storing w_t for every token and the state before
-//      every 32nd token of each sequence (checkpoints); each 32-token block's alpha
-//      and k rows are staged in shared memory first;
-//   2. grads:  the backward sweep, 32-token blocks from the last: each block's alpha
-//      and k rows are staged in shared memory first (off the per-token critical path);
+//   1. states: the forward sweep, one warp per slice (lane (rs, cq) holding rows
+//      16 rs .. 16 rs + 15 and columns 4 cq .. 4 cq + 3), four slices of one (sequence,
+//      head) per block; its one reduction over key rows (w_t) is three shuffle rounds.
+//      It stores w_t for every token and the state before every 32nd token of each
+//      sequence (checkpoints); each 32-token block's alpha and k rows are staged in
+//      shared memory first;
+//   2. grads:  the backward sweep, one 128-thread block per (sequence, head, slice),
+//      thread i owning key row i of the slice; its reduction over key rows (de) is a
+//      transposed warp butterfly plus a 4-warp exchange in shared memory.  32-token
+//      blocks from the last: each block's alpha and k rows are staged in shared memory
+//      first (off the per-token critical path);
 //      the 4-token sub-blocks (last first) are replayed with the stored w (no reduction
 //      needed) from the block's checkpoint or, past the middle, from the state before
 //      the block's 16th token, their input states kept in shared memory;
@@ -144,42 +147,64 @@ __device__ __forceinline__ float4 *ck_slice(const BwdArgs &a, const Unit &u, int
     return a.ck + (((u.base + blk) * a.H + u.h) * a.nsl + u.sl) * (4 * kRows);
 }
 
+// The forward sweep, one warp per slice: lane (rs, cq) holds rows 16 rs .. 16 rs + 15 and
+// columns 4 cq .. 4 cq + 3 of the slice (64 registers), so the one sum over key rows a
+// token needs (P_t^T k_t) is 3 shuffle rounds over the 8 lanes that share a column quad,
+// and no token waits at a barrier.  A block's kSw warps take kSw slices of one (sequence,
+// head) and share each 32-token block's alpha and k rows, v and beta, staged in shared
+// memory behind one barrier per block.
+constexpr int kSw = 4;  // slices (warps) per block of the forward sweep
+static_assert(kSw * 32 == kRows, "the staging gives one key row to each thread");
+
 template <typename T>
-__global__ void __launch_bounds__(kRows) bwd_states_kernel(const BwdArgs a) {
-    __shared__ float4 red[2][4][4];
-    __shared__ float vs[kBlk][kCols];
+__global__ void __launch_bounds__(kSw * 32, 4) bwd_states_kernel(const BwdArgs a) {
+    __shared__ __align__(16) float vs[kBlk][kSw * kCols];
     __shared__ float bs[kBlk];
-    __shared__ float al_s[kBlk][kRows], k_s[kBlk][kRows];
-    const Unit u = unit_of(a);
+    __shared__ __align__(16) float al_s[kBlk][kRows];
+    __shared__ __align__(16) float k_s[kBlk][kRows];
     const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
+    const int rs = lane >> 2, cq = lane & 3;
+    const int nparts = (a.nsl + kSw - 1) / kSw;
+    const int part = int(blockIdx.x % unsigned(nparts));
+    const int64_t sh = blockIdx.x / unsigned(nparts);
     const int H = a.H, dk = a.dk, dv = a.dv, dvp = a.nsl * kCols;
-    const bool row = i < dk;
+    const int h = int(sh % H), s = int(sh / H);
+    const int sl = part * kSw + warp;  // this warp's slice; past the last one it only joins the barriers
+    const bool live = sl < a.nsl;
+    const int c0 = sl * kCols;
+    const int64_t cs = a.cu_seqlens[s], ce = a.cu_seqlens[s + 1], base = cs / kBlk + s;
+    const bool row = i < dk;  // the staging thread's key row
     const T *kp = static_cast<const T *>(a.k);
     const T *vp = static_cast<const T *>(a.v);
 
-    float S[kCols];
+    float S[16][4];
 #pragma unroll
-    for (int j = 0; j < kCols; ++j)
-        S[j] = (a.S0 && row && u.c0 + j < dv) ? a.S0[((int64_t(u.s) * H + u.h) * dk + i) * dv + u.c0 + j] : 0.f;
-    int rp = 0;
-    for (int64_t tb = u.cs; tb < u.ce; tb += kBlk) {
-        const int n = int(min(int64_t(kBlk), u.ce - tb));
-        float4 *ckp = ck_slice(a, u, (tb - u.cs) / kBlk);
+    for (int m = 0; m < 16; ++m)
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-            ckp[q4 * kRows + i] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
-        __syncthreads();  // the previous block's reads of the staged rows are done
-        for (int e = i; e < kBlk * kCols; e += kRows) {
-            const int tt = e / kCols, j = e % kCols;
-            vs[tt][j] = (tt < n && u.c0 + j < dv) ? ldf(vp + ((tb + tt) * H + u.h) * dv + u.c0 + j) : 0.f;
+        for (int c = 0; c < 4; ++c) {
+            const int r = 16 * rs + m, col = c0 + 4 * cq + c;
+            S[m][c] = (a.S0 && live && r < dk && col < dv) ? a.S0[((int64_t(s) * H + h) * dk + r) * dv + col] : 0.f;
         }
-        if (i < kBlk) bs[i] = i < n ? a.beta[(tb + i) * H + u.h] : 0.f;
-        for (int t8 = 0; t8 < kBlk; t8 += 8) {  // this row's alpha and k, eight tokens' loads at a time
+    for (int64_t tb = cs; tb < ce; tb += kBlk) {
+        const int n = int(min(int64_t(kBlk), ce - tb));
+        if (live) {  // the checkpoint: quad cq of row r at [cq][r]
+            float4 *ckp = a.ck + (((base + (tb - cs) / kBlk) * H + h) * a.nsl + sl) * (4 * kRows);
+#pragma unroll
+            for (int m = 0; m < 16; ++m)
+                ckp[cq * kRows + 16 * rs + m] = make_float4(S[m][0], S[m][1], S[m][2], S[m][3]);
+        }
+        __syncthreads();  // the previous block's reads of the staged rows are done
+        for (int e = i; e < kBlk * kSw * kCols; e += kRows) {
+            const int tt = e / (kSw * kCols), j = e % (kSw * kCols), col = part * kSw * kCols + j;
+            vs[tt][j] = (tt < n && col < dv) ? ldf(vp + ((tb + tt) * H + h) * dv + col) : 0.f;
+        }
+        if (i < kBlk) bs[i] = i < n ? a.beta[(tb + i) * H + h] : 0.f;
+        for (int t8 = 0; t8 < kBlk; t8 += 8) {  // this thread's row of alpha and k, eight tokens' loads at a time
             float la[8], kx[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 const bool in = row && t8 + j < n;
-                const int64_t r = ((tb + t8 + j) * H + u.h) * dk + i;
+                const int64_t r = ((tb + t8 + j) * H + h) * dk + i;
                 la[j] = in ? a.log_alpha[r] : 0.f;
                 kx[j] = in ? ldf(kp + r) : 0.f;
             }
@@ -187,26 +212,42 @@ __global__ void __launch_bounds__(kRows) bwd_states_kernel(const BwdArgs a) {
             for (int j = 0; j < 8; ++j) al_s[t8 + j][i] = expf(la[j]), k_s[t8 + j][i] = kx[j];
         }
         __syncthreads();
+        if (!live) continue;
         for (int tt = 0; tt < n; ++tt) {
-            const int64_t t = tb + tt;
-            const float al = al_s[tt][i];
-            const float kk = k_s[tt][i];
-            float c[kCols], ps[kCols];
+            const float4 *a4 = reinterpret_cast<const float4 *>(&al_s[tt][16 * rs]);
+            const float4 *k4 = reinterpret_cast<const float4 *>(&k_s[tt][16 * rs]);
+            float ps[4] = {0.f, 0.f, 0.f, 0.f}, kv[16];
 #pragma unroll
-            for (int j = 0; j < kCols; ++j) {
-                S[j] *= al;
-                c[j] = S[j] * kk;
+            for (int m4 = 0; m4 < 4; ++m4) {
+                const float4 al = a4[m4], kk = k4[m4];
+                const float alv[4] = {al.x, al.y, al.z, al.w};
+                kv[4 * m4] = kk.x;
+                kv[4 * m4 + 1] = kk.y;
+                kv[4 * m4 + 2] = kk.z;
+                kv[4 * m4 + 3] = kk.w;
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        S[4 * m4 + u][c] *= alv[u];
+                        ps[c] = fmaf(kv[4 * m4 + u], S[4 * m4 + u][c], ps[c]);
+                    }
             }
-            column_sums(c, red[rp], warp, lane, ps);  // ps = P_t^T k_t over this slice
-            rp ^= 1;
+            // P_t^T k_t: the sums over the 8 row groups (lane bits 2-4)
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) ps[c] += __shfl_xor_sync(0xffffffffu, ps[c], off);
             const float b = bs[tt];
-            float wv[kCols];
+            const float4 vv = *reinterpret_cast<const float4 *>(&vs[tt][warp * kCols + 4 * cq]);
+            const float wv[4] = {vv.x - ps[0], vv.y - ps[1], vv.z - ps[2], vv.w - ps[3]};
 #pragma unroll
-            for (int j = 0; j < kCols; ++j) {
-                wv[j] = vs[tt][j] - ps[j];
-                S[j] = fmaf(kk, b * wv[j], S[j]);
-            }
-            if (i < kCols) a.w[(t * H + u.h) * dvp + u.c0 + i] = pick(wv, i);
+            for (int m = 0; m < 16; ++m)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) S[m][c] = fmaf(kv[m], b * wv[c], S[m][c]);
+            if (rs == 0)
+                *reinterpret_cast<float4 *>(a.w + ((tb + tt) * H + h) * dvp + c0 + 4 * cq) =
+                    make_float4(wv[0], wv[1], wv[2], wv[3]);
         }
     }
 }
@@ -385,7 +426,8 @@ __global__ void __launch_bounds__(256) bwd_reduce_kernel(const BwdArgs a) {
 template <typename T>
 cudaError_t launch_backward_t(const BwdArgs &a, cudaStream_t st) {
     const unsigned grid = unsigned(int64_t(a.num_seqs) * a.H * a.nsl);
-    bwd_states_kernel<T><<<grid, kRows, 0, st>>>(a);
+    const unsigned sgrid = unsigned(int64_t(a.num_seqs) * a.H * ((a.nsl + kSw - 1) / kSw));
+    bwd_states_kernel<T><<<sgrid, kSw * 32, 0, st>>>(a);
     constexpr int dyn = kBlk * kRows * int(sizeof(float) + sizeof(T));
     cudaError_t err = cudaFuncSetAttribute(bwd_grads_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
     if (err != cudaSuccess) return err;
