@@ -19,8 +19,9 @@
 //
 // Three launches:
 //   1. states: the forward sweep, one warp per slice (lane (rs, cq) holding rows
-//      16 rs .. 16 rs + 15 and columns 4 cq .. 4 cq + 3), four slices of one (sequence,
-//      head) per block; its one reduction over key rows (w_t) is three shuffle rounds.
+//      32 g + 4 rs + u (g, u = 0..3) and columns 4 cq .. 4 cq + 3), four slices of one
+//      (sequence, head) per block; its one reduction over key rows (w_t) is three
+//      shuffle rounds.
 //      It stores w_t for every token and the state before every 32nd token of each
 //      sequence (checkpoints); each 32-token block's alpha and k rows are staged in
 //      shared memory first;
@@ -147,10 +148,11 @@ __device__ __forceinline__ float4 *ck_slice(const BwdArgs &a, const Unit &u, int
     return a.ck + (((u.base + blk) * a.H + u.h) * a.nsl + u.sl) * (4 * kRows);
 }
 
-// The forward sweep, one warp per slice: lane (rs, cq) holds rows 16 rs .. 16 rs + 15 and
-// columns 4 cq .. 4 cq + 3 of the slice (64 registers), so the one sum over key rows a
-// token needs (P_t^T k_t) is 3 shuffle rounds over the 8 lanes that share a column quad,
-// and no token waits at a barrier.  A block's kSw warps take kSw slices of one (sequence,
+// The forward sweep, one warp per slice: lane (rs, cq) holds columns 4 cq .. 4 cq + 3 of
+// rows 32 g + 4 rs + u (g, u = 0..3) of the slice (64 registers; S[4 g + u]), so the 8
+// row groups read consecutive 16-byte pieces of a staged row (no bank conflicts), and
+// the one sum over key rows a token needs (P_t^T k_t) is 3 shuffle rounds over the 8
+// lanes that share a column quad; no token waits at a barrier.  A block's kSw warps take kSw slices of one (sequence,
 // head) and share each 32-token block's alpha and k rows, v and beta, staged in shared
 // memory behind one barrier per block.
 constexpr int kSw = 4;  // slices (warps) per block of the forward sweep
@@ -182,7 +184,7 @@ __global__ void __launch_bounds__(kSw * 32, 4) bwd_states_kernel(const BwdArgs a
     for (int m = 0; m < 16; ++m)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            const int r = 16 * rs + m, col = c0 + 4 * cq + c;
+            const int r = 32 * (m >> 2) + 4 * rs + (m & 3), col = c0 + 4 * cq + c;
             S[m][c] = (a.S0 && live && r < dk && col < dv) ? a.S0[((int64_t(s) * H + h) * dk + r) * dv + col] : 0.f;
         }
     for (int64_t tb = cs; tb < ce; tb += kBlk) {
@@ -191,7 +193,7 @@ __global__ void __launch_bounds__(kSw * 32, 4) bwd_states_kernel(const BwdArgs a
             float4 *ckp = a.ck + (((base + (tb - cs) / kBlk) * H + h) * a.nsl + sl) * (4 * kRows);
 #pragma unroll
             for (int m = 0; m < 16; ++m)
-                ckp[cq * kRows + 16 * rs + m] = make_float4(S[m][0], S[m][1], S[m][2], S[m][3]);
+                ckp[cq * kRows + 32 * (m >> 2) + 4 * rs + (m & 3)] = make_float4(S[m][0], S[m][1], S[m][2], S[m][3]);
         }
         __syncthreads();  // the previous block's reads of the staged rows are done
         for (int e = i; e < kBlk * kSw * kCols; e += kRows) {
@@ -214,12 +216,12 @@ __global__ void __launch_bounds__(kSw * 32, 4) bwd_states_kernel(const BwdArgs a
         __syncthreads();
         if (!live) continue;
         for (int tt = 0; tt < n; ++tt) {
-            const float4 *a4 = reinterpret_cast<const float4 *>(&al_s[tt][16 * rs]);
-            const float4 *k4 = reinterpret_cast<const float4 *>(&k_s[tt][16 * rs]);
+            const float4 *a4 = reinterpret_cast<const float4 *>(&al_s[tt][4 * rs]);
+            const float4 *k4 = reinterpret_cast<const float4 *>(&k_s[tt][4 * rs]);
             float ps[4] = {0.f, 0.f, 0.f, 0.f}, kv[16];
 #pragma unroll
             for (int m4 = 0; m4 < 4; ++m4) {
-                const float4 al = a4[m4], kk = k4[m4];
+                const float4 al = a4[8 * m4], kk = k4[8 * m4];
                 const float alv[4] = {al.x, al.y, al.z, al.w};
                 kv[4 * m4] = kk.x;
                 kv[4 * m4 + 1] = kk.y;

@@ -258,10 +258,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_tokens_kernel(DecodeTokens
 // lanes that share the column), so no token waits at a block-wide barrier.  A block's
 // four warps take four slices of the same (sequence, head) and share the token vectors,
 // staged once per group of up to 4 tokens (alpha = e^{log alpha}, k, q, v in fp32,
-// q . k and beta).  Lane (rs, cq) holds rows 16 rs .. 16 rs + 15 and columns
-// 4 cq .. 4 cq + 3 of its slice (64 registers).  While a block computes one
-// (sequence, head), the next one's four slices and its first token group arrive in
-// shared memory by cp.async.
+// q . k and beta).  Lane (rs, cq) holds columns 4 cq .. 4 cq + 3 of rows
+// 32 g + 4 rs + u (g, u = 0..3) of its slice (64 registers), so that the 8 row groups
+// read consecutive 16-byte pieces of a staged vector (no bank conflicts).  While a
+// block computes one (sequence, head), the next one's four slices and its first token
+// group arrive in shared memory by cp.async.
 constexpr int kSliceCols = 16;
 constexpr int kSlices = kMaxD / kSliceCols;
 constexpr int kWarpsPerBlock = 4;                      // slices of one unit per block
@@ -275,10 +276,10 @@ template <typename T> constexpr uint32_t slice_smem() {
 }
 
 // byte offset of (row, 16-byte quad q) in a slice buffer: 64-byte rows, with the two
-// 64-byte halves of each 128-byte line swapped for rows 16..31 of every 32, so that the
-// two rows a quarter-warp reads at once (r and r + 16) fall in different banks
+// 64-byte halves of each 128-byte line swapped for rows 4..7 of every 8, so that the
+// two rows a quarter-warp reads at once (r and r + 4) fall in different banks
 __device__ __forceinline__ uint32_t slice_off(int row, int q) {
-    return ((uint32_t(row) * 64u) ^ (uint32_t((row >> 4) & 1) << 6)) + uint32_t(q) * 16u;
+    return ((uint32_t(row) * 64u) ^ (uint32_t((row >> 2) & 1) << 6)) + uint32_t(q) * 16u;
 }
 
 // four consecutive elements as floats
@@ -391,10 +392,12 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kSliceBlocksPerSm) decode
         const int cbase = ((bi % kParts) * kWarpsPerBlock + warp) * kSliceCols;  // this warp's first value column
         ptx::cp_async_wait_all();
         __syncthreads();  // this unit's slices and first token group have landed
+        // s[m] is row 32 (m / 4) + 4 rs + m % 4: the 8 row groups of a warp read consecutive
+        // 16-byte pieces of a staged token vector
         float s[16][4];
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
-            const float4 f = *reinterpret_cast<const float4 *>(buf + slice_off(16 * rs + m, cq));
+            const float4 f = *reinterpret_cast<const float4 *>(buf + slice_off(32 * (m >> 2) + 4 * rs + (m & 3), cq));
             s[m][0] = f.x;
             s[m][1] = f.y;
             s[m][2] = f.z;
@@ -418,14 +421,14 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kSliceBlocksPerSm) decode
                 __syncthreads();
             }
             for (int j = 0; j < nt; ++j) {
-                const float4 *a4 = reinterpret_cast<const float4 *>(st_a + j * kMaxD + 16 * rs);
-                const float4 *k4 = reinterpret_cast<const float4 *>(st_k + j * kMaxD + 16 * rs);
-                const float4 *q4 = reinterpret_cast<const float4 *>(st_q + j * kMaxD + 16 * rs);
+                const float4 *a4 = reinterpret_cast<const float4 *>(st_a + j * kMaxD + 4 * rs);
+                const float4 *k4 = reinterpret_cast<const float4 *>(st_k + j * kMaxD + 4 * rs);
+                const float4 *q4 = reinterpret_cast<const float4 *>(st_q + j * kMaxD + 4 * rs);
                 // DS = Diag(alpha) S; partial y = DS^T k, z = DS^T q over this lane's rows
                 float y[4] = {0.f, 0.f, 0.f, 0.f}, z[4] = {0.f, 0.f, 0.f, 0.f}, kv[16];
 #pragma unroll
                 for (int m4 = 0; m4 < 4; ++m4) {
-                    const float4 al = a4[m4], kk = k4[m4], qq = q4[m4];
+                    const float4 al = a4[8 * m4], kk = k4[8 * m4], qq = q4[8 * m4];
                     const float alv[4] = {al.x, al.y, al.z, al.w}, qv[4] = {qq.x, qq.y, qq.z, qq.w};
                     kv[4 * m4] = kk.x;
                     kv[4 * m4 + 1] = kk.y;
@@ -469,7 +472,7 @@ __global__ void __launch_bounds__(kWarpsPerBlock * 32, kSliceBlocksPerSm) decode
         float *dst = a.S_pool + (size_t(slot_of(bi)) * H + h) * kMaxD * kMaxD + cbase;
 #pragma unroll
         for (int m = 0; m < 16; ++m)
-            __stcs(reinterpret_cast<float4 *>(dst + (16 * rs + m) * kMaxD + 4 * cq),
+            __stcs(reinterpret_cast<float4 *>(dst + (32 * (m >> 2) + 4 * rs + (m & 3)) * kMaxD + 4 * cq),
                    make_float4(s[m][0], s[m][1], s[m][2], s[m][3]));
         bi = nbi;
     }
