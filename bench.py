@@ -514,8 +514,9 @@ def run_ours(args):
         del pin, pout
 
     # the backward pass (training) on the same batch: dO and dS_final given, gradients of
-    # q, k, v, log alpha, beta and S0 out; three launches (forward sweep with checkpoints,
-    # backward sweep, reduction over value-column slices), float32 on CUDA cores
+    # q, k, v, log alpha, beta and S0 out; two kernels (forward sweep with checkpoints,
+    # backward sweep adding its value-column slices' sums into the zeroed outputs) after
+    # four memsets, float32 on CUDA cores
     backward = None
     if not args.no_backward:
         dO, dSf = inputs.grad_inputs(T, N, w.H, w.dk, w.dv, w.dtype, seed=w.seed + 13 + 1000 * rank,
@@ -540,7 +541,7 @@ def run_ours(args):
         sm_mhz = float(peaks.get("sm_max_mhz", 1965.0))
         alu_peak = sms * 128 * 2 * sm_mhz * 1e6 / 1e12
         backward = {"value": weak_scaling_value(T, b_steps, b_el, world), "unit": UNIT,
-                    "ms_per_step": b_t * 1e3, "steps": b_steps, "gpu_launches_per_step": 3,
+                    "ms_per_step": b_t * 1e3, "steps": b_steps, "gpu_launches_per_step": 2,
                     "grads": "dq, dk, dv, dlog_alpha, dbeta, dS0 (float32)",
                     "roofline": {"bound": "alu", "achieved": b_tf, "peak": alu_peak, "unit": "TFLOP/s",
                                  "frac": b_tf / alu_peak, "alg_flops_per_launch": b_flops,

@@ -15,9 +15,11 @@
 // Every value column j of the state evolves on its own given (k, alpha, beta): the
 // key-side operators act on rows only.  So the work is cut into slices of 16 value
 // columns.  The reductions over value columns (dq, dk, dlog_alpha, dbeta) are
-// per-slice partial sums that a third kernel adds up.
+// per-slice sums, which the slices add into the zeroed outputs with fp32 atomics in
+// L2; the order in which the slices arrive is not fixed, so repeated calls can
+// differ in the last bits of those four gradients.
 //
-// Three launches:
+// Two launches, after the four outputs are zeroed:
 //   1. states: the forward sweep, one warp per slice (lane (rs, cq) holding rows
 //      32 g + 4 rs + u (g, u = 0..3) and columns 4 cq .. 4 cq + 3), four slices of one
 //      (sequence, head) per block; its one reduction over key rows (w_t) is three
@@ -32,10 +34,8 @@
 //      first (off the per-token critical path);
 //      the 4-token sub-blocks (last first) are replayed with the stored w (no reduction
 //      needed) from the block's checkpoint or, past the middle, from the state before
-//      the block's 16th token, their input states kept in shared memory;
-//   3. reduce: sums the slices' partial dq, dk, dlog_alpha and dbeta.
+//      the block's 16th token, their input states kept in shared memory.
 // CUDA cores in fp32 throughout; no tensor cores and no waits on other blocks.
-#include <algorithm>
 #include <cmath>
 
 #include "kda_internal.h"
@@ -57,13 +57,10 @@ struct BwdArgs {
     float *dq, *dk_out, *dv_out, *dla, *dbeta, *dS0;
     float4 *ck;            // [blk][H][nsl][4][128] float4: checkpoint slices, row-interleaved
     float *w;              // [T][H][nsl * 16]
-    float *pq, *pk, *pg;   // [nsl][T][H][dk] partial sums over a slice's columns
-    float *pb;             // [nsl][T][H]
 };
 
 struct BwdLayout {
-    size_t ck_offset = 0, w_offset = 0, p_offset = 0, pb_offset = 0, total = 0;
-    size_t p_bytes = 0;  // one of pq, pk, pg
+    size_t ck_offset = 0, w_offset = 0, total = 0;
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -76,10 +73,7 @@ BwdLayout bwd_layout(int num_seqs, int64_t T, int H, int dk, int dv) {
     const size_t nblk = size_t(T / kBlk) + size_t(num_seqs) + 1;
     L.ck_offset = kda::WorkspaceLayout::kStatusBytes;
     L.w_offset = L.ck_offset + align256(nblk * size_t(H) * nsl * 4 * kRows * sizeof(float4));
-    L.p_offset = L.w_offset + align256(size_t(T) * H * nsl * kCols * sizeof(float));
-    L.p_bytes = align256(size_t(nsl) * T * H * dk * sizeof(float));
-    L.pb_offset = L.p_offset + 3 * L.p_bytes;
-    L.total = L.pb_offset + align256(size_t(nsl) * T * H * sizeof(float));
+    L.total = L.w_offset + align256(size_t(T) * H * nsl * kCols * sizeof(float));
     return L;
 }
 
@@ -268,7 +262,6 @@ __global__ void __launch_bounds__(kRows, 3) bwd_grads_kernel(const BwdArgs a) {
     const Unit u = unit_of(a);
     const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
     const int H = a.H, dk = a.dk, dv = a.dv, dvp = a.nsl * kCols;
-    const int64_t nT = a.T;
     const bool row = i < dk;
     const T *qp = static_cast<const T *>(a.q);
     const T *kp = static_cast<const T *>(a.k);
@@ -388,13 +381,13 @@ __global__ void __launch_bounds__(kRows, 3) bwd_grads_kernel(const BwdArgs a) {
                     G[j] = al * dP;
                 }
                 if (i < kCols && u.c0 + i < dv) a.dv_out[(t * H + u.h) * dv + u.c0 + i] = b * pick(de, i);
-                const int64_t pr = ((int64_t(u.sl) * nT + t) * H + u.h) * dk + i;
+                const int64_t pr = (t * H + u.h) * dk + i;  // the 8 slices' sums meet in L2
                 if (row) {
-                    a.pq[pr] = pq;
-                    a.pk[pr] = dka + dkb;
-                    a.pg[pr] = dg;
+                    atomicAdd(a.dq + pr, pq);
+                    atomicAdd(a.dk_out + pr, dka + dkb);
+                    atomicAdd(a.dla + pr, dg);
                 }
-                if (i == 0) a.pb[(int64_t(u.sl) * nT + t) * H + u.h] = db;
+                if (i == 0) atomicAdd(a.dbeta + t * H + u.h, db);
             }
         }
     }
@@ -402,26 +395,6 @@ __global__ void __launch_bounds__(kRows, 3) bwd_grads_kernel(const BwdArgs a) {
 #pragma unroll
         for (int j = 0; j < kCols; ++j)
             if (u.c0 + j < dv) a.dS0[((int64_t(u.s) * H + u.h) * dk + i) * dv + u.c0 + j] = G[j];
-    }
-}
-
-__global__ void __launch_bounds__(256) bwd_reduce_kernel(const BwdArgs a) {
-    const int64_t n = a.T * a.H * a.dk, nb = a.T * a.H;
-    for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < n; e += int64_t(gridDim.x) * blockDim.x) {
-        float sq = 0.f, sk = 0.f, sg = 0.f;
-        for (int sl = 0; sl < a.nsl; ++sl) {
-            sq += a.pq[sl * n + e];
-            sk += a.pk[sl * n + e];
-            sg += a.pg[sl * n + e];
-        }
-        a.dq[e] = sq;
-        a.dk_out[e] = sk;
-        a.dla[e] = sg;
-        if (e < nb) {
-            float sb = 0.f;
-            for (int sl = 0; sl < a.nsl; ++sl) sb += a.pb[sl * nb + e];
-            a.dbeta[e] = sb;
-        }
     }
 }
 
@@ -433,12 +406,16 @@ cudaError_t launch_backward_t(const BwdArgs &a, cudaStream_t st) {
     constexpr int dyn = kBlk * kRows * int(sizeof(float) + sizeof(T));
     cudaError_t err = cudaFuncSetAttribute(bwd_grads_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
     if (err != cudaSuccess) return err;
-    bwd_grads_kernel<T><<<grid, kRows, dyn, st>>>(a);
     if (a.T > 0) {
-        const int64_t n = a.T * a.H * a.dk;
-        const unsigned rg = unsigned(std::min<int64_t>((n + 255) / 256, int64_t(kda::device_sm_count()) * 16));
-        bwd_reduce_kernel<<<rg, 256, 0, st>>>(a);
+        const size_t n = size_t(a.T) * a.H * a.dk * sizeof(float);
+        for (float *p : {a.dq, a.dk_out, a.dla}) {
+            err = cudaMemsetAsync(p, 0, n, st);
+            if (err != cudaSuccess) return err;
+        }
+        err = cudaMemsetAsync(a.dbeta, 0, size_t(a.T) * a.H * sizeof(float), st);
+        if (err != cudaSuccess) return err;
     }
+    bwd_grads_kernel<T><<<grid, kRows, dyn, st>>>(a);
     return cudaGetLastError();
 }
 
@@ -484,10 +461,6 @@ kda_status_t kda_backward(const void *q, const void *k, const void *v, kda_dtype
     char *base = static_cast<char *>(workspace);
     a.ck = reinterpret_cast<float4 *>(base + L.ck_offset);
     a.w = reinterpret_cast<float *>(base + L.w_offset);
-    a.pq = reinterpret_cast<float *>(base + L.p_offset);
-    a.pk = reinterpret_cast<float *>(base + L.p_offset + L.p_bytes);
-    a.pg = reinterpret_cast<float *>(base + L.p_offset + 2 * L.p_bytes);
-    a.pb = reinterpret_cast<float *>(base + L.pb_offset);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const cudaError_t e = qkv_dtype == KDA_DTYPE_F32 ? launch_backward_t<float>(a, st)
                                                      : launch_backward_t<__nv_bfloat16>(a, st);

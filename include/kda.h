@@ -277,8 +277,7 @@ KDA_API kda_status_t kda_workspace_status(const void *workspace, kda_stream_t st
  * these sizes (0 when they are unsupported).  About
  *   (T/32 + N + 1) * H * ceil(d_v/16) * 8 KiB      state checkpoints
  *   + T * H * 64 * ceil(d_v/16)                    per-token residuals w_t
- *   + T * H * ceil(d_v/16) * (12 d_k + 4)          per-slice partial sums
- * (plus 256 bytes and rounding), e.g. 7.8 GB for T = 16384, H = 32, d = 128.
+ * (plus 256 bytes and rounding), e.g. 1.35 GB for T = 16384, H = 32, d = 128.
  */
 KDA_API size_t kda_backward_workspace_size(int num_seqs, int64_t total_tokens, int H, int d_k, int d_v);
 
@@ -302,14 +301,17 @@ KDA_API size_t kda_backward_workspace_size(int num_seqs, int64_t total_tokens, i
  * All arithmetic is float32 on CUDA cores; the forward states are recomputed
  * inside the call (no forward output is needed).  Every output element is
  * written (gradients of empty sequences' tokens do not exist; dS0 of an empty
- * sequence is dS_final).
+ * sequence is dS_final).  dq, dk, dlog_alpha and dbeta are sums over slices of 16
+ * value channels, which the kernel adds into the zeroed outputs with float32
+ * atomics: the order of those additions is not fixed, so repeated calls can differ
+ * in the last bits of these four outputs (dv and dS0 are written once).
  *
  * Supported: 1 <= d_k, d_v <= 128, float32 or bfloat16 q/k/v/dO, num_seqs * H *
  * ceil(d_v / 16) < 2^31 (KDA_ERR_UNSUPPORTED otherwise); no alignment beyond each
  * type's own.  Workspace: kda_backward_workspace_size bytes,
- * 256-byte aligned (KDA_ERR_WORKSPACE otherwise).  Launches three kernels on
- * `stream`, asynchronously; the workspace and outputs must not be touched until
- * they finish.  Argument errors are reported before anything is queued.
+ * 256-byte aligned (KDA_ERR_WORKSPACE otherwise).  Queues four memsets of the
+ * outputs and two kernels on `stream`, asynchronously; the workspace and outputs
+ * must not be touched until they finish.  Argument errors are reported before anything is queued.
  */
 KDA_API kda_status_t kda_backward(const void *q, const void *k, const void *v, kda_dtype_t qkv_dtype,
                                   const float *log_alpha, const float *beta, const float *S0,

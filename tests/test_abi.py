@@ -171,9 +171,8 @@ def test_decode_tokens_rejects_bad_arguments(lib):
 def test_backward_workspace_size(lib):
     ws = lib.kda_backward_workspace_size
     n = ws(2, 16384, 32, 128, 128)
-    # checkpoints (16384/32 + 3 blocks x 32 heads x 8 slices x 8 KiB) + w (16384 x 32 x 128 x 4)
-    # + 3 partial arrays (8 x 16384 x 32 x 128 x 4) + dbeta partials (8 x 16384 x 32 x 4) + status
-    assert n == 256 + 515 * 32 * 8 * 8192 + 16384 * 32 * 128 * 4 + 3 * 8 * 16384 * 32 * 128 * 4 + 8 * 16384 * 32 * 4
+    # status + checkpoints (16384/32 + 3 blocks x 32 heads x 8 slices x 8 KiB) + w (16384 x 32 x 128 x 4)
+    assert n == 256 + 515 * 32 * 8 * 8192 + 16384 * 32 * 128 * 4
     assert ws(1, 10, 1, 7, 5) > 256
     assert ws(1, 10, 1, 129, 5) == 0 and ws(1, 10, 1, 7, 129) == 0
     assert ws(-1, 10, 1, 7, 5) == 0 and ws(1, -1, 1, 7, 5) == 0 and ws(1, 10, 0, 7, 5) == 0
