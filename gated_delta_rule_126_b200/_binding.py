@@ -386,7 +386,9 @@ def kda_backward(q, k, v, log_alpha, beta, cu_seqlens, dO, cu_seqlens_host=None,
 
     Inputs as ``kda_prefill`` plus dO [T,H,d_v] (dtype of q) and dS_final
     [N,H,d_k,d_v] f32 or None.  Returns a dict of float32 tensors dq, dk, dv,
-    dlog_alpha, dbeta and dS0 (None unless ``want_dS0``).
+    dlog_alpha, dbeta and dS0 (None unless ``want_dS0``).  dq, dk, dlog_alpha and
+    dbeta are added up from 16-channel slices with float32 atomics, so repeated
+    calls can differ in their last bits; dv and dS0 do not.
     """
     lib = load()
     T, H, dk = _dims(q, "q", 3)
