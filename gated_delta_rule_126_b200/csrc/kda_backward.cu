@@ -23,18 +23,17 @@
 //   1. states: the forward sweep, one warp per slice (lane (rs, cq) holding rows
 //      32 g + 4 rs + u (g, u = 0..3) and columns 4 cq .. 4 cq + 3), four slices of one
 //      (sequence, head) per block; its one reduction over key rows (w_t) is three
-//      shuffle rounds.
-//      It stores w_t for every token and the state before every 32nd token of each
-//      sequence (checkpoints); each 32-token block's alpha and k rows are staged in
-//      shared memory first;
-//   2. grads:  the backward sweep, one 128-thread block per (sequence, head, slice),
+//      shuffle rounds.  It stores w_t for every token and the state before every 32nd
+//      token of each sequence (checkpoints); each 32-token block's alpha and k rows are
+//      staged in shared memory first;
+//   2. grads: the backward sweep, one 128-thread block per (sequence, head, slice),
 //      thread i owning key row i of the slice; its reduction over key rows (de) is a
-//      transposed warp butterfly plus a 4-warp exchange in shared memory.  32-token
-//      blocks from the last: each block's alpha and k rows are staged in shared memory
-//      first (off the per-token critical path);
-//      the 4-token sub-blocks (last first) are replayed with the stored w (no reduction
-//      needed) from the block's checkpoint or, past the middle, from the state before
-//      the block's 16th token, their input states kept in shared memory.
+//      transposed warp butterfly plus a 4-warp exchange in shared memory.  It walks
+//      32-token blocks from the last; each block's alpha and k rows are staged in
+//      shared memory first (off the per-token critical path), and its 4-token
+//      sub-blocks (last first) are replayed with the stored w (no reduction needed)
+//      from the block's checkpoint or, past the middle, from the state before the
+//      block's 16th token, their input states kept in shared memory.
 // CUDA cores in fp32 throughout; no tensor cores and no waits on other blocks.
 #include <cmath>
 
