@@ -277,11 +277,22 @@ __global__ void __launch_bounds__(kRows, 3) bwd_grads_kernel(const BwdArgs a) {
         const int64_t t0 = u.cs + bi * kBlk;
         const int n = int(min(int64_t(kBlk), u.ce - t0));
         __syncthreads();  // the previous block's reads of ws, dos and bs are done
-        for (int e = i; e < kBlk * kCols; e += kRows) {
-            const int tt = e / kCols, j = e % kCols;
-            const bool in = tt < n;
-            ws[tt][j] = in ? a.w[((t0 + tt) * H + u.h) * dvp + u.c0 + j] : 0.f;
-            dos[tt][j] = (in && u.c0 + j < dv) ? ldf(dop + ((t0 + tt) * H + u.h) * dv + u.c0 + j) : 0.f;
+        {  // w and dO of the block's tokens: every load issued before any is stored
+            constexpr int kPer = kBlk * kCols / kRows;
+            float xw[kPer], xd[kPer];
+#pragma unroll
+            for (int c = 0; c < kPer; ++c) {
+                const int e = i + c * kRows, tt = e / kCols, j = e % kCols;
+                const bool in = tt < n;
+                xw[c] = in ? a.w[((t0 + tt) * H + u.h) * dvp + u.c0 + j] : 0.f;
+                xd[c] = (in && u.c0 + j < dv) ? ldf(dop + ((t0 + tt) * H + u.h) * dv + u.c0 + j) : 0.f;
+            }
+#pragma unroll
+            for (int c = 0; c < kPer; ++c) {
+                const int e = i + c * kRows;
+                ws[e / kCols][e % kCols] = xw[c];
+                dos[e / kCols][e % kCols] = xd[c];
+            }
         }
         if (i < kBlk) bs[i] = i < n ? a.beta[(t0 + i) * H + u.h] : 0.f;
         for (int t8 = 0; t8 < kBlk; t8 += 8) {  // this thread's row, eight tokens' loads at a time (no barrier needed)
